@@ -1,0 +1,189 @@
+/*
+ * moe.h -- C ABI of libmoe_b200.so: one Mixture-of-Experts layer on one B200.
+ *
+ * The layer follows the tutorial page "Expert Parallelism" (learning-materials,
+ * inference engineering IX.05):
+ *   §1 "What is it?"        each layer has E expert FFNs; each token is routed
+ *                           to k of them; experts are placed on GPUs in
+ *                           contiguous blocks (GPU 0 holds experts 0-15, ...).
+ *   §4 "The All-to-All"     DISPATCH: sort tokens by destination expert (and so
+ *                           by destination GPU), count per GPU, exchange, so each
+ *                           GPU holds a contiguous set of tokens per expert.
+ *                           COMPUTE: one grouped GEMM over all experts.
+ *                           COMBINE: results back in the original order and a
+ *                           weighted sum of each token's k expert outputs.
+ *   §5 "Load imbalance"     the imbalance of the most loaded GPU against the
+ *                           ideal (max / mean), worked example 140/64.
+ * On this one GPU the "GPUs" of the page are R logical expert-parallel ranks:
+ * rank r owns experts [r*E/R, (r+1)*E/R). Nothing crosses a GPU boundary; the
+ * exchange becomes the rank-major row layout of the permuted buffer.
+ *
+ * Conventions for every entry point
+ *  - All tensor pointers are DEVICE pointers, row-major and contiguous, owned
+ *    by the caller. bf16 tensors are passed as uint16_t bit patterns
+ *    (moe_bf16_t). bf16 tensors must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Every call
+ *    is asynchronous on that stream, except moe_get_status which synchronises it.
+ *  - `ws` is a caller-owned device workspace of at least moe_workspace_bytes()
+ *    bytes, 256-byte aligned. Its first 256 bytes hold the device status word;
+ *    clear it once with moe_clear_status before first use. The library
+ *    allocates nothing and keeps no per-call state outside `ws`.
+ *  - Shapes are validated on the host before anything is launched; an invalid
+ *    argument returns MOE_ERR_INVALID_ARG (or MOE_ERR_UNSUPPORTED for a shape
+ *    the kernels do not tile) and launches nothing.
+ *  - Data-dependent problems found on the device (a NaN logit, an expert index
+ *    out of range, a bounded wait that ran out) never trap: they OR bits into
+ *    the status word (MOE_DEV_*), read with moe_get_status.
+ *  - Calls that share a workspace must be ordered on one stream.
+ *
+ * Supported shapes: 0 <= T, T*k <= 2^27; 1 <= E <= 256; 1 <= k <= min(E, 8);
+ * 1 <= R, E % R == 0; d % 128 == 0 and f % 128 == 0 (128 <= d, f <= 65536);
+ * n_shared in {0, 1}.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16_t; /* bfloat16 bit pattern */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null pointer, bad shape, misaligned buffer */
+  MOE_ERR_UNSUPPORTED = 2, /* shape outside what the kernels tile (see above) */
+  MOE_ERR_WORKSPACE = 3,   /* ws too small or misaligned */
+  MOE_ERR_CUDA = 4         /* a CUDA runtime call or launch failed */
+} moe_status_t;
+
+/* device status bits (OR-ed by kernels into the workspace status word) */
+#define MOE_DEV_NAN_LOGIT 1u      /* a NaN router logit (ordered as -inf) */
+#define MOE_DEV_BOUNDS 2u         /* an expert index or row index out of range (entry skipped) */
+#define MOE_DEV_TIMEOUT 4u        /* a bounded pipeline wait ran out; the kernel returned early */
+#define MOE_DEV_COUNT_MISMATCH 8u /* expert_offsets inconsistent with the shape */
+
+typedef struct moe_shape {
+  int32_t T;        /* tokens in the batch */
+  int32_t d;        /* model width (expert input/output size) */
+  int32_t E;        /* routed experts */
+  int32_t k;        /* experts per token (top-k) */
+  int32_t f;        /* expert FFN width (SwiGLU hidden size) */
+  int32_t R;        /* logical expert-parallel ranks */
+  int32_t n_shared; /* shared experts applied to every token: 0 or 1 */
+} moe_shape_t;
+
+/* Bytes of workspace the entry points need for `shape` (0 if the shape is invalid). */
+size_t moe_workspace_bytes(const moe_shape_t* shape);
+
+/* Zero the device status word in `ws` (asynchronous on `stream`). */
+moe_status_t moe_clear_status(void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, then copy the device status word (MOE_DEV_* bits) to *bits.
+ * The word is left as it is (clear it with moe_clear_status). */
+moe_status_t moe_get_status(const void* ws, size_t ws_bytes, uint32_t* bits, void* stream);
+
+/* Router: top-k selection and gates.
+ * Page "Expert Parallelism" §1 (each token is routed to k of E experts) and §4
+ * ("Router output: for each token, which expert(s) it needs").
+ *   logits    [T, E] fp32 in
+ *   topk_idx  [T, k] int32 out: the k experts with the largest logits, in
+ *             descending logit order; equal logits go to the lower expert index
+ *             (-0.0 == +0.0); a NaN logit orders as -inf and sets MOE_DEV_NAN_LOGIT.
+ *   topk_gate [T, k] fp32 out: softmax over the k selected logits,
+ *             g_j = exp(l_j - l_0) / sum_i exp(l_i - l_0) (1/k if l_0 = -inf). */
+moe_status_t moe_route(const moe_shape_t* shape, const float* logits, int32_t* topk_idx, float* topk_gate,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* Dispatch: per-expert histogram, exclusive scan and stable permute.
+ * Page "Expert Parallelism" §4 DISPATCH steps 1-4 and §5 (max/mean imbalance).
+ * Assignment a = t*k + j (token t, choice j) goes to expert e = topk_idx[a].
+ *   x              [T, d] bf16 in
+ *   topk_idx       [T, k] int32 in (values in [0, E); others set MOE_DEV_BOUNDS and are skipped)
+ *   expert_counts  [E]   int32 out: assignments per expert
+ *   expert_offsets [E+1] int32 out: exclusive scan of expert_counts, [E] = total
+ *   rank_counts    [R]   int32 out: assignments per logical rank
+ *   rank_offsets   [R+1] int32 out: expert_offsets[r*E/R]
+ *   row_src        [T*k] int32 out: permuted row p holds assignment row_src[p]
+ *   assign_row     [T*k] int32 out: inverse, assignment a sits at row assign_row[a]
+ *   x_perm         [T*k, d] bf16 out: x_perm[assign_row[a]] = x[a / k]; rows are
+ *                  expert-contiguous (expert e at [off[e], off[e+1])), so rank-major;
+ *                  inside an expert, rows keep assignment order (stable).
+ *   imbalance      [2] fp32 out: [0] = max_r rank_counts[r] / mean (= *R / (T*k)),
+ *                  [1] = max_e expert_counts[e] / mean; {1, 1} when T = 0. */
+moe_status_t moe_dispatch(const moe_shape_t* shape, const moe_bf16_t* x, const int32_t* topk_idx,
+                          int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
+                          int32_t* rank_offsets, int32_t* row_src, int32_t* assign_row, moe_bf16_t* x_perm,
+                          float* imbalance, void* ws, size_t ws_bytes, void* stream);
+
+/* Expert FFN: one grouped GEMM over all experts (tcgen05 tensor cores).
+ * Page "Expert Parallelism" §4 COMPUTE ("each expert processes its tokens ...
+ * many different-shaped GEMMs in one launch") and §1 (E expert FFNs); the FFN is
+ * SwiGLU: y = W2_e (silu(W_gate,e x) * (W_up,e x)), silu(a) = a / (1 + e^-a).
+ *   x_perm         [T*k, d] bf16 in (from moe_dispatch)
+ *   expert_offsets [E+1]    int32 in (from moe_dispatch)
+ *   w13            [E, 2f, d] bf16 in: rows [0, f) = W_gate, [f, 2f) = W_up (K = d contiguous)
+ *   w2             [E, d, f]  bf16 in (K = f contiguous)
+ *   x              [T, d] bf16 in, used by the shared expert (may be NULL if n_shared = 0)
+ *   w13s [2f, d], w2s [d, f] bf16 in: shared expert (NULL if n_shared = 0)
+ *   y_perm         [T*k, d] bf16 out: row p = FFN of expert(p) applied to x_perm[p]
+ *   y_shared       [T, d]   bf16 out: shared FFN of x (NULL if n_shared = 0)
+ * fp32 accumulation; the hidden activation is rounded to bf16 between the GEMMs. */
+moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_bf16_t* x_perm, const int32_t* expert_offsets,
+                            const moe_bf16_t* w13, const moe_bf16_t* w2, const moe_bf16_t* x,
+                            const moe_bf16_t* w13s, const moe_bf16_t* w2s, moe_bf16_t* y_perm,
+                            moe_bf16_t* y_shared, void* ws, size_t ws_bytes, void* stream);
+
+/* Combine: un-permute and gate-weighted sum, back in original token order.
+ * Page "Expert Parallelism" §4 COMBINE.
+ *   out[t] = sum_{j<k} topk_gate[t,j] * y_perm[assign_row[t*k+j]] (+ y_shared[t])
+ *   fp32 accumulation in j order, one bf16 rounding at the end.
+ *   y_perm [T*k, d] bf16 in, assign_row [T*k] int32 in, topk_gate [T, k] fp32 in,
+ *   y_shared [T, d] bf16 in (NULL: no shared term), out [T, d] bf16 out. */
+moe_status_t moe_combine(const moe_shape_t* shape, const moe_bf16_t* y_perm, const int32_t* assign_row,
+                         const float* topk_gate, const moe_bf16_t* y_shared, moe_bf16_t* out, void* ws,
+                         size_t ws_bytes, void* stream);
+
+/* All buffers of one layer call (device pointers; see the steps above). */
+typedef struct moe_layer_buffers {
+  const float* logits;       /* [T, E]  in */
+  const moe_bf16_t* x;       /* [T, d]  in */
+  const moe_bf16_t* w13;     /* [E, 2f, d] in */
+  const moe_bf16_t* w2;      /* [E, d, f]  in */
+  const moe_bf16_t* w13s;    /* [2f, d] in (NULL if n_shared = 0) */
+  const moe_bf16_t* w2s;     /* [d, f]  in (NULL if n_shared = 0) */
+  int32_t* topk_idx;         /* [T, k]  out */
+  float* topk_gate;          /* [T, k]  out */
+  int32_t* expert_counts;    /* [E]     out */
+  int32_t* expert_offsets;   /* [E+1]   out */
+  int32_t* rank_counts;      /* [R]     out */
+  int32_t* rank_offsets;     /* [R+1]   out */
+  int32_t* row_src;          /* [T*k]   out */
+  int32_t* assign_row;       /* [T*k]   out */
+  moe_bf16_t* x_perm;        /* [T*k, d] out */
+  float* imbalance;          /* [2]     out */
+  moe_bf16_t* y_perm;        /* [T*k, d] out */
+  moe_bf16_t* y_shared;      /* [T, d]  out (NULL if n_shared = 0) */
+  moe_bf16_t* out;           /* [T, d]  out */
+} moe_layer_buffers_t;
+
+/* The whole layer: route -> dispatch -> expert FFN -> combine, on one stream,
+ * with no host synchronisation (the grouped GEMM reads the per-expert row
+ * counts on the device). Same results as the four calls in sequence. */
+moe_status_t moe_layer(const moe_shape_t* shape, const moe_layer_buffers_t* buf, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* moe_status_string(moe_status_t status);
+
+/* Text of the last CUDA error seen by this thread in a library call ("" if none). */
+const char* moe_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */
