@@ -1,0 +1,371 @@
+"""Benchmark of the MoE layer (route -> dispatch -> grouped SwiGLU FFN -> combine).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
+
+One step = one pass of the whole layer over one batch of synthetic inputs that
+are already resident in HBM (weights, x, logits), timed with CUDA events on the
+launching stream. L2 is flushed (a 512 MiB write) between steps, outside the
+step's events. Prints one JSON line (rank 0).
+
+N > 1 runs under torchrun: each rank runs an independent replica of the layer on
+its own batch (the path has no cross-GPU exchange on one node here; "replicas
+only"), value = all ranks' tokens / the max over ranks of the timed region.
+
+--impl reference times the CPU oracle (the plain fp64 definition of the layer)
+on the host cores, on a bounded sample of tokens of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s (route+dispatch+grouped GEMM+combine); % of roofline"
+UNIT = "tokens/s"
+DEFAULT_CONFIG = "mixtral_prefill"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work (bytes / flops) of one layer call, from the actual routing
+# ---------------------------------------------------------------------------
+
+def algorithmic(wl, counts):
+    """Per-step algorithmic bytes and flops of each step (padding excluded)."""
+    T, d, E, k, f, A = wl.T, wl.d, wl.E, wl.k, wl.f, wl.T * wl.k
+    n_act = int(sum(1 for c in counts if c > 0))
+    sh = wl.n_shared
+    w = {}
+    w["route"] = dict(bytes=T * E * 4 + A * 8, flops=0)
+    w["dispatch"] = dict(bytes=T * d * 2 + A * d * 2 + A * 8, flops=0)
+    w["gate_up"] = dict(flops=4 * A * d * f + sh * 4 * T * d * f,
+                        bytes=(n_act + sh) * 2 * d * f * 2 + A * d * 2 + sh * T * d * 2)
+    w["down"] = dict(flops=2 * A * d * f + sh * 2 * T * d * f,
+                     bytes=(n_act + sh) * d * f * 2 + A * d * 2 + sh * T * d * 2)
+    w["combine"] = dict(bytes=A * d * 2 + A * 8 + T * d * 2 + sh * T * d * 2, flops=0)
+    w["_n_act"] = n_act
+    return w
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            j = json.load(fh)
+        return dict(hbm=float(j["hbm_gbs"]), bf16=float(j["bf16_tflops"]),
+                    bf16_sustained=float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# reference arm / CPU baseline: the oracle on a bounded sample
+# ---------------------------------------------------------------------------
+
+def oracle_sample_run(wl, n_tokens: int, weights=None):
+    """Time the oracle's whole layer on the first n_tokens tokens of the batch."""
+    import numpy as np
+    import moe_synth
+    import oracle
+    toks = np.arange(n_tokens)
+    x = moe_synth.host_x(wl, toks)
+    lg = moe_synth.host_logits(wl, toks)
+    if weights is None:
+        weights = (moe_synth.host_w13(wl), moe_synth.host_w2(wl),
+                   moe_synth.host_w13s(wl) if wl.n_shared else None, moe_synth.host_w2s(wl) if wl.n_shared else None)
+    w13, w2, w13s, w2s = weights
+    t0 = time.perf_counter()
+    oracle.layer(x, lg, w13, w2, wl.k, wl.R, w13s, w2s)
+    return time.perf_counter() - t0, weights
+
+
+def cpu_baseline(wl, budget_s: float = 20.0):
+    import moe_synth  # noqa: F401
+    n = 4
+    dt, weights = oracle_sample_run(wl, n)
+    # grow the sample to roughly the time budget (the oracle's cost is about linear in tokens)
+    if dt < budget_s / 4:
+        n = int(min(wl.T, max(n, n * (budget_s * 0.6) / max(dt, 1e-3))))
+        dt, _ = oracle_sample_run(wl, n, weights)
+    return dict(value=n / dt, unit=UNIT, cores=os.cpu_count(), kind="oracle",
+                sample=f"oracle layer (fp64, OpenMP over rows) on the first {n} of {wl.T} tokens of {wl.name}, "
+                       f"all {wl.E} experts' weights resident; {dt:.1f} s")
+
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return
+    steps = []
+    weights = None
+    n = 4
+    dt, weights = oracle_sample_run(wl, n)
+    # size one step to ~ (2 min) / (K + W)
+    per_step = max(2.0, 120.0 / max(1, args.steps + args.warmup))
+    n = int(min(wl.T, max(1, n * per_step / max(dt, 1e-3))))
+    for _ in range(args.warmup):
+        oracle_sample_run(wl, n, weights)
+    for _ in range(args.steps):
+        dt, _ = oracle_sample_run(wl, n, weights)
+        steps.append(dt)
+    tot = sum(steps)
+    value = n * len(steps) / tot
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)",
+        "config": {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "f": wl.f, "R": wl.R,
+                   "n_shared": wl.n_shared, "sample_tokens_per_step": n},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": f"oracle layer on the first {n} of {wl.T} tokens per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def run_gpu(args, wl, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import combine_warp_top_expert_b200 as moe
+    import moe_synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl_r = wl.with_(seed=wl.seed + rank)  # each replica: its own batch
+    shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, n_shared=wl.n_shared)
+    dv = moe_synth.device_inputs(wl_r, device=dev)
+    layer = moe.MoELayer(shape, dv["w13"], dv["w2"], dv.get("w13s"), dv.get("w2s"), device=dev)
+    o = layer.outs
+    ws = layer.ws
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    def step(evs):
+        evs[0].record(stream)
+        moe.moe_route(shape, dv["logits"], o["topk_idx"], o["topk_gate"], ws, stream)
+        evs[1].record(stream)
+        moe.moe_dispatch(shape, dv["x"], o["topk_idx"], o["expert_counts"], o["expert_offsets"], o["rank_counts"],
+                         o["rank_offsets"], o["row_src"], o["assign_row"], o["x_perm"], o["imbalance"], ws, stream)
+        evs[2].record(stream)
+        moe.moe_expert_gate_up(shape, o["x_perm"], o["expert_offsets"], dv["w13"], dv["x"], dv.get("w13s"), ws,
+                               stream)
+        evs[3].record(stream)
+        moe.moe_expert_down(shape, o["expert_offsets"], dv["w2"], dv.get("w2s"), o["y_perm"], o.get("y_shared"), ws,
+                            stream)
+        evs[4].record(stream)
+        moe.moe_combine(shape, o["y_perm"], o["assign_row"], o["topk_gate"], o.get("y_shared"), o["out"], ws,
+                        stream)
+        evs[5].record(stream)
+
+    names = ("route", "dispatch", "gate_up", "down", "combine")
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(6)]  # noqa: E731
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(mk())
+    torch.cuda.synchronize(dev)
+    status = moe.get_status(ws)
+    counts = o["expert_counts"].cpu().numpy().tolist()
+    imbalance = o["imbalance"].cpu().numpy().tolist()
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    events = [mk() for _ in range(args.steps)]
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    smi_index = vis.split(",")[local_rank].strip() if vis else str(local_rank)
+    with ClockSampler(smi_index) as clocks:
+        region0 = torch.cuda.Event(enable_timing=True)
+        region1 = torch.cuda.Event(enable_timing=True)
+        region0.record(stream)
+        for i in range(args.steps):
+            flush.zero_()
+            step(events[i])
+        region1.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    per_step = [ev[0].elapsed_time(ev[5]) for ev in events]
+    per_kernel = {n: [ev[j].elapsed_time(ev[j + 1]) for ev in events] for j, n in enumerate(names)}
+    step_ms = sum(per_step)
+    t = torch.tensor([step_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    value = world * wl.T * args.steps / (max_ms / 1e3)
+
+    # e2e through the public API with host buffers (pinned), copies inside the timed region
+    x_h = dv["x"].cpu().pin_memory()
+    lg_h = dv["logits"].cpu().pin_memory()
+    out_h = torch.empty((wl.T, wl.d), dtype=torch.bfloat16).pin_memory()
+    for _ in range(max(1, args.warmup)):
+        layer.forward_host(lg_h, x_h, out_h, stream)
+    torch.cuda.synchronize(dev)
+    e2e_times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        layer.forward_host(lg_h, x_h, out_h, stream)
+        stream.synchronize()
+        e2e_times.append(time.perf_counter() - t0)
+    te = torch.tensor([sum(e2e_times)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = world * wl.T * args.steps / float(te.item())
+
+    if rank != 0:
+        return
+    peaks = load_peaks()
+    work = algorithmic(wl, counts)
+    kern_ms = {n: statistics.mean(v) for n, v in per_kernel.items()}
+    # roofline of each step and of the layer
+    roof = {}
+    t_roof = 0.0
+    for n in names:
+        b = work[n]["bytes"] / (peaks["hbm"] * 1e9)
+        fl = work[n]["flops"] / (peaks["bf16"] * 1e12)
+        t_roof += max(b, fl)
+        roof[n] = dict(ms=kern_ms[n], bound="tensor" if fl > b else "hbm",
+                       achieved=(work[n]["flops"] / (kern_ms[n] * 1e-3) / 1e12) if fl > b
+                       else (work[n]["bytes"] / (kern_ms[n] * 1e-3) / 1e9),
+                       frac=max(b, fl) / (kern_ms[n] * 1e-3))
+    dom = max(("gate_up", "down"), key=lambda n: kern_ms[n])
+    d = roof[dom]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded generator; weights random-init, no checkpoints)",
+        "config": {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "f": wl.f, "R": wl.R,
+                   "n_shared": wl.n_shared, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed between steps (512 MiB write, outside the step's events)",
+                   "experts_active": work["_n_act"], "imbalance_rank_expert": imbalance,
+                   "layer_roofline_frac": t_roof / (max_ms / args.steps / 1e3),
+                   "per_step_ms": {n: round(v, 4) for n, v in kern_ms.items()},
+                   "per_step_roofline": {n: {"bound": r["bound"], "frac": round(r["frac"], 4)} for n, r in roof.items()},
+                   "peaks": peaks, "device_status": status},
+        "roofline": {"kernel": f"moe_expert_{dom}", "bound": d["bound"], "achieved": d["achieved"],
+                     "peak": peaks["bf16"] if d["bound"] == "tensor" else peaks["hbm"],
+                     "unit": "TFLOP/s" if d["bound"] == "tensor" else "GB/s",
+                     "frac": d["achieved"] / (peaks["bf16"] if d["bound"] == "tensor" else peaks["hbm"]),
+                     "peak_kind": f"{peaks['source']} burst", "traffic": None},
+        "clocks": clocks.summary(),
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(x_h.numel() * 2 + lg_h.numel() * 4),
+                "d2h_bytes_per_step": int(out_h.numel() * 2)},
+        "gpu_launches": args.steps * (1 + (3 if wl.T > 0 else 1) + 1 + 1 + 1),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    import moe_synth
+    wl = moe_synth.workload(args.config)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, wl, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_gpu(args, wl, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,330 @@
+"""B200-native MoE layer: route -> dispatch -> grouped SwiGLU FFN -> combine.
+
+Thin ctypes binding of libmoe_b200.so (the C ABI in include/moe.h). The
+functions keep the ABI's names and only marshal arguments: every step runs in
+the library's CUDA kernels. PyTorch supplies device memory and streams.
+There is no CPU fallback: if the library is missing or cannot be loaded,
+every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+from . import build as _build
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA = range(5)
+MOE_DEV_NAN_LOGIT, MOE_DEV_BOUNDS, MOE_DEV_TIMEOUT, MOE_DEV_COUNT_MISMATCH = 1, 2, 4, 8
+
+LIB_PATH = _build.LIB_PATH
+
+ABI_FUNCTIONS = (
+    "moe_workspace_bytes", "moe_clear_status", "moe_get_status", "moe_route", "moe_dispatch", "moe_expert_ffn",
+    "moe_combine", "moe_layer", "moe_status_string", "moe_last_cuda_error", "moe_set_wait_timeout_ns",
+    "moe_expert_gate_up", "moe_expert_down",
+)
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} failed: {msg}")
+        self.code = code
+
+
+class moe_shape_t(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("T", "d", "E", "k", "f", "R", "n_shared")]
+
+
+class moe_layer_buffers_t(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "logits", "x", "w13", "w2", "w13s", "w2s", "topk_idx", "topk_gate", "expert_counts", "expert_offsets",
+        "rank_counts", "rank_offsets", "row_src", "assign_row", "x_perm", "imbalance", "y_perm", "y_shared", "out")]
+
+
+_lib = None
+
+
+def load(build_if_missing: bool = True) -> ctypes.CDLL:
+    """Load the in-tree libmoe_b200.so (building it with nvcc if absent)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH) or (build_if_missing and not _build.up_to_date()):
+        if not build_if_missing:
+            raise RuntimeError(f"libmoe_b200.so not built ({LIB_PATH}); run python -m combine_warp_top_expert_b200.build")
+        _build.build()
+    L = ctypes.CDLL(LIB_PATH)
+    vp, sz, st = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    shp = ctypes.POINTER(moe_shape_t)
+    L.moe_workspace_bytes.restype = sz
+    L.moe_workspace_bytes.argtypes = [shp]
+    L.moe_clear_status.restype = st
+    L.moe_clear_status.argtypes = [vp, sz, vp]
+    L.moe_get_status.restype = st
+    L.moe_get_status.argtypes = [vp, sz, ctypes.POINTER(ctypes.c_uint32), vp]
+    L.moe_route.restype = st
+    L.moe_route.argtypes = [shp, vp, vp, vp, vp, sz, vp]
+    L.moe_dispatch.restype = st
+    L.moe_dispatch.argtypes = [shp] + [vp] * 10 + [vp, sz, vp]
+    L.moe_expert_ffn.restype = st
+    L.moe_expert_ffn.argtypes = [shp] + [vp] * 9 + [vp, sz, vp]
+    L.moe_expert_gate_up.restype = st
+    L.moe_expert_gate_up.argtypes = [shp] + [vp] * 5 + [vp, sz, vp]
+    L.moe_expert_down.restype = st
+    L.moe_expert_down.argtypes = [shp] + [vp] * 5 + [vp, sz, vp]
+    L.moe_combine.restype = st
+    L.moe_combine.argtypes = [shp] + [vp] * 5 + [vp, sz, vp]
+    L.moe_layer.restype = st
+    L.moe_layer.argtypes = [shp, ctypes.POINTER(moe_layer_buffers_t), vp, sz, vp]
+    L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_status_string.argtypes = [st]
+    L.moe_last_cuda_error.restype = ctypes.c_char_p
+    L.moe_last_cuda_error.argtypes = []
+    L.moe_set_wait_timeout_ns.restype = ctypes.c_uint64
+    L.moe_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+    _lib = L
+    return L
+
+
+def _check(fn: str, code: int):
+    if code != MOE_OK:
+        L = load()
+        msg = L.moe_status_string(code).decode()
+        if code == MOE_ERR_CUDA:
+            msg += " (" + L.moe_last_cuda_error().decode() + ")"
+        raise MoEError(fn, code, msg)
+
+
+@dataclass(frozen=True)
+class Shape:
+    T: int
+    d: int
+    E: int
+    k: int
+    f: int
+    R: int
+    n_shared: int = 0
+
+    @property
+    def A(self) -> int:
+        return self.T * self.k
+
+    def c(self) -> moe_shape_t:
+        return moe_shape_t(self.T, self.d, self.E, self.k, self.f, self.R, self.n_shared)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _dev(t, dtype, shape, name):
+    import torch
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def workspace_bytes(shape: Shape) -> int:
+    n = load().moe_workspace_bytes(ctypes.byref(shape.c()))
+    if n == 0:
+        raise MoEError("moe_workspace_bytes", MOE_ERR_INVALID_ARG, "invalid shape")
+    return n
+
+
+def new_workspace(shape: Shape, device="cuda"):
+    """A zeroed device workspace (the status word starts clear)."""
+    import torch
+    return torch.zeros(workspace_bytes(shape), dtype=torch.uint8, device=device)
+
+
+def clear_status(ws, stream=None):
+    _check("moe_clear_status", load().moe_clear_status(_ptr(ws), ws.numel(), _stream(stream)))
+
+
+def get_status(ws, stream=None) -> int:
+    bits = ctypes.c_uint32(0)
+    _check("moe_get_status", load().moe_get_status(_ptr(ws), ws.numel(), ctypes.byref(bits), _stream(stream)))
+    return bits.value
+
+
+def set_wait_timeout_ns(ns: int) -> int:
+    return load().moe_set_wait_timeout_ns(ns)
+
+
+def moe_route(shape: Shape, logits, topk_idx, topk_gate, ws, stream=None):
+    import torch
+    _dev(logits, torch.float32, (shape.T, shape.E), "logits")
+    _dev(topk_idx, torch.int32, (shape.T, shape.k), "topk_idx")
+    _dev(topk_gate, torch.float32, (shape.T, shape.k), "topk_gate")
+    _check("moe_route", load().moe_route(ctypes.byref(shape.c()), _ptr(logits), _ptr(topk_idx), _ptr(topk_gate),
+                                         _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_dispatch(shape: Shape, x, topk_idx, expert_counts, expert_offsets, rank_counts, rank_offsets, row_src,
+                 assign_row, x_perm, imbalance, ws, stream=None):
+    import torch
+    i32, bf = torch.int32, torch.bfloat16
+    _dev(x, bf, (shape.T, shape.d), "x")
+    _dev(topk_idx, i32, (shape.T, shape.k), "topk_idx")
+    _dev(expert_counts, i32, (shape.E,), "expert_counts")
+    _dev(expert_offsets, i32, (shape.E + 1,), "expert_offsets")
+    _dev(rank_counts, i32, (shape.R,), "rank_counts")
+    _dev(rank_offsets, i32, (shape.R + 1,), "rank_offsets")
+    _dev(row_src, i32, (shape.A,), "row_src")
+    _dev(assign_row, i32, (shape.A,), "assign_row")
+    _dev(x_perm, bf, (shape.A, shape.d), "x_perm")
+    _dev(imbalance, torch.float32, (2,), "imbalance")
+    _check("moe_dispatch", load().moe_dispatch(
+        ctypes.byref(shape.c()), _ptr(x), _ptr(topk_idx), _ptr(expert_counts), _ptr(expert_offsets),
+        _ptr(rank_counts), _ptr(rank_offsets), _ptr(row_src), _ptr(assign_row), _ptr(x_perm), _ptr(imbalance),
+        _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_expert_ffn(shape: Shape, x_perm, expert_offsets, w13, w2, x, w13s, w2s, y_perm, y_shared, ws, stream=None):
+    import torch
+    bf = torch.bfloat16
+    _dev(x_perm, bf, (shape.A, shape.d), "x_perm")
+    _dev(expert_offsets, torch.int32, (shape.E + 1,), "expert_offsets")
+    _dev(w13, bf, (shape.E, 2 * shape.f, shape.d), "w13")
+    _dev(w2, bf, (shape.E, shape.d, shape.f), "w2")
+    _dev(y_perm, bf, (shape.A, shape.d), "y_perm")
+    if shape.n_shared:
+        _dev(x, bf, (shape.T, shape.d), "x")
+        _dev(w13s, bf, (2 * shape.f, shape.d), "w13s")
+        _dev(w2s, bf, (shape.d, shape.f), "w2s")
+        _dev(y_shared, bf, (shape.T, shape.d), "y_shared")
+    _check("moe_expert_ffn", load().moe_expert_ffn(
+        ctypes.byref(shape.c()), _ptr(x_perm), _ptr(expert_offsets), _ptr(w13), _ptr(w2), _ptr(x), _ptr(w13s),
+        _ptr(w2s), _ptr(y_perm), _ptr(y_shared), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_expert_gate_up(shape: Shape, x_perm, expert_offsets, w13, x, w13s, ws, stream=None):
+    """GEMM1 + SwiGLU into the workspace (first half of moe_expert_ffn)."""
+    import torch
+    bf = torch.bfloat16
+    _dev(x_perm, bf, (shape.A, shape.d), "x_perm")
+    _dev(expert_offsets, torch.int32, (shape.E + 1,), "expert_offsets")
+    _dev(w13, bf, (shape.E, 2 * shape.f, shape.d), "w13")
+    if shape.n_shared:
+        _dev(x, bf, (shape.T, shape.d), "x")
+        _dev(w13s, bf, (2 * shape.f, shape.d), "w13s")
+    _check("moe_expert_gate_up", load().moe_expert_gate_up(
+        ctypes.byref(shape.c()), _ptr(x_perm), _ptr(expert_offsets), _ptr(w13), _ptr(x), _ptr(w13s), _ptr(ws),
+        ws.numel(), _stream(stream)))
+
+
+def moe_expert_down(shape: Shape, expert_offsets, w2, w2s, y_perm, y_shared, ws, stream=None):
+    """GEMM2 from the workspace's hidden rows (second half of moe_expert_ffn)."""
+    import torch
+    bf = torch.bfloat16
+    _dev(expert_offsets, torch.int32, (shape.E + 1,), "expert_offsets")
+    _dev(w2, bf, (shape.E, shape.d, shape.f), "w2")
+    _dev(y_perm, bf, (shape.A, shape.d), "y_perm")
+    if shape.n_shared:
+        _dev(w2s, bf, (shape.d, shape.f), "w2s")
+        _dev(y_shared, bf, (shape.T, shape.d), "y_shared")
+    _check("moe_expert_down", load().moe_expert_down(
+        ctypes.byref(shape.c()), _ptr(expert_offsets), _ptr(w2), _ptr(w2s), _ptr(y_perm), _ptr(y_shared), _ptr(ws),
+        ws.numel(), _stream(stream)))
+
+
+def moe_combine(shape: Shape, y_perm, assign_row, topk_gate, y_shared, out, ws, stream=None):
+    import torch
+    bf = torch.bfloat16
+    _dev(y_perm, bf, (shape.A, shape.d), "y_perm")
+    _dev(assign_row, torch.int32, (shape.A,), "assign_row")
+    _dev(topk_gate, torch.float32, (shape.T, shape.k), "topk_gate")
+    _dev(y_shared, bf, (shape.T, shape.d), "y_shared")
+    _dev(out, bf, (shape.T, shape.d), "out")
+    _check("moe_combine", load().moe_combine(
+        ctypes.byref(shape.c()), _ptr(y_perm), _ptr(assign_row), _ptr(topk_gate), _ptr(y_shared), _ptr(out),
+        _ptr(ws), ws.numel(), _stream(stream)))
+
+
+_LAYER_OUTPUTS = ("topk_idx", "topk_gate", "expert_counts", "expert_offsets", "rank_counts", "rank_offsets",
+                  "row_src", "assign_row", "x_perm", "imbalance", "y_perm", "y_shared", "out")
+
+
+def alloc_layer_outputs(shape: Shape, device="cuda") -> dict:
+    """Device buffers for every output of moe_layer."""
+    import torch
+    i32, f32, bf = torch.int32, torch.float32, torch.bfloat16
+    T, k, E, R, d, A = shape.T, shape.k, shape.E, shape.R, shape.d, shape.A
+    o = dict(
+        topk_idx=torch.empty((T, k), dtype=i32, device=device),
+        topk_gate=torch.empty((T, k), dtype=f32, device=device),
+        expert_counts=torch.empty((E,), dtype=i32, device=device),
+        expert_offsets=torch.empty((E + 1,), dtype=i32, device=device),
+        rank_counts=torch.empty((R,), dtype=i32, device=device),
+        rank_offsets=torch.empty((R + 1,), dtype=i32, device=device),
+        row_src=torch.empty((A,), dtype=i32, device=device),
+        assign_row=torch.empty((A,), dtype=i32, device=device),
+        x_perm=torch.empty((A, d), dtype=bf, device=device),
+        imbalance=torch.empty((2,), dtype=f32, device=device),
+        y_perm=torch.empty((A, d), dtype=bf, device=device),
+        y_shared=torch.empty((T, d), dtype=bf, device=device) if shape.n_shared else None,
+        out=torch.empty((T, d), dtype=bf, device=device),
+    )
+    return o
+
+
+def moe_layer(shape: Shape, logits, x, w13, w2, w13s, w2s, outs: dict, ws, stream=None):
+    """The whole layer on one stream, writing every buffer of `outs` (see alloc_layer_outputs)."""
+    import torch
+    bf = torch.bfloat16
+    _dev(logits, torch.float32, (shape.T, shape.E), "logits")
+    _dev(x, bf, (shape.T, shape.d), "x")
+    _dev(w13, bf, (shape.E, 2 * shape.f, shape.d), "w13")
+    _dev(w2, bf, (shape.E, shape.d, shape.f), "w2")
+    if shape.n_shared:
+        _dev(w13s, bf, (2 * shape.f, shape.d), "w13s")
+        _dev(w2s, bf, (shape.d, shape.f), "w2s")
+    b = moe_layer_buffers_t(_ptr(logits), _ptr(x), _ptr(w13), _ptr(w2), _ptr(w13s), _ptr(w2s),
+                            *(_ptr(outs[n]) for n in _LAYER_OUTPUTS))
+    _check("moe_layer", load().moe_layer(ctypes.byref(shape.c()), ctypes.byref(b), _ptr(ws), ws.numel(),
+                                         _stream(stream)))
+    return outs
+
+
+class MoELayer:
+    """Weights resident on the device plus a reusable workspace and output set."""
+
+    def __init__(self, shape: Shape, w13, w2, w13s=None, w2s=None, device="cuda"):
+        self.shape = shape
+        self.w13, self.w2, self.w13s, self.w2s = w13, w2, w13s, w2s
+        self.ws = new_workspace(shape, device)
+        self.outs = alloc_layer_outputs(shape, device)
+
+    def __call__(self, logits, x, stream=None) -> dict:
+        return moe_layer(self.shape, logits, x, self.w13, self.w2, self.w13s, self.w2s, self.outs, self.ws, stream)
+
+    def forward_host(self, logits_host, x_host, out_host, stream=None):
+        """End-to-end call with HOST tensors (pinned for async copies): copies the
+        step's inputs to the device, runs the layer, copies `out` back."""
+        import torch
+        s = stream or torch.cuda.current_stream()
+        with torch.cuda.stream(s):
+            if not hasattr(self, "_in_logits"):
+                self._in_logits = torch.empty(logits_host.shape, dtype=logits_host.dtype, device=self.ws.device)
+                self._in_x = torch.empty(x_host.shape, dtype=x_host.dtype, device=self.ws.device)
+            self._in_logits.copy_(logits_host, non_blocking=True)
+            self._in_x.copy_(x_host, non_blocking=True)
+            self(self._in_logits, self._in_x, s)
+            out_host.copy_(self.outs["out"], non_blocking=True)
+        return out_host

@@ -1,0 +1,256 @@
+/*
+ * moe_abi.cu -- the C ABI of libmoe_b200.so (declared in include/moe.h):
+ * argument validation, workspace layout, and the launch sequence of each entry
+ * point. Every check runs on the host before anything is launched; the library
+ * allocates no memory and holds no per-call state.
+ */
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+std::atomic<uint64_t> g_wait_timeout_ns{kDefaultWaitNs};
+
+moe_status_t cuda_fail(cudaError_t e) {
+  std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+  return MOE_ERR_CUDA;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+moe_status_t validate_shape(const moe_shape_t* s) {
+  if (!s) return MOE_ERR_INVALID_ARG;
+  if (s->T < 0 || s->d < 1 || s->f < 1 || s->E < 1 || s->k < 1 || s->R < 1) return MOE_ERR_INVALID_ARG;
+  if (s->k > s->E || s->E % s->R != 0 || (s->n_shared != 0 && s->n_shared != 1)) return MOE_ERR_INVALID_ARG;
+  if (s->E > kMaxE || s->k > kMaxK) return MOE_ERR_UNSUPPORTED;
+  if ((int64_t)s->T * s->k > (int64_t(1) << 27)) return MOE_ERR_UNSUPPORTED;
+  if (s->d % 128 != 0 || s->f % 128 != 0 || s->d > 65536 || s->f > 65536) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status_t check_ws(const moe_shape_t& s, const void* ws, size_t ws_bytes) {
+  if (!ws || !aligned(ws, 256)) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < ws_layout(s).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+}  // namespace
+
+WsLayout ws_layout(const moe_shape_t& s) {
+  WsLayout L;
+  L.A = (int64_t)s.T * s.k;
+  L.tok_per_chunk = s.k > 0 ? (kChunkAssign / s.k > 0 ? kChunkAssign / s.k : 1) : 1;
+  L.n_chunks = (s.T + L.tok_per_chunk - 1) / L.tok_per_chunk;
+  L.mt_routed_max = L.A / kTileM + (L.A < s.E ? L.A : s.E);
+  L.h_rows = (int64_t)kTileM * (L.mt_routed_max + (s.n_shared ? (s.T + kTileM - 1) / kTileM : 0));
+  size_t off = 256;
+  L.status = 0;
+  L.chunk = off;
+  off = round_up(off + (size_t)L.n_chunks * s.E * sizeof(int32_t), 256);
+  L.local_rank = off;
+  off = round_up(off + (size_t)L.A * sizeof(int32_t), 256);
+  L.h = off;
+  off = round_up(off + (size_t)L.h_rows * s.f * sizeof(uint16_t), 256);
+  L.total = off;
+  return L;
+}
+
+int num_sms() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) dev = 0;
+  const int slot = dev < 64 ? dev : 63;
+  int n = cache[slot].load(std::memory_order_relaxed);
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[slot].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
+uint64_t wait_timeout_ns() { return g_wait_timeout_ns.load(std::memory_order_relaxed); }
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_bytes(const moe_shape_t* shape) {
+  if (validate_shape(shape) != MOE_OK) return 0;
+  return ws_layout(*shape).total;
+}
+
+moe_status_t moe_clear_status(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || !aligned(ws, 256) || ws_bytes < 256) return MOE_ERR_WORKSPACE;
+  const cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(uint32_t), (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+moe_status_t moe_get_status(const void* ws, size_t ws_bytes, uint32_t* bits, void* stream) {
+  if (!bits) return MOE_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256) || ws_bytes < 256) return MOE_ERR_WORKSPACE;
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaMemcpy(bits, ws, sizeof(uint32_t), cudaMemcpyDeviceToHost);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+moe_status_t moe_route(const moe_shape_t* shape, const float* logits, int32_t* topk_idx, float* topk_gate, void* ws,
+                       size_t ws_bytes, void* stream) {
+  moe_status_t st = validate_shape(shape);
+  if (st != MOE_OK) return st;
+  if (shape->T > 0 && (!logits || !topk_idx || !topk_gate)) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
+  const WsLayout L = ws_layout(*shape);
+  const cudaError_t e = launch_route(logits, topk_idx, topk_gate, shape->T, shape->E, shape->k,
+                                     reinterpret_cast<uint32_t*>((uint8_t*)ws + L.status), (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+moe_status_t moe_dispatch(const moe_shape_t* shape, const moe_bf16_t* x, const int32_t* topk_idx,
+                          int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
+                          int32_t* rank_offsets, int32_t* row_src, int32_t* assign_row, moe_bf16_t* x_perm,
+                          float* imbalance, void* ws, size_t ws_bytes, void* stream) {
+  moe_status_t st = validate_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!expert_counts || !expert_offsets || !rank_counts || !rank_offsets || !imbalance) return MOE_ERR_INVALID_ARG;
+  if (shape->T > 0 && (!x || !topk_idx || !row_src || !assign_row || !x_perm)) return MOE_ERR_INVALID_ARG;
+  if (shape->T > 0 && (!aligned(x, 16) || !aligned(x_perm, 16))) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
+  const WsLayout L = ws_layout(*shape);
+  const cudaError_t e = launch_dispatch(*shape, L, (uint8_t*)ws, x, topk_idx, expert_counts, expert_offsets,
+                                        rank_counts, rank_offsets, row_src, assign_row, x_perm, imbalance,
+                                        (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_bf16_t* x_perm, const int32_t* expert_offsets,
+                            const moe_bf16_t* w13, const moe_bf16_t* w2, const moe_bf16_t* x,
+                            const moe_bf16_t* w13s, const moe_bf16_t* w2s, moe_bf16_t* y_perm,
+                            moe_bf16_t* y_shared, void* ws, size_t ws_bytes, void* stream) {
+  moe_status_t st = validate_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!expert_offsets || !w13 || !w2) return MOE_ERR_INVALID_ARG;
+  if (shape->T > 0 && (!x_perm || !y_perm)) return MOE_ERR_INVALID_ARG;
+  if (shape->n_shared && shape->T > 0 && (!x || !w13s || !w2s || !y_shared)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(w13, 16) || !aligned(w2, 16) || (x_perm && !aligned(x_perm, 16)) || (y_perm && !aligned(y_perm, 16)))
+    return MOE_ERR_INVALID_ARG;
+  if (shape->n_shared && ((x && !aligned(x, 16)) || (w13s && !aligned(w13s, 16)) || (w2s && !aligned(w2s, 16)) ||
+                          (y_shared && !aligned(y_shared, 16))))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
+  const WsLayout L = ws_layout(*shape);
+  cudaError_t e = launch_gate_up(*shape, L, (uint8_t*)ws, x_perm, expert_offsets, w13, x, w13s, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = launch_down(*shape, L, (uint8_t*)ws, expert_offsets, w2, w2s, y_perm, shape->n_shared ? y_shared : nullptr,
+                  (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+moe_status_t moe_expert_gate_up(const moe_shape_t* shape, const moe_bf16_t* x_perm, const int32_t* expert_offsets,
+                                const moe_bf16_t* w13, const moe_bf16_t* x, const moe_bf16_t* w13s, void* ws,
+                                size_t ws_bytes, void* stream) {
+  moe_status_t st = validate_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!expert_offsets || !w13 || !aligned(w13, 16)) return MOE_ERR_INVALID_ARG;
+  if (shape->T > 0 && (!x_perm || !aligned(x_perm, 16))) return MOE_ERR_INVALID_ARG;
+  if (shape->n_shared && shape->T > 0 && (!x || !w13s || !aligned(x, 16) || !aligned(w13s, 16)))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
+  const cudaError_t e = launch_gate_up(*shape, ws_layout(*shape), (uint8_t*)ws, x_perm, expert_offsets, w13, x, w13s,
+                                       (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+moe_status_t moe_expert_down(const moe_shape_t* shape, const int32_t* expert_offsets, const moe_bf16_t* w2,
+                             const moe_bf16_t* w2s, moe_bf16_t* y_perm, moe_bf16_t* y_shared, void* ws,
+                             size_t ws_bytes, void* stream) {
+  moe_status_t st = validate_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!expert_offsets || !w2 || !aligned(w2, 16)) return MOE_ERR_INVALID_ARG;
+  if (shape->T > 0 && (!y_perm || !aligned(y_perm, 16))) return MOE_ERR_INVALID_ARG;
+  if (shape->n_shared && shape->T > 0 && (!w2s || !y_shared || !aligned(w2s, 16) || !aligned(y_shared, 16)))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
+  const cudaError_t e = launch_down(*shape, ws_layout(*shape), (uint8_t*)ws, expert_offsets, w2, w2s, y_perm,
+                                    shape->n_shared ? y_shared : nullptr, (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+moe_status_t moe_combine(const moe_shape_t* shape, const moe_bf16_t* y_perm, const int32_t* assign_row,
+                         const float* topk_gate, const moe_bf16_t* y_shared, moe_bf16_t* out, void* ws,
+                         size_t ws_bytes, void* stream) {
+  moe_status_t st = validate_shape(shape);
+  if (st != MOE_OK) return st;
+  if (shape->T > 0 && (!y_perm || !assign_row || !topk_gate || !out)) return MOE_ERR_INVALID_ARG;
+  if ((y_perm && !aligned(y_perm, 16)) || (out && !aligned(out, 16)) || (y_shared && !aligned(y_shared, 16)))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
+  const WsLayout L = ws_layout(*shape);
+  const cudaError_t e = launch_combine(*shape, y_perm, assign_row, topk_gate, y_shared, out,
+                                       reinterpret_cast<uint32_t*>((uint8_t*)ws + L.status), (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+moe_status_t moe_layer(const moe_shape_t* shape, const moe_layer_buffers_t* b, void* ws, size_t ws_bytes,
+                       void* stream) {
+  moe_status_t st = validate_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!b) return MOE_ERR_INVALID_ARG;
+  if (!b->w13 || !b->w2 || !b->expert_counts || !b->expert_offsets || !b->rank_counts || !b->rank_offsets ||
+      !b->imbalance)
+    return MOE_ERR_INVALID_ARG;
+  if (shape->T > 0 && (!b->logits || !b->x || !b->topk_idx || !b->topk_gate || !b->row_src || !b->assign_row ||
+                       !b->x_perm || !b->y_perm || !b->out))
+    return MOE_ERR_INVALID_ARG;
+  if (shape->n_shared && shape->T > 0 && (!b->w13s || !b->w2s || !b->y_shared)) return MOE_ERR_INVALID_ARG;
+  const void* al[] = {b->x, b->w13, b->w2, b->w13s, b->w2s, b->x_perm, b->y_perm, b->y_shared, b->out};
+  for (const void* p : al)
+    if (p && !aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
+  const WsLayout L = ws_layout(*shape);
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* w = (uint8_t*)ws;
+  uint32_t* status = reinterpret_cast<uint32_t*>(w + L.status);
+  cudaError_t e = launch_route(b->logits, b->topk_idx, b->topk_gate, shape->T, shape->E, shape->k, status, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = launch_dispatch(*shape, L, w, b->x, b->topk_idx, b->expert_counts, b->expert_offsets, b->rank_counts,
+                      b->rank_offsets, b->row_src, b->assign_row, b->x_perm, b->imbalance, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const uint16_t* ysh_in = shape->n_shared ? b->y_shared : nullptr;
+  e = launch_gate_up(*shape, L, w, b->x_perm, b->expert_offsets, b->w13, b->x, b->w13s, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = launch_down(*shape, L, w, b->expert_offsets, b->w2, b->w2s, b->y_perm, shape->n_shared ? b->y_shared : nullptr,
+                  s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = launch_combine(*shape, b->y_perm, b->assign_row, b->topk_gate, ysh_in, b->out, status, s);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+const char* moe_status_string(moe_status_t status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+const char* moe_last_cuda_error(void) { return g_last_cuda_error; }
+
+uint64_t moe_set_wait_timeout_ns(uint64_t ns) {
+  return g_wait_timeout_ns.exchange(ns ? ns : kDefaultWaitNs, std::memory_order_relaxed);
+}
+
+}  // extern "C"

@@ -1,0 +1,64 @@
+/*
+ * moe_internal.h -- host-side internals shared by the translation units of
+ * libmoe_b200.so: workspace layout and kernel launchers. Not part of the ABI.
+ */
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kMaxE = 256;
+constexpr int kMaxK = 8;
+constexpr int kTileM = 128;           /* rows per grouped-GEMM tile (tcgen05 M) */
+constexpr int kChunkAssign = 2048;    /* assignments per dispatch histogram chunk */
+constexpr uint64_t kDefaultWaitNs = 2000000000ull; /* bounded-wait limit of the GEMM pipeline */
+
+/* Byte offsets into the caller's workspace (all 256-byte aligned). */
+struct WsLayout {
+  size_t status = 0;      /* uint32 device status word (first 256 bytes) */
+  size_t chunk = 0;       /* int32 [C][E]: per-chunk expert counts, then chunk base rows */
+  size_t local_rank = 0;  /* int32 [A]: rank of an assignment among its chunk's same-expert ones */
+  size_t h = 0;           /* bf16 [h_rows][f]: SwiGLU hidden rows, 128-row padded per expert */
+  size_t total = 0;
+  int64_t A = 0;          /* T * k */
+  int64_t tok_per_chunk = 1;
+  int64_t n_chunks = 0;
+  int64_t mt_routed_max = 0; /* upper bound of sum_e ceil(count_e / 128) */
+  int64_t h_rows = 0;
+};
+
+WsLayout ws_layout(const moe_shape_t& s);
+
+/* Device SM count of the current device (cached). */
+int num_sms();
+
+uint64_t wait_timeout_ns();
+
+cudaError_t launch_route(const float* logits, int32_t* topk_idx, float* topk_gate, int64_t T, int E, int k,
+                         uint32_t* status, cudaStream_t stream);
+
+cudaError_t launch_dispatch(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const uint16_t* x,
+                            const int32_t* topk_idx, int32_t* expert_counts, int32_t* expert_offsets,
+                            int32_t* rank_counts, int32_t* rank_offsets, int32_t* row_src, int32_t* assign_row,
+                            uint16_t* x_perm, float* imbalance, cudaStream_t stream);
+
+/* GEMM1: h (workspace) = silu(A W_gate^T) * (A W_up^T) per expert group */
+cudaError_t launch_gate_up(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const uint16_t* x_perm,
+                           const int32_t* expert_offsets, const uint16_t* w13, const uint16_t* x,
+                           const uint16_t* w13s, cudaStream_t stream);
+
+/* GEMM2: y_perm / y_shared = h W2^T per expert group */
+cudaError_t launch_down(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const int32_t* expert_offsets,
+                        const uint16_t* w2, const uint16_t* w2s, uint16_t* y_perm, uint16_t* y_shared,
+                        cudaStream_t stream);
+
+cudaError_t launch_combine(const moe_shape_t& s, const uint16_t* y_perm, const int32_t* assign_row,
+                           const float* topk_gate, const uint16_t* y_shared, uint16_t* out, uint32_t* status,
+                           cudaStream_t stream);
+
+}  // namespace moe

@@ -137,6 +137,20 @@ moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_bf16_t* x_perm, 
                             const moe_bf16_t* w13s, const moe_bf16_t* w2s, moe_bf16_t* y_perm,
                             moe_bf16_t* y_shared, void* ws, size_t ws_bytes, void* stream);
 
+/* The two halves of moe_expert_ffn, for callers that schedule or time them
+ * separately; moe_expert_ffn is exactly gate_up followed by down.
+ * moe_expert_gate_up: GEMM1 + SwiGLU, h = silu(x W_gate^T) * (x W_up^T), written
+ *   to the workspace (each expert's rows padded to a multiple of 128).
+ * moe_expert_down: GEMM2, y_perm (and y_shared) = h W2^T, reading the h rows that
+ *   the preceding moe_expert_gate_up on the same workspace, shape and
+ *   expert_offsets left there. Arguments as for moe_expert_ffn. */
+moe_status_t moe_expert_gate_up(const moe_shape_t* shape, const moe_bf16_t* x_perm, const int32_t* expert_offsets,
+                                const moe_bf16_t* w13, const moe_bf16_t* x, const moe_bf16_t* w13s, void* ws,
+                                size_t ws_bytes, void* stream);
+moe_status_t moe_expert_down(const moe_shape_t* shape, const int32_t* expert_offsets, const moe_bf16_t* w2,
+                             const moe_bf16_t* w2s, moe_bf16_t* y_perm, moe_bf16_t* y_shared, void* ws,
+                             size_t ws_bytes, void* stream);
+
 /* Combine: un-permute and gate-weighted sum, back in original token order.
  * Page "Expert Parallelism" §4 COMBINE.
  *   out[t] = sum_{j<k} topk_gate[t,j] * y_perm[assign_row[t*k+j]] (+ y_shared[t])
@@ -181,6 +195,14 @@ const char* moe_status_string(moe_status_t status);
 
 /* Text of the last CUDA error seen by this thread in a library call ("" if none). */
 const char* moe_last_cuda_error(void);
+
+/* Diagnostic knob: the limit, in nanoseconds, of each bounded wait inside the
+ * grouped-GEMM pipeline (default 2e9; 0 restores the default). A wait that runs
+ * out sets MOE_DEV_TIMEOUT; the kernel then stops issuing work, waits for its
+ * copies and MMAs in flight, frees its tensor memory and returns, leaving the
+ * context usable. Applies to launches made after the call, process-wide.
+ * Returns the previous value. */
+uint64_t moe_set_wait_timeout_ns(uint64_t ns);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,103 @@
+"""The C ABI library: loads, exports every declared symbol, validates on the host (no GPU).
+
+Every call here fails validation before anything is launched, so no CUDA device
+is touched.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import combine_warp_top_expert_b200 as moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+TINY = moe.Shape(T=256, d=512, E=8, k=2, f=1024, R=2)
+FAKE = 1 << 20  # an aligned, never-dereferenced address
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(moe_\w+)\s*\(", text, re.M)))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = moe.load()
+    names = declared_functions()
+    assert set(names) >= {"moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_layer"}
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(moe.ABI_FUNCTIONS)
+
+
+def test_workspace_bytes_layout():
+    lib = moe.load()
+    n = moe.workspace_bytes(TINY)
+    A = TINY.T * TINY.k
+    chunks = -(-TINY.T // (2048 // TINY.k))
+    h_rows = 128 * (A // 128 + min(TINY.E, A))
+    expect = 256 + (-(-chunks * TINY.E * 4 // 256) * 256) + (-(-A * 4 // 256) * 256) + (-(-h_rows * TINY.f * 2 // 256) * 256)
+    assert n == expect
+    # shared expert adds its padded hidden rows
+    sh = moe.Shape(T=256, d=512, E=8, k=2, f=1024, R=2, n_shared=1)
+    assert moe.workspace_bytes(sh) == n + 256 * TINY.f * 2
+    # empty batch still has the status header
+    assert moe.workspace_bytes(moe.Shape(T=0, d=512, E=8, k=2, f=1024, R=2)) >= 256
+    for bad in (moe.Shape(-1, 512, 8, 2, 1024, 2), moe.Shape(8, 512, 8, 9, 1024, 2), moe.Shape(8, 512, 8, 2, 1024, 3),
+                moe.Shape(8, 500, 8, 2, 1024, 2), moe.Shape(8, 512, 300, 2, 1024, 2),
+                moe.Shape(8, 512, 8, 2, 1024, 2, n_shared=2)):
+        assert lib.moe_workspace_bytes(ctypes.byref(bad.c())) == 0
+
+
+@pytest.mark.parametrize("shape,code", [
+    (moe.Shape(T=8, d=512, E=8, k=0, f=1024, R=2), moe.MOE_ERR_INVALID_ARG),
+    (moe.Shape(T=8, d=512, E=4, k=5, f=1024, R=2), moe.MOE_ERR_INVALID_ARG),
+    (moe.Shape(T=8, d=512, E=8, k=2, f=1024, R=3), moe.MOE_ERR_INVALID_ARG),
+    (moe.Shape(T=8, d=512, E=8, k=2, f=1024, R=2, n_shared=3), moe.MOE_ERR_INVALID_ARG),
+    (moe.Shape(T=8, d=520, E=8, k=2, f=1024, R=2), moe.MOE_ERR_UNSUPPORTED),
+    (moe.Shape(T=8, d=512, E=8, k=2, f=1000, R=2), moe.MOE_ERR_UNSUPPORTED),
+    (moe.Shape(T=8, d=512, E=512, k=2, f=1024, R=2), moe.MOE_ERR_UNSUPPORTED),
+    (moe.Shape(T=8, d=512, E=16, k=9, f=1024, R=2), moe.MOE_ERR_UNSUPPORTED),
+])
+def test_invalid_shapes_are_rejected_before_launch(shape, code):
+    lib = moe.load()
+    s = ctypes.byref(shape.c())
+    assert lib.moe_route(s, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == code
+    assert lib.moe_dispatch(s, *([FAKE] * 10), FAKE, 1 << 30, None) == code
+    assert lib.moe_expert_ffn(s, *([FAKE] * 9), FAKE, 1 << 30, None) == code
+    assert lib.moe_combine(s, *([FAKE] * 5), FAKE, 1 << 30, None) == code
+
+
+def test_null_pointers_and_small_workspace_are_rejected():
+    lib = moe.load()
+    s = ctypes.byref(TINY.c())
+    assert lib.moe_route(None, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_route(s, None, FAKE, FAKE, FAKE, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_route(s, FAKE, FAKE, FAKE, FAKE, 16, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_route(s, FAKE, FAKE, FAKE, FAKE + 8, 1 << 30, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_dispatch(s, FAKE + 2, *([FAKE] * 9), FAKE, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_ffn(s, *([FAKE] * 9), FAKE, 100, None) == moe.MOE_ERR_WORKSPACE
+    sh = ctypes.byref(moe.Shape(T=8, d=512, E=8, k=2, f=1024, R=2, n_shared=1).c())
+    assert lib.moe_expert_ffn(sh, FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE, None, FAKE, 1 << 30,
+                              None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(s, None, FAKE, FAKE, None, FAKE, FAKE, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_layer(s, None, FAKE, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    b = moe.moe_layer_buffers_t()
+    assert lib.moe_layer(s, ctypes.byref(b), FAKE, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    bits = ctypes.c_uint32()
+    assert lib.moe_get_status(FAKE, 1 << 30, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_get_status(FAKE + 1, 1 << 30, ctypes.byref(bits), None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_clear_status(None, 1 << 30, None) == moe.MOE_ERR_WORKSPACE
+
+
+def test_status_strings_and_timeout_knob():
+    lib = moe.load()
+    assert lib.moe_status_string(0) == b"MOE_OK"
+    assert lib.moe_status_string(4) == b"MOE_ERR_CUDA"
+    assert lib.moe_status_string(99) == b"MOE_ERR_UNKNOWN"
+    old = lib.moe_set_wait_timeout_ns(12345)
+    assert old == 2_000_000_000
+    assert lib.moe_set_wait_timeout_ns(0) == 12345
+    assert lib.moe_set_wait_timeout_ns(0) == 2_000_000_000

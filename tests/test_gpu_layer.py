@@ -1,0 +1,143 @@
+"""The whole layer (moe_layer) against the oracle, at oracle-sized and full sizes.
+
+Full sizes (the workloads the benchmark times): inputs are filled on the device
+by the seeded generator; routing, counts, offsets, permutation and imbalance are
+compared bit for bit with the oracle over the whole batch, x_perm by a property
+that holds at any size, and the floating-point outputs (out, y_perm rows) on a
+sample of tokens that the oracle computes one by one from host-regenerated
+inputs (only the sampled tokens' experts' weights are regenerated).
+"""
+import numpy as np
+import pytest
+
+import combine_warp_top_expert_b200 as moe
+import moe_synth
+import oracle
+from parity_util import GATE_TOL, bits, close, f64, np_i32
+
+pytestmark = pytest.mark.gpu
+
+
+def _shape(wl):
+    return moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, n_shared=wl.n_shared)
+
+
+def _run_layer(wl):
+    dv = moe_synth.device_inputs(wl)
+    layer = moe.MoELayer(_shape(wl), dv["w13"], dv["w2"], dv.get("w13s"), dv.get("w2s"))
+    outs = layer(dv["logits"], dv["x"])
+    status = moe.get_status(layer.ws)
+    return dv, layer, outs, status
+
+
+def _check_routing(wl, outs):
+    lg = moe_synth.host_logits(wl)
+    ridx, rgate, _ = oracle.route(lg, wl.k)
+    assert np.array_equal(np_i32(outs["topk_idx"]), ridx)
+    assert np.max(np.abs(outs["topk_gate"].cpu().numpy().astype(np.float64) - rgate)) <= GATE_TOL
+    ref = oracle.dispatch(ridx, wl.E, wl.R)
+    for n in ("expert_counts", "expert_offsets", "rank_counts", "rank_offsets", "row_src", "assign_row"):
+        assert np.array_equal(np_i32(outs[n]), ref[n]), n
+    assert np.array_equal(outs["imbalance"].cpu().numpy().view(np.uint32), ref["imbalance"].view(np.uint32))
+    return ridx, rgate, ref
+
+
+def test_layer_tiny_full_parity():
+    wl = moe_synth.workload("tiny")
+    dv, layer, outs, status = _run_layer(wl)
+    assert status == 0
+    _check_routing(wl, outs)
+    res = oracle.layer(moe_synth.host_x(wl), moe_synth.host_logits(wl), moe_synth.host_w13(wl),
+                       moe_synth.host_w2(wl), wl.k, wl.R)
+    assert np.array_equal(bits(outs["x_perm"]), res["x_perm"])
+    close(f64(bits(outs["y_perm"])), res["y_perm"], "y_perm")
+    close(f64(bits(outs["out"])), res["out"], "out")
+
+
+def test_layer_with_shared_expert_full_parity():
+    wl = moe_synth.Workload("sh", T=200, d=256, E=16, k=4, f=256, R=4, n_shared=1, bias_kind="zipf", zipf_s=1.0)
+    dv, layer, outs, status = _run_layer(wl)
+    assert status == 0
+    _check_routing(wl, outs)
+    res = oracle.layer(moe_synth.host_x(wl), moe_synth.host_logits(wl), moe_synth.host_w13(wl),
+                       moe_synth.host_w2(wl), wl.k, wl.R, moe_synth.host_w13s(wl), moe_synth.host_w2s(wl))
+    close(f64(bits(outs["y_shared"])), res["y_shared"], "y_shared")
+    close(f64(bits(outs["out"])), res["out"], "out")
+
+
+def test_layer_is_deterministic_across_calls():
+    import torch
+    wl = moe_synth.workload("tiny")
+    dv, layer, outs, status = _run_layer(wl)
+    first = {n: outs[n].clone() for n in ("x_perm", "y_perm", "out", "row_src", "topk_gate")}
+    layer(dv["logits"], dv["x"])
+    for n, t in first.items():
+        a, b = t, layer.outs[n]
+        if a.dtype == torch.bfloat16:
+            a, b = a.view(torch.int16), b.view(torch.int16)
+        assert torch.equal(a, b), n
+
+
+def _sampled_parity(wl, outs, ridx, rgate, ref, n_tokens, seed=0):
+    toks = np.sort(np.random.default_rng(seed).choice(wl.T, n_tokens, replace=False))
+    x_rows = moe_synth.host_x(wl, toks)
+    out_gpu = f64(bits(outs["out"][toks]))
+    y_perm_gpu = outs["y_perm"]
+    want = np.zeros((len(toks), wl.d))
+    experts = sorted(set(ridx[toks].reshape(-1).tolist()))
+    import torch
+    for e in experts:
+        sel = [(i, j) for i, t in enumerate(toks) for j in range(wl.k) if ridx[t, j] == e]
+        y = oracle.swiglu(x_rows[[i for i, _ in sel]], moe_synth.host_w13(wl, e), moe_synth.host_w2(wl, e))
+        rows = [ref["assign_row"][toks[i] * wl.k + j] for i, j in sel]
+        close(f64(bits(y_perm_gpu[torch.tensor(rows, device="cuda").long()])), y, f"y_perm expert {e}")
+        for (i, j), yr in zip(sel, y):
+            want[i] += float(rgate[toks[i], j]) * yr
+    if wl.n_shared:
+        ys = oracle.swiglu(x_rows, moe_synth.host_w13s(wl), moe_synth.host_w2s(wl))
+        close(f64(bits(outs["y_shared"][toks])), ys, "y_shared")
+        want += ys
+    close(out_gpu, want, "out")
+
+
+@pytest.mark.parametrize("name,n_tokens", [("mixtral_prefill", 6), ("dsv3_decode", 6), ("qwen3_mixed", 8),
+                                           ("dsv3_skewed_prefill", 3)])
+def test_layer_full_size_sampled_parity(name, n_tokens):
+    import torch
+    wl = moe_synth.workload(name)
+    dv, layer, outs, status = _run_layer(wl)
+    assert status == 0
+    ridx, rgate, ref = _check_routing(wl, outs)
+    # x_perm: every assignment's row equals its token's row (any size)
+    rows = torch.from_numpy(ref["assign_row"]).cuda().long()
+    a = torch.arange(wl.T * wl.k, device="cuda")
+    for c in torch.split(a, 1 << 14):
+        assert torch.equal(outs["x_perm"].view(torch.int16)[rows[c]], dv["x"].view(torch.int16)[c // wl.k])
+    assert torch.isfinite(outs["out"].float()).all()
+    _sampled_parity(wl, outs, ridx, rgate, ref, n_tokens)
+    del layer, outs, dv
+    torch.cuda.empty_cache()
+
+
+def test_empty_batch_is_a_no_op():
+    wl = moe_synth.workload("tiny").with_(T=0)
+    dv, layer, outs, status = _run_layer(wl)
+    assert status == 0
+    assert np.all(np_i32(outs["expert_counts"]) == 0)
+    assert outs["imbalance"].cpu().numpy().tolist() == [1.0, 1.0]
+
+
+def test_inconsistent_offsets_are_reported_not_hung():
+    import torch
+    wl = moe_synth.workload("tiny")
+    shape = _shape(wl)
+    dv = moe_synth.device_inputs(wl)
+    offs = torch.tensor([0, 100, 50, 300, 400, 450, 500, 510, 512], dtype=torch.int32, device="cuda")  # decreasing
+    y = torch.zeros((shape.A, wl.d), dtype=torch.bfloat16, device="cuda")
+    ws = moe.new_workspace(shape)
+    xp = torch.zeros((shape.A, wl.d), dtype=torch.bfloat16, device="cuda")
+    moe.moe_expert_ffn(shape, xp, offs, dv["w13"], dv["w2"], None, None, None, y, None, ws)
+    assert moe.get_status(ws) & moe.MOE_DEV_COUNT_MISMATCH
+    # the context stays usable
+    dv2, layer, outs, status = _run_layer(wl)
+    assert status == 0

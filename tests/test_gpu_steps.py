@@ -1,0 +1,304 @@
+"""GPU parity of each step against the CPU oracle, through the C ABI.
+
+Inputs come from the seeded generator (host fill for the oracle, device fill or
+a host->device copy for the GPU); every expected value comes from the oracle.
+Routing, counts, offsets, permutation, x_perm and imbalance are compared bit
+for bit; gates within 2^-20; bf16 outputs within rel-L2 5e-3 and max-abs
+3e-2 * max|ref| (tests/parity_util.py).
+"""
+import numpy as np
+import pytest
+
+import combine_warp_top_expert_b200 as moe
+import moe_synth
+import oracle
+from parity_util import GATE_TOL, bits, close, f64, np_i32
+
+pytestmark = pytest.mark.gpu
+
+WORKLOADS = ["tiny", "mixtral_prefill", "dsv3_decode", "qwen3_mixed", "dsv3_skewed_prefill"]
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _shape(wl):
+    return moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, n_shared=wl.n_shared)
+
+
+def _bf16_dev(a_bits):
+    torch = _torch()
+    return torch.from_numpy(np.ascontiguousarray(a_bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def _gpu_route(shape, logits_np):
+    torch = _torch()
+    lg = torch.from_numpy(np.ascontiguousarray(logits_np, np.float32)).cuda()
+    idx = torch.empty((shape.T, shape.k), dtype=torch.int32, device="cuda")
+    gate = torch.empty((shape.T, shape.k), dtype=torch.float32, device="cuda")
+    ws = moe.new_workspace(shape)
+    moe.moe_route(shape, lg, idx, gate, ws)
+    return np_i32(idx), gate.cpu().numpy(), moe.get_status(ws)
+
+
+def _gpu_dispatch(shape, x_dev, idx_np):
+    torch = _torch()
+    i32 = torch.int32
+    dev = "cuda"
+    o = dict(expert_counts=torch.empty(shape.E, dtype=i32, device=dev),
+             expert_offsets=torch.empty(shape.E + 1, dtype=i32, device=dev),
+             rank_counts=torch.empty(shape.R, dtype=i32, device=dev),
+             rank_offsets=torch.empty(shape.R + 1, dtype=i32, device=dev),
+             row_src=torch.empty(shape.A, dtype=i32, device=dev),
+             assign_row=torch.empty(shape.A, dtype=i32, device=dev),
+             x_perm=torch.empty((shape.A, shape.d), dtype=torch.bfloat16, device=dev),
+             imbalance=torch.empty(2, dtype=torch.float32, device=dev))
+    ws = moe.new_workspace(shape)
+    idx = torch.from_numpy(np.ascontiguousarray(idx_np, np.int32)).cuda()
+    moe.moe_dispatch(shape, x_dev, idx, o["expert_counts"], o["expert_offsets"], o["rank_counts"],
+                     o["rank_offsets"], o["row_src"], o["assign_row"], o["x_perm"], o["imbalance"], ws)
+    o["status"] = moe.get_status(ws)
+    return o
+
+
+# ---------------------------------------------------------------------------
+# generator: device fill == host fill
+# ---------------------------------------------------------------------------
+
+def test_device_fill_equals_host_fill():
+    wl = moe_synth.workload("tiny").with_(n_shared=1)
+    dv = moe_synth.device_inputs(wl)
+    assert np.array_equal(bits(dv["x"]), moe_synth.host_x(wl))
+    assert np.array_equal(dv["logits"].cpu().numpy().view(np.uint32), moe_synth.host_logits(wl).view(np.uint32))
+    assert np.array_equal(bits(dv["w13"]), moe_synth.host_w13(wl))
+    assert np.array_equal(bits(dv["w2"]), moe_synth.host_w2(wl))
+    assert np.array_equal(bits(dv["w13s"]), moe_synth.host_w13s(wl))
+    wl5 = moe_synth.workload("dsv3_skewed_prefill")
+    lg = moe_synth.device_inputs(wl5, weights=False)["logits"]
+    assert np.array_equal(lg.cpu().numpy().view(np.uint32), moe_synth.host_logits(wl5).view(np.uint32))
+
+
+# ---------------------------------------------------------------------------
+# route
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", WORKLOADS)
+def test_route_matches_oracle(name):
+    wl = moe_synth.workload(name)
+    lg = moe_synth.host_logits(wl)
+    idx, gate, status = _gpu_route(_shape(wl), lg)
+    ridx, rgate, _ = oracle.route(lg, wl.k)
+    assert status == 0
+    assert np.array_equal(idx, ridx)
+    assert np.max(np.abs(gate.astype(np.float64) - rgate)) <= GATE_TOL
+
+
+@pytest.mark.parametrize("E,k", [(1, 1), (5, 3), (8, 8), (33, 4), (64, 2), (256, 8), (255, 7)])
+def test_route_ties_signed_zeros_and_infinities(E, k):
+    rng = np.random.default_rng(E * 7 + k)
+    T = 777
+    lg = rng.integers(-2, 3, size=(T, E)).astype(np.float32)           # exact ties everywhere
+    lg[::5] = np.where(lg[::5] == 0, np.float32(-0.0), lg[::5])         # -0.0 ties +0.0
+    lg[3] = -np.inf                                                      # all -inf: gates 1/k
+    lg[4, : E // 2] = -np.inf
+    shape = moe.Shape(T=T, d=128, E=E, k=k, f=128, R=1)
+    idx, gate, status = _gpu_route(shape, lg)
+    ridx, rgate, nan = oracle.route(lg, k)
+    assert status == 0 and nan == 0
+    assert np.array_equal(idx, ridx)
+    assert np.max(np.abs(gate.astype(np.float64) - rgate)) <= GATE_TOL
+
+
+def test_route_nan_is_ordered_last_and_flagged():
+    lg = np.random.default_rng(0).normal(size=(64, 16)).astype(np.float32)
+    lg[7, 3] = np.nan
+    lg[9, :] = np.nan
+    shape = moe.Shape(T=64, d=128, E=16, k=4, f=128, R=1)
+    idx, gate, status = _gpu_route(shape, lg)
+    ridx, rgate, nan = oracle.route(lg, 4)
+    assert nan == 17 and status & moe.MOE_DEV_NAN_LOGIT
+    assert np.array_equal(idx, ridx)
+    assert np.max(np.abs(gate.astype(np.float64) - rgate)) <= GATE_TOL
+
+
+# ---------------------------------------------------------------------------
+# dispatch
+# ---------------------------------------------------------------------------
+
+def _check_dispatch(o, ref, x_np=None, k=None):
+    for n in ("expert_counts", "expert_offsets", "rank_counts", "rank_offsets", "row_src", "assign_row"):
+        assert np.array_equal(np_i32(o[n]), ref[n]), n
+    assert np.array_equal(o["imbalance"].cpu().numpy().view(np.uint32), ref["imbalance"].view(np.uint32))
+    if x_np is not None:
+        ref_xp = oracle.permute_rows(x_np, ref["row_src"], k)
+        total = ref["expert_offsets"][-1]
+        assert np.array_equal(bits(o["x_perm"])[:total], ref_xp[:total])
+
+
+@pytest.mark.parametrize("name", WORKLOADS)
+def test_dispatch_matches_oracle(name):
+    torch = _torch()
+    wl = moe_synth.workload(name)
+    shape = _shape(wl)
+    ridx, _, _ = oracle.route(moe_synth.host_logits(wl), wl.k)
+    ref = oracle.dispatch(ridx, wl.E, wl.R)
+    x_dev = moe_synth.device_inputs(wl, weights=False)["x"]
+    o = _gpu_dispatch(shape, x_dev, ridx)
+    assert o["status"] == 0
+    if wl.T * wl.d <= (1 << 24):
+        _check_dispatch(o, ref, moe_synth.host_x(wl), wl.k)
+    else:
+        _check_dispatch(o, ref)
+        # x_perm at full size: every row equals its token's row (property), checked on the device
+        a = torch.arange(shape.A, device="cuda")
+        rows = torch.from_numpy(ref["assign_row"]).cuda().long()
+        xp = o["x_perm"].view(torch.int16)
+        xs = x_dev.view(torch.int16)
+        for c in torch.split(a, 1 << 14):
+            assert torch.equal(xp[rows[c]], xs[c // wl.k])
+        # and a sample of rows against the host-generated x, bit for bit
+        samp = np.random.default_rng(1).choice(shape.A, 64, replace=False)
+        toks = samp // wl.k
+        got = bits(o["x_perm"][torch.from_numpy(ref["assign_row"][samp]).cuda().long()])
+        assert np.array_equal(got, moe_synth.host_x(wl, toks))
+
+
+def test_dispatch_worked_imbalance_example():
+    counts = np.array([140, 95, 78, 62, 48, 40, 31, 18])
+    experts = np.repeat(np.arange(8), counts)
+    np.random.default_rng(7).shuffle(experts)
+    idx = experts.reshape(512, 1).astype(np.int32)
+    x_np = moe_synth.host_x(moe_synth.Workload("p5", T=512, d=512, E=8, k=1, f=1024, R=8))
+    for R, imb in ((8, (2.1875, 2.1875)), (2, (1.46484375, 2.1875))):
+        shape = moe.Shape(T=512, d=512, E=8, k=1, f=1024, R=R)
+        o = _gpu_dispatch(shape, _bf16_dev(x_np), idx)
+        ref = oracle.dispatch(idx, 8, R)
+        _check_dispatch(o, ref, x_np, 1)
+        assert tuple(o["imbalance"].cpu().numpy().tolist()) == imb
+        assert list(np_i32(o["expert_counts"])) == counts.tolist()
+
+
+@pytest.mark.parametrize("T,E,k,R", [(0, 8, 2, 2), (1, 1, 1, 1), (1, 256, 8, 8), (1000, 37, 5, 1), (4099, 64, 3, 16),
+                                     (2049, 8, 1, 4), (3000, 256, 8, 8)])
+def test_dispatch_edge_shapes(T, E, k, R):
+    rng = np.random.default_rng(T + E)
+    idx = rng.integers(0, E, size=(T, k)).astype(np.int32)   # repeats within a token allowed
+    shape = moe.Shape(T=T, d=128, E=E, k=k, f=128, R=R)
+    x_np = moe_synth.host_x(moe_synth.Workload("e", T=T, d=128, E=E, k=k, f=128, R=R))
+    o = _gpu_dispatch(shape, _bf16_dev(x_np), idx)
+    assert o["status"] == 0
+    _check_dispatch(o, oracle.dispatch(idx, E, R), x_np, k)
+    if T == 0:
+        assert o["imbalance"].cpu().numpy().tolist() == [1.0, 1.0]
+
+
+def test_dispatch_out_of_range_entries_are_skipped_and_flagged():
+    T, E, k = 300, 16, 2
+    idx = np.random.default_rng(3).integers(0, E, size=(T, k)).astype(np.int32)
+    idx[5, 1] = E
+    idx[100, 0] = -3
+    shape = moe.Shape(T=T, d=128, E=E, k=k, f=128, R=4)
+    x_np = moe_synth.host_x(moe_synth.Workload("e", T=T, d=128, E=E, k=k, f=128, R=4))
+    o = _gpu_dispatch(shape, _bf16_dev(x_np), idx)
+    ref = oracle.dispatch(idx, E, 4)
+    assert ref["skipped"] == 2 and o["status"] & moe.MOE_DEV_BOUNDS
+    _check_dispatch(o, ref, x_np, k)
+
+
+# ---------------------------------------------------------------------------
+# combine
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("shared", [False, True])
+@pytest.mark.parametrize("T,d,E,k", [(256, 512, 8, 2), (130, 1024, 64, 8), (1, 128, 4, 3)])
+def test_combine_matches_oracle(T, d, E, k, shared):
+    torch = _torch()
+    wl = moe_synth.Workload("c", T=T, d=d, E=E, k=k, f=128, R=1, seed=11)
+    idx, gate, _ = oracle.route(moe_synth.host_logits(wl), k)
+    ref = oracle.dispatch(idx, E, 1)
+    y_np = moe_synth.host_x(wl.with_(T=T * k, seed=12))     # any bf16 rows stand in for expert outputs
+    ys_np = moe_synth.host_x(wl.with_(seed=13)) if shared else None
+    shape = moe.Shape(T=T, d=d, E=E, k=k, f=128, R=1)
+    out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    ws = moe.new_workspace(shape)
+    moe.moe_combine(shape, _bf16_dev(y_np), torch.from_numpy(ref["assign_row"]).cuda(),
+                    torch.from_numpy(gate).cuda(), _bf16_dev(ys_np) if shared else None, out, ws)
+    assert moe.get_status(ws) == 0
+    expect = oracle.combine(f64(y_np), ref["assign_row"], gate, f64(ys_np) if shared else None)
+    close(f64(bits(out)), expect, "combine")
+    # one bf16 rounding of an fp32 sum: within one bf16 ulp of the fp64 value
+    assert np.all(np.abs(f64(bits(out)) - expect) <= 2.0 ** -7 * np.abs(expect) + 1e-6)
+
+
+def test_dispatch_then_combine_k1_is_exact_identity():
+    torch = _torch()
+    wl = moe_synth.workload("tiny").with_(k=1)
+    shape = _shape(wl)
+    lg = moe_synth.host_logits(wl)
+    ridx, rgate, _ = oracle.route(lg, 1)
+    x_np = moe_synth.host_x(wl)
+    o = _gpu_dispatch(shape, _bf16_dev(x_np), ridx)
+    out = torch.empty((wl.T, wl.d), dtype=torch.bfloat16, device="cuda")
+    ws = moe.new_workspace(shape)
+    moe.moe_combine(shape, o["x_perm"], o["assign_row"], torch.from_numpy(rgate).cuda(), None, out, ws)
+    assert np.array_equal(bits(out), x_np)
+
+
+# ---------------------------------------------------------------------------
+# expert FFN (grouped GEMM)
+# ---------------------------------------------------------------------------
+
+def _ffn_case(wl, idx=None):
+    torch = _torch()
+    shape = _shape(wl)
+    x_np = moe_synth.host_x(wl)
+    if idx is None:
+        idx, _, _ = oracle.route(moe_synth.host_logits(wl), wl.k)
+    ref = oracle.dispatch(idx, wl.E, wl.R)
+    xp_np = oracle.permute_rows(x_np, ref["row_src"], wl.k)
+    w13, w2 = moe_synth.host_w13(wl), moe_synth.host_w2(wl)
+    w13s = moe_synth.host_w13s(wl) if wl.n_shared else None
+    w2s = moe_synth.host_w2s(wl) if wl.n_shared else None
+    y_ref, ys_ref = oracle.expert_ffn(xp_np, ref["expert_offsets"], w13, w2, x_np, w13s, w2s)
+    y = torch.empty((shape.A, wl.d), dtype=torch.bfloat16, device="cuda")
+    ys = torch.empty((wl.T, wl.d), dtype=torch.bfloat16, device="cuda") if wl.n_shared else None
+    ws = moe.new_workspace(shape)
+    moe.moe_expert_ffn(shape, _bf16_dev(xp_np), torch.from_numpy(ref["expert_offsets"]).cuda(), _bf16_dev(w13),
+                       _bf16_dev(w2), _bf16_dev(x_np) if wl.n_shared else None,
+                       _bf16_dev(w13s) if wl.n_shared else None, _bf16_dev(w2s) if wl.n_shared else None, y, ys, ws)
+    assert moe.get_status(ws) == 0
+    total = ref["expert_offsets"][-1]
+    close(f64(bits(y))[:total], y_ref[:total], "y_perm")
+    for e in range(wl.E):   # per expert too, so one bad expert cannot hide in the global norm
+        r0, r1 = ref["expert_offsets"][e], ref["expert_offsets"][e + 1]
+        if r1 > r0:
+            close(f64(bits(y))[r0:r1], y_ref[r0:r1], f"y_perm expert {e}")
+    if wl.n_shared:
+        close(f64(bits(ys)), ys_ref, "y_shared")
+
+
+def test_expert_ffn_tiny():
+    _ffn_case(moe_synth.workload("tiny"))
+
+
+@pytest.mark.parametrize("wl", [
+    # skewed: one expert with several m-tiles and a ragged tail, empty experts, shared expert, N=256 down tiles
+    moe_synth.Workload("skew", T=300, d=256, E=6, k=2, f=384, R=2, n_shared=1, bias_kind="hot", n_hot=1, beta=3.0),
+    # d % 256 != 0: 128-column down tiles
+    moe_synth.Workload("d384", T=200, d=384, E=4, k=1, f=256, R=2),
+    # one expert, top-1: a dense SwiGLU with a 2-row ragged tail
+    moe_synth.Workload("dense", T=130, d=128, E=1, k=1, f=128, R=1),
+    # many experts, few rows each (decode-like)
+    moe_synth.Workload("decode", T=16, d=256, E=64, k=8, f=256, R=8, n_shared=1, bias_kind="zipf", zipf_s=1.2),
+])
+def test_expert_ffn_shapes(wl):
+    _ffn_case(wl)
+
+
+def test_expert_ffn_with_empty_and_full_experts():
+    wl = moe_synth.Workload("emp", T=257, d=128, E=5, k=1, f=256, R=1)
+    idx = np.zeros((257, 1), np.int32)
+    idx[200:, 0] = 3          # experts 1, 2, 4 empty; expert 0 has 200 rows, expert 3 57
+    _ffn_case(wl, idx)
