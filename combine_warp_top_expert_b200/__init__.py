@@ -23,7 +23,7 @@ LIB_PATH = _build.LIB_PATH
 ABI_FUNCTIONS = (
     "moe_workspace_bytes", "moe_clear_status", "moe_get_status", "moe_route", "moe_dispatch", "moe_expert_ffn",
     "moe_combine", "moe_layer", "moe_status_string", "moe_last_cuda_error", "moe_set_wait_timeout_ns",
-    "moe_expert_gate_up", "moe_expert_down",
+    "moe_expert_gate_up", "moe_expert_down", "moe_dispatch_static",
 )
 
 
@@ -68,6 +68,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     L.moe_route.argtypes = [shp, vp, vp, vp, vp, sz, vp]
     L.moe_dispatch.restype = st
     L.moe_dispatch.argtypes = [shp] + [vp] * 10 + [vp, sz, vp]
+    L.moe_dispatch_static.restype = st
+    L.moe_dispatch_static.argtypes = [shp] + [vp] * 11 + [vp]
     L.moe_expert_ffn.restype = st
     L.moe_expert_ffn.argtypes = [shp] + [vp] * 9 + [vp, sz, vp]
     L.moe_expert_gate_up.restype = st

@@ -17,14 +17,20 @@ namespace {
 thread_local char g_last_cuda_error[256] = "";
 std::atomic<uint64_t> g_wait_timeout_ns{kDefaultWaitNs};
 
+}  // namespace
+
 moe_status_t cuda_fail(cudaError_t e) {
   std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
   return MOE_ERR_CUDA;
 }
 
+namespace {
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace
 
 moe_status_t validate_shape(const moe_shape_t* s) {
   if (!s) return MOE_ERR_INVALID_ARG;
@@ -35,6 +41,8 @@ moe_status_t validate_shape(const moe_shape_t* s) {
   if (s->d % 128 != 0 || s->f % 128 != 0 || s->d > 65536 || s->f > 65536) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
+
+namespace {
 
 moe_status_t check_ws(const moe_shape_t& s, const void* ws, size_t ws_bytes) {
   if (!ws || !aligned(ws, 256)) return MOE_ERR_WORKSPACE;

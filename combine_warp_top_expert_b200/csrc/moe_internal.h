@@ -34,6 +34,12 @@ struct WsLayout {
 
 WsLayout ws_layout(const moe_shape_t& s);
 
+/* Host-side shape validation shared by every entry point. */
+moe_status_t validate_shape(const moe_shape_t* s);
+
+/* Record a CUDA error for moe_last_cuda_error() and return MOE_ERR_CUDA. */
+moe_status_t cuda_fail(cudaError_t e);
+
 /* Device SM count of the current device (cached). */
 int num_sms();
 

@@ -119,6 +119,31 @@ moe_status_t moe_dispatch(const moe_shape_t* shape, const moe_bf16_t* x, const i
                           int32_t* rank_offsets, int32_t* row_src, int32_t* assign_row, moe_bf16_t* x_perm,
                           float* imbalance, void* ws, size_t ws_bytes, void* stream);
 
+/* moe_dispatch for callers that cannot allocate device memory. The pages have
+ * no counterpart to this entry point: it exists for callers such as engine
+ * plugins or serving runtimes whose device memory is planned and owned by their
+ * own arena, and FFI callers with no CUDA allocator, for whom a cudaMalloc on the
+ * hot path is not allowed or would synchronise the device.
+ * Same kernels, arguments (minus the workspace) and outputs as moe_dispatch. The
+ * scratch the kernels need (status word, per-chunk counts, in-chunk ranks) is a
+ * fixed 1 MiB array inside the library, held on every GPU that loads the library
+ * until the process exits. Shapes whose scratch exceeds it are rejected with
+ * MOE_ERR_UNSUPPORTED before anything runs: the need is 256 + (bytes of
+ * ceil(T / floor(2048 / k)) * E int32 rounded up to 256) + (bytes of T*k int32
+ * rounded up to 256), e.g. T = 16384, k = 8, E = 256 needs 590,080 bytes.
+ * This entry point allocates nothing (no cudaMalloc/cudaFree). Its first call on
+ * a device looks up the array's device address (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture. Every call
+ * shares the one array and clears its status word at the start, so calls whose
+ * executions overlap on the GPU (other streams, other host threads) race and
+ * must be serialised by the caller.
+ *   status  device pointer to one uint32 (may be NULL): receives this call's
+ *           MOE_DEV_* bits (asynchronously, on `stream`). */
+moe_status_t moe_dispatch_static(const moe_shape_t* shape, const moe_bf16_t* x, const int32_t* topk_idx,
+                                 int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
+                                 int32_t* rank_offsets, int32_t* row_src, int32_t* assign_row, moe_bf16_t* x_perm,
+                                 float* imbalance, uint32_t* status, void* stream);
+
 /* Expert FFN: one grouped GEMM over all experts (tcgen05 tensor cores).
  * Page "Expert Parallelism" §4 COMPUTE ("each expert processes its tokens ...
  * many different-shaped GEMMs in one launch") and §1 (E expert FFNs); the FFN is
