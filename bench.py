@@ -146,13 +146,12 @@ def oracle_sample_run(wl, n_tokens: int, weights=None):
     return time.perf_counter() - t0, weights
 
 
-def cpu_baseline(wl, budget_s: float = 20.0):
-    import moe_synth  # noqa: F401
+def cpu_baseline(wl, min_s: float = 10.0, target_s: float = 15.0):
+    """The oracle as it stands on a bounded token sample, grown until it takes 10-30 s of CPU time."""
     n = 4
     dt, weights = oracle_sample_run(wl, n)
-    # grow the sample to roughly the time budget (the oracle's cost is about linear in tokens)
-    if dt < budget_s / 4:
-        n = int(min(wl.T, max(n, n * (budget_s * 0.6) / max(dt, 1e-3))))
+    while dt < min_s and n < wl.T:
+        n = int(min(wl.T, max(n + 1, n * min(8.0, max(1.5, target_s / max(dt, 1e-3))))))
         dt, _ = oracle_sample_run(wl, n, weights)
     return dict(value=n / dt, unit=UNIT, cores=os.cpu_count(), kind="oracle",
                 sample=f"oracle layer (fp64, OpenMP over rows) on the first {n} of {wl.T} tokens of {wl.name}, "
@@ -338,12 +337,16 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the workload's batch size T (smaller cases for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
 
     import moe_synth
     wl = moe_synth.workload(args.config)
+    if args.tokens is not None:
+        wl = wl.with_(T=args.tokens)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
