@@ -65,6 +65,60 @@ def load_peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
 
 
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "dram_traffic.md")
+KERNEL_SOURCES = ("combine_warp_top_expert_b200/csrc/expert_ffn.cu", "combine_warp_top_expert_b200/csrc/moe_device.cuh",
+                  "combine_warp_top_expert_b200/csrc/moe_internal.h")
+
+
+def kernel_source_hash() -> str:
+    """Hash of the grouped-GEMM sources; a traffic figure is valid only for the source it was taken on."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum) recorded in
+    profiles/dram_traffic.md for this workload and kernel, or None if absent or taken on other sources."""
+    if not os.path.exists(TRAFFIC_RECORD):
+        return None
+    text = open(TRAFFIC_RECORD).read()
+    if "```json" not in text:
+        return None
+    try:
+        rec = json.loads(text.split("```json", 1)[1].split("```", 1)[0])
+    except ValueError:
+        return None
+    if rec.get("source_hash") != kernel_source_hash():
+        return None
+    e = rec.get("workloads", {}).get(workload, {}).get(kernel)
+    return None if e is None else int(e["dram_bytes_per_launch"])
+
+
+def replica_seed(base_seed: int, rank: int) -> int:
+    """Each replica (rank) runs the workload on its own batch."""
+    return base_seed + rank
+
+
+def max_over_ranks(local_value: float, world: int, device=None) -> float:
+    """The slowest rank's value (device-timed milliseconds or seconds); identity at world = 1."""
+    if world <= 1:
+        return float(local_value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(local_value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(tokens_per_rank: int, steps: int, world: int, max_seconds: float) -> float:
+    """Whole-job tokens/s: all ranks' tokens over the slowest rank's timed region (weak scaling)."""
+    return world * tokens_per_rank * steps / max_seconds
+
+
 # ---------------------------------------------------------------------------
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
@@ -202,7 +256,8 @@ def run_gpu(args, wl, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    wl_r = wl.with_(seed=wl.seed + rank)  # each replica: its own batch
+    moe.set_gemm_policy({"auto": moe.GEMM_AUTO, "single": moe.GEMM_SINGLE, "pair": moe.GEMM_PAIR}[args.gemm_policy])
+    wl_r = wl.with_(seed=replica_seed(wl.seed, rank))
     shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, n_shared=wl.n_shared)
     dv = moe_synth.device_inputs(wl_r, device=dev)
     layer = moe.MoELayer(shape, dv["w13"], dv["w2"], dv.get("w13s"), dv.get("w2s"), device=dev)
@@ -257,12 +312,8 @@ def run_gpu(args, wl, rank, world, local_rank):
         dist.barrier()
     per_step = [ev[0].elapsed_time(ev[5]) for ev in events]
     per_kernel = {n: [ev[j].elapsed_time(ev[j + 1]) for ev in events] for j, n in enumerate(names)}
-    step_ms = sum(per_step)
-    t = torch.tensor([step_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
-    value = world * wl.T * args.steps / (max_ms / 1e3)
+    max_ms = max_over_ranks(sum(per_step), world, dev)
+    value = aggregate_throughput(wl.T, args.steps, world, max_ms / 1e3)
 
     # e2e through the public API with host buffers (pinned), copies inside the timed region
     x_h = dv["x"].cpu().pin_memory()
@@ -279,10 +330,7 @@ def run_gpu(args, wl, rank, world, local_rank):
         layer.forward_host(lg_h, x_h, out_h, stream)
         stream.synchronize()
         e2e_times.append(time.perf_counter() - t0)
-    te = torch.tensor([sum(e2e_times)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = world * wl.T * args.steps / float(te.item())
+    e2e_value = aggregate_throughput(wl.T, args.steps, world, max_over_ranks(sum(e2e_times), world, dev))
 
     if rank != 0:
         return
@@ -309,6 +357,7 @@ def run_gpu(args, wl, rank, world, local_rank):
         "config": {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "f": wl.f, "R": wl.R,
                    "n_shared": wl.n_shared, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "flushed between steps (512 MiB write, outside the step's events)",
+                   "gemm_tiles": args.gemm_policy,
                    "experts_active": work["_n_act"], "imbalance_rank_expert": imbalance,
                    "layer_roofline_frac": t_roof / (max_ms / args.steps / 1e3),
                    "per_step_ms": {n: round(v, 4) for n, v in kern_ms.items()},
@@ -318,7 +367,8 @@ def run_gpu(args, wl, rank, world, local_rank):
                      "peak": peaks["bf16"] if d["bound"] == "tensor" else peaks["hbm"],
                      "unit": "TFLOP/s" if d["bound"] == "tensor" else "GB/s",
                      "frac": d["achieved"] / (peaks["bf16"] if d["bound"] == "tensor" else peaks["hbm"]),
-                     "peak_kind": f"{peaks['source']} burst", "traffic": None},
+                     "peak_kind": f"{peaks['source']} burst",
+                     "traffic": recorded_traffic(wl.name, f"moe_expert_{dom}") if args.tokens is None else None},
         "clocks": clocks.summary(),
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(x_h.numel() * 2 + lg_h.numel() * 4),
                 "d2h_bytes_per_step": int(out_h.numel() * 2)},
@@ -337,6 +387,8 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gemm-policy", default="auto", choices=["auto", "single", "pair"],
+                    help="grouped-GEMM tiles: per-GEMM choice (auto), single-CTA 128-row, or CTA-pair 256x256")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the workload's batch size T (smaller cases for profiling)")
     args = ap.parse_args()

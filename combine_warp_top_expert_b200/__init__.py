@@ -23,8 +23,10 @@ LIB_PATH = _build.LIB_PATH
 ABI_FUNCTIONS = (
     "moe_workspace_bytes", "moe_clear_status", "moe_get_status", "moe_route", "moe_dispatch", "moe_expert_ffn",
     "moe_combine", "moe_layer", "moe_status_string", "moe_last_cuda_error", "moe_set_wait_timeout_ns",
-    "moe_expert_gate_up", "moe_expert_down", "moe_dispatch_static",
+    "moe_expert_gate_up", "moe_expert_down", "moe_dispatch_static", "moe_set_gemm_policy",
+    "moe_set_test_stall",
 )
+GEMM_AUTO, GEMM_SINGLE, GEMM_PAIR = 0, 1, 2
 
 
 class MoEError(RuntimeError):
@@ -84,6 +86,10 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     L.moe_status_string.argtypes = [st]
     L.moe_last_cuda_error.restype = ctypes.c_char_p
     L.moe_last_cuda_error.argtypes = []
+    L.moe_set_gemm_policy.restype = ctypes.c_int
+    L.moe_set_gemm_policy.argtypes = [ctypes.c_int]
+    L.moe_set_test_stall.restype = ctypes.c_int
+    L.moe_set_test_stall.argtypes = [ctypes.c_int]
     L.moe_set_wait_timeout_ns.restype = ctypes.c_uint64
     L.moe_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
     _lib = L
@@ -167,6 +173,19 @@ def get_status(ws, stream=None) -> int:
 
 def set_wait_timeout_ns(ns: int) -> int:
     return load().moe_set_wait_timeout_ns(ns)
+
+
+def set_test_stall(enable: bool) -> int:
+    """Test hook of the bounded-wait path (see moe_set_test_stall in include/moe.h)."""
+    return load().moe_set_test_stall(1 if enable else 0)
+
+
+def set_gemm_policy(policy: int) -> int:
+    """GEMM_AUTO (per-GEMM choice), GEMM_SINGLE (128-row tiles) or GEMM_PAIR (CTA-pair 256x256 tiles)."""
+    old = load().moe_set_gemm_policy(policy)
+    if old < 0:
+        raise ValueError(f"unknown GEMM policy {policy}")
+    return old
 
 
 def moe_route(shape: Shape, logits, topk_idx, topk_gate, ws, stream=None):

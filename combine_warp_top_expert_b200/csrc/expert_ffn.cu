@@ -21,17 +21,23 @@
  * Inside a group the 128-row m-tiles are the inner index, so consecutive tiles
  * (running on neighbouring SMs at the same time) share one weight tile in L2.
  *
- * CTA = 6 warps: warp 0 issues TMA loads (one thread), warp 1 allocates TMEM
- * and issues tcgen05.mma (one thread), warps 2-5 drain the accumulator
- * (tcgen05.ld) and run the epilogue. 4-stage shared-memory ring (A 128x64 +
- * B 256x64 bf16 per stage, 128-byte swizzle), two TMEM accumulators of 128 x
- * 256 fp32 so the epilogue of tile i overlaps the main loop of tile i+1.
+ * Two tile shapes, same roles (warp 0 issues TMA loads from one thread, warp 1
+ * owns TMEM and issues tcgen05.mma from one thread, warps 2-5 drain the
+ * accumulator with tcgen05.ld and run the epilogue), two TMEM accumulators of
+ * 256 fp32 columns so the epilogue of tile i overlaps the main loop of tile i+1:
+ *   pair   (default) a cluster of 2 CTAs on neighbouring SMs computes a 256 x 256
+ *          tile with cta_group::2 MMAs: each CTA stages its own 128 rows of A
+ *          and 128 of the 256 rows of B (6-stage ring of 32 KB), so each SM moves
+ *          32 KB of operands per 64-deep K step instead of 48 KB;
+ *   single one CTA computes a 128 x 256 (GEMM1) or 128 x BN (GEMM2) tile with
+ *          cta_group::1 MMAs (4-stage ring of 48 KB); used for GEMM2 when d is
+ *          not a multiple of 256.
  * GEMM1's B tile stacks 128 gate rows over the matching 128 up rows, so one
  * N=256 MMA yields both halves of the SwiGLU for 128 output columns and the
  * epilogue combines them before anything leaves the SM.
- * The hidden rows h live in the workspace, padded to 128 rows per expert, so
- * GEMM1 stores whole tiles and GEMM2 loads whole tiles; GEMM2 masks its stores
- * to the expert's real rows.
+ * The hidden rows h live in the workspace, each group's rows padded to a
+ * multiple of 256, so GEMM1 stores whole tiles and GEMM2 loads whole tiles with
+ * either tile shape; GEMM2 masks its stores to the group's real rows.
  *
  * Every mbarrier wait is bounded (MOE_DEV_TIMEOUT on expiry); on abort each
  * role stops issuing, waits for its in-flight copies / MMAs, and the CTA frees
@@ -39,6 +45,8 @@
  */
 #include <cudaTypedefs.h>
 
+#include <atomic>
+#include <cstdio>
 #include <mutex>
 
 #include "moe_device.cuh"
@@ -47,25 +55,11 @@ namespace moe {
 
 namespace {
 
-constexpr int BM = 128;
 constexpr int BK = 64; /* bf16 elements = 128 bytes = one swizzle row */
-constexpr int STAGES = 4;
 constexpr int kThreads = 192;
-constexpr uint32_t A_BYTES = BM * BK * 2;
+constexpr int kHPad = 256; /* h rows per group are padded to a multiple of this */
 constexpr uint64_t kDrainNs = 2000000000ull;
-
-template <int MODE, int BN>
-struct Cfg {
-  static constexpr int B_ROWS = (MODE == 0) ? 256 : BN; /* rows of W per tile (N of the MMA) */
-  static constexpr int N_OUT = (MODE == 0) ? 128 : BN;  /* output columns per tile */
-  static constexpr uint32_t B_BYTES = (uint32_t)B_ROWS * BK * 2;
-  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr uint32_t ACC_COLS = B_ROWS;
-  static constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
-  static constexpr uint32_t IDESC = umma_idesc_bf16(BM, B_ROWS);
-  static constexpr size_t SMEM_BYTES = 1024 /* alignment slack */ + (size_t)STAGES * STAGE_BYTES + 4096;
-  static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
-};
+constexpr uint32_t HALF_TILE = 128 * BK * 2; /* 16 KB: 128 rows x 64 bf16 */
 
 struct FfnParams {
   const int32_t* expert_offsets; /* [E+1] */
@@ -73,68 +67,81 @@ struct FfnParams {
   int n_shared;
   int64_t T;
   int64_t A;
-  int K;           /* reduction length: d (GEMM1) or f (GEMM2) */
-  int n_tiles_n;   /* output column tiles */
+  int K;          /* reduction length: d (GEMM1) or f (GEMM2) */
+  int n_tiles_n;  /* output column tiles */
   int f;
   int d;
-  uint16_t* out0;  /* GEMM1: h; GEMM2: y_perm */
-  uint16_t* out1;  /* GEMM2: y_shared */
-  int64_t ld_out;  /* row stride of the output in elements */
+  uint16_t* out0; /* GEMM1: h; GEMM2: y_perm */
+  uint16_t* out1; /* GEMM2: y_shared */
+  int64_t ld_out; /* row stride of the output in elements */
   uint32_t* status;
   uint64_t timeout_ns;
+  int stall_first_stage; /* test hook: arm the first stage of each CTA's first tile but never load it */
 };
 
 struct Tile {
   int g;           /* group: expert index, or E for the shared expert */
   int m, n;        /* m-tile inside the group, n-tile */
-  int valid;       /* real rows in this m-tile (<= 128) */
+  int valid;       /* real rows in this m-tile (<= TM) */
   int a_row;       /* first A row (TMA coordinate) */
   int b_row;       /* first B row (TMA coordinate); GEMM1: the gate rows */
   int64_t out_row; /* first output row */
 };
 
-/* Shared-memory schedule: s_mpref[g] = m-tiles of groups < g (prefix, G+1 entries);
- * s_off = expert_offsets. */
-__device__ __forceinline__ bool build_schedule(const FfnParams& p, int32_t* s_off, int32_t* s_mpref, int lane) {
+/* Shared-memory schedule, built by one warp: s_off = expert_offsets,
+ * s_mpref[g] = m-tiles (TM rows) of groups < g, s_hpref[g] = 256-row blocks of h
+ * of groups < g. Returns false if expert_offsets is inconsistent. */
+template <int TM>
+__device__ __forceinline__ bool build_schedule(const FfnParams& p, int32_t* s_off, int32_t* s_mpref, int32_t* s_hpref,
+                                               int lane) {
   const int E = p.E;
   const int G = E + p.n_shared;
   bool ok = true;
   for (int i = lane; i <= E; i += 32) s_off[i] = __ldg(p.expert_offsets + i);
   __syncwarp();
-  int carry = 0;
+  int carry_m = 0, carry_h = 0;
   for (int base = 0; base < G; base += 32) {
     const int g = base + lane;
-    int mt = 0;
+    int rows = 0;
     if (g < E) {
       const int lo = s_off[g], hi = s_off[g + 1];
       if (lo < 0 || hi < lo || hi > p.A) ok = false;
-      mt = (max(0, hi - lo) + BM - 1) / BM;
+      rows = max(0, hi - lo);
     } else if (g < G) {
-      mt = (int)((p.T + BM - 1) / BM);
+      rows = (int)p.T;
     }
-    int incl = mt;
+    int im = (rows + TM - 1) / TM, ih = (rows + kHPad - 1) / kHPad;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-      if (lane >= o) incl += y;
+      const int ym = __shfl_up_sync(0xFFFFFFFFu, im, o);
+      const int yh = __shfl_up_sync(0xFFFFFFFFu, ih, o);
+      if (lane >= o) {
+        im += ym;
+        ih += yh;
+      }
     }
-    if (g < G) s_mpref[g + 1] = carry + incl;
-    carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    if (g < G) {
+      s_mpref[g + 1] = carry_m + im;
+      s_hpref[g + 1] = carry_h + ih;
+    }
+    carry_m += __shfl_sync(0xFFFFFFFFu, im, 31);
+    carry_h += __shfl_sync(0xFFFFFFFFu, ih, 31);
   }
   if (lane == 0) {
     s_mpref[0] = 0;
+    s_hpref[0] = 0;
     if (s_off[0] != 0) ok = false;
   }
-  ok = __all_sync(0xFFFFFFFFu, ok);
-  return ok;
+  return __all_sync(0xFFFFFFFFu, ok);
 }
 
-template <int MODE, int BN>
+/* Linear tile index -> tile. Inside a group the m-tiles are the inner index. */
+template <int MODE, int TM, int BN>
 __device__ __forceinline__ Tile decode_tile(int64_t L, const FfnParams& p, const int32_t* s_off,
-                                            const int32_t* s_mpref) {
+                                            const int32_t* s_mpref, const int32_t* s_hpref) {
   const int G = p.E + p.n_shared;
   const int q = (int)(L / p.n_tiles_n); /* s_mpref[g] <= q < s_mpref[g+1] */
-  int lo = 0, hi = G;                   /* find the last g with s_mpref[g] <= q */
+  int lo = 0, hi = G;                   /* the last g with s_mpref[g] <= q */
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (s_mpref[mid] <= q)
@@ -150,57 +157,124 @@ __device__ __forceinline__ Tile decode_tile(int64_t L, const FfnParams& p, const
   t.m = local - t.n * mt;
   const bool shared = lo >= p.E;
   const int rows = shared ? (int)p.T : s_off[lo + 1] - s_off[lo];
-  t.valid = min(BM, rows - t.m * BM);
-  const int hrow = (s_mpref[lo] + t.m) * BM;
+  t.valid = min(TM, rows - t.m * TM);
+  const int hrow = s_hpref[lo] * kHPad + t.m * TM;
   if (MODE == 0) {
-    t.a_row = shared ? t.m * BM : s_off[lo] + t.m * BM;
+    t.a_row = shared ? t.m * TM : s_off[lo] + t.m * TM;
     t.b_row = shared ? t.n * 128 : lo * 2 * p.f + t.n * 128;
     t.out_row = hrow;
   } else {
     t.a_row = hrow;
     t.b_row = shared ? t.n * BN : lo * p.d + t.n * BN;
-    t.out_row = shared ? (int64_t)t.m * BM : (int64_t)s_off[lo] + t.m * BM;
+    t.out_row = shared ? (int64_t)t.m * TM : (int64_t)s_off[lo] + t.m * TM;
   }
   return t;
 }
 
 __device__ __forceinline__ float silu_f(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
 
+/* Epilogue of one accumulator row held by this thread: `taddr` addresses this
+ * warp's TMEM lane quarter at the accumulator's first column, `r` is the row
+ * inside the tile. GEMM1: h = silu(gate) * up -> bf16, 128 columns (always
+ * stored: h is padded). GEMM2: bf16 of BN columns, stored if r < valid. */
+template <int MODE, int BN>
+__device__ __forceinline__ void epilogue_row(const FfnParams& p, const Tile& t, uint32_t taddr, int r) {
+  if (MODE == 0) {
+    uint16_t* dst = p.out0 + (t.out_row + r) * p.ld_out + (int64_t)t.n * 128;
+#pragma unroll 1
+    for (int c0 = 0; c0 < 128; c0 += 16) {
+      uint32_t gr[16], ur[16];
+      tmem_ld16(taddr + c0, gr);
+      tmem_ld16(taddr + 128 + c0, ur);
+      tmem_ld_wait();
+      uint32_t hw[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float h0 = silu_f(__uint_as_float(gr[2 * i])) * __uint_as_float(ur[2 * i]);
+        const float h1 = silu_f(__uint_as_float(gr[2 * i + 1])) * __uint_as_float(ur[2 * i + 1]);
+        hw[i] = pack_bf16x2(h0, h1);
+      }
+      st_v4(dst + c0, make_uint4(hw[0], hw[1], hw[2], hw[3]));
+      st_v4(dst + c0 + 8, make_uint4(hw[4], hw[5], hw[6], hw[7]));
+    }
+  } else {
+    const bool shared = t.g >= p.E;
+    uint16_t* dst = (shared ? p.out1 : p.out0) + (t.out_row + r) * p.ld_out + (int64_t)t.n * BN;
+    const bool live = r < t.valid;
+#pragma unroll 1
+    for (int c0 = 0; c0 < BN; c0 += 16) {
+      uint32_t vr[16];
+      tmem_ld16(taddr + c0, vr);
+      tmem_ld_wait();
+      if (live) {
+        uint32_t hw[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) hw[i] = pack_bf16x2(__uint_as_float(vr[2 * i]), __uint_as_float(vr[2 * i + 1]));
+        st_v4(dst + c0, make_uint4(hw[0], hw[1], hw[2], hw[3]));
+        st_v4(dst + c0 + 8, make_uint4(hw[4], hw[5], hw[6], hw[7]));
+      }
+    }
+  }
+}
+
+/* Shared-memory control block that follows the operand ring. */
+struct Ctrl {
+  uint64_t full[8];
+  uint64_t empty[8];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_slot;
+  int abort_flag;
+  int ok;
+  int32_t off[kMaxE + 2];
+  int32_t mpref[kMaxE + 2];
+  int32_t hpref[kMaxE + 2];
+};
+
+/* ======================= single-CTA tiles (128 x N) ======================== */
+
+template <int MODE, int BN>
+struct SingleCfg {
+  static constexpr int STAGES = 4;
+  static constexpr int B_ROWS = (MODE == 0) ? 256 : BN; /* rows of W per tile (N of the MMA) */
+  static constexpr uint32_t B_BYTES = (uint32_t)B_ROWS * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = HALF_TILE + B_BYTES;
+  static constexpr uint32_t ACC_COLS = B_ROWS;
+  static constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
+  static constexpr uint32_t IDESC = umma_idesc_bf16(128, B_ROWS);
+  static constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Ctrl);
+  static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
+};
+
 template <int MODE, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-                            const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
-                            const FfnParams p) {
-  using C = Cfg<MODE, BN>;
+    ffn_gemm_single_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                           const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+                           const FfnParams p) {
+  using C = SingleCfg<MODE, BN>;
+  constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   /* 128-byte swizzled tiles need 1024-byte aligned shared-space addresses */
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * C::B_BYTES);
-  uint64_t* empty = full + STAGES;
-  uint64_t* tfull = empty + STAGES;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* s_ok = reinterpret_cast<int*>(tmem_slot + 2);
-  int32_t* s_off = reinterpret_cast<int32_t*>(tmem_slot + 4);
-  int32_t* s_mpref = s_off + (kMaxE + 2);
+  uint8_t* sB = smem + STAGES * HALF_TILE;
+  Ctrl* ctl = reinterpret_cast<Ctrl*>(sB + STAGES * C::B_BYTES);
+  volatile int* s_abort = &ctl->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&ctl->tfull[b], 1);
+      mbar_init(&ctl->tempty[b], 4);
     }
-    mbar_init(drain, 1);
-    *s_abort = 0;
+    mbar_init(&ctl->drain, 1);
+    ctl->abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -210,21 +284,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmB1);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_alloc(&ctl->tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
   if (warp == 2) {
-    const bool ok = build_schedule(p, s_off, s_mpref, lane);
-    if (lane == 0) *s_ok = ok ? 1 : 0;
+    const bool ok = build_schedule<128>(p, ctl->off, ctl->mpref, ctl->hpref, lane);
+    if (lane == 0) ctl->ok = ok ? 1 : 0;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
 
-  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t tmem_base = ctl->tmem_slot;
   const int G = p.E + p.n_shared;
-  int64_t total = (int64_t)s_mpref[G] * p.n_tiles_n;
-  if (!*s_ok) {
+  int64_t total = (int64_t)ctl->mpref[G] * p.n_tiles_n;
+  if (!ctl->ok) {
     total = 0;
     if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(p.status, MOE_DEV_COUNT_MISMATCH);
   }
@@ -244,26 +318,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       bool abort = false;
       for (int64_t L = blockIdx.x; L < total && !abort; L += gridDim.x) {
-        const Tile t = decode_tile<MODE, BN>(L, p, s_off, s_mpref);
+        const Tile t = decode_tile<MODE, 128, BN>(L, p, ctl->off, ctl->mpref, ctl->hpref);
         const bool shared = t.g >= p.E;
         const CUtensorMap* mA = shared ? &tmA1 : &tmA0;
         const CUtensorMap* mB = shared ? &tmB1 : &tmB0;
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, p.timeout_ns, s_abort)) {
+          if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, p.timeout_ns, s_abort)) {
             abort = true;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          mbar_arrive_expect_tx(&ctl->full[stage], C::STAGE_BYTES);
+          if (p.stall_first_stage && L == blockIdx.x && kb == 0) {
+            /* test hook: this stage's bytes never arrive, so the MMA's bounded wait runs out */
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            continue;
+          }
           armed[stage] = true;
           armed_phase[stage] = phase;
-          uint8_t* a_dst = sA + stage * A_BYTES;
+          uint8_t* a_dst = sA + stage * HALF_TILE;
           uint8_t* b_dst = sB + stage * C::B_BYTES;
-          tma_load_2d(a_dst, mA, &full[stage], kb * BK, t.a_row);
+          tma_load_2d(a_dst, mA, &ctl->full[stage], kb * BK, t.a_row);
           if (MODE == 0) {
-            tma_load_2d(b_dst, mB, &full[stage], kb * BK, t.b_row);
-            tma_load_2d(b_dst + 128 * BK * 2, mB, &full[stage], kb * BK, t.b_row + p.f);
+            tma_load_2d(b_dst, mB, &ctl->full[stage], kb * BK, t.b_row);
+            tma_load_2d(b_dst + HALF_TILE, mB, &ctl->full[stage], kb * BK, t.b_row + p.f);
           } else {
-            tma_load_2d(b_dst, mB, &full[stage], kb * BK, t.b_row);
+            tma_load_2d(b_dst, mB, &ctl->full[stage], kb * BK, t.b_row);
           }
           if (++stage == STAGES) {
             stage = 0;
@@ -277,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       /* every armed stage's copies must land before the CTA may exit */
       for (int s = 0; s < STAGES; ++s)
-        if (armed[s]) mbar_wait(&full[s], armed_phase[s], kDrainNs, nullptr);
+        if (armed[s]) mbar_wait(&ctl->full[s], armed_phase[s], kDrainNs, nullptr);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -288,51 +370,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool abort = false;
       for (int64_t L = blockIdx.x; L < total && !abort; L += gridDim.x, ++acc) {
         const uint32_t b = acc & 1u, use = (acc >> 1) & 1u;
-        if (!mbar_wait(&tempty[b], use ^ 1u, p.timeout_ns, s_abort)) {
+        if (!mbar_wait(&ctl->tempty[b], use ^ 1u, p.timeout_ns, s_abort)) {
           abort = true;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + b * C::ACC_COLS;
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&full[stage], phase, p.timeout_ns, s_abort)) {
+          if (!mbar_wait(&ctl->full[stage], phase, p.timeout_ns, s_abort)) {
             abort = true;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
+          const uint32_t a_addr = smem_u32(sA + stage * HALF_TILE);
           const uint32_t b_addr = smem_u32(sB + stage * C::B_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             umma_bf16(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32), C::IDESC,
                       (kb | kk) != 0 ? 1u : 0u);
           }
-          umma_commit(&empty[stage]);
+          umma_commit(&ctl->empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (abort) break;
-        umma_commit(&tfull[b]);
+        umma_commit(&ctl->tfull[b]);
       }
       if (abort) {
         raise_status(p.status, MOE_DEV_TIMEOUT);
         *s_abort = 1;
       }
       /* all issued MMAs must finish before TMEM is released */
-      umma_commit(drain);
-      mbar_wait(drain, 0, kDrainNs, nullptr);
+      umma_commit(&ctl->drain);
+      mbar_wait(&ctl->drain, 0, kDrainNs, nullptr);
     }
   } else {
     /* ---------------- epilogue (warps 2..5, 128 threads) ---------------- */
     const int q = warp & 3; /* TMEM lane quarter this warp may access */
-    const int row = q * 32 + lane;
     uint32_t acc = 0;
     for (int64_t L = blockIdx.x; L < total; L += gridDim.x, ++acc) {
-      const Tile t = decode_tile<MODE, BN>(L, p, s_off, s_mpref);
+      const Tile t = decode_tile<MODE, 128, BN>(L, p, ctl->off, ctl->mpref, ctl->hpref);
       const uint32_t b = acc & 1u, use = (acc >> 1) & 1u;
-      if (!mbar_wait(&tfull[b], use, p.timeout_ns, s_abort)) {
+      if (!mbar_wait(&ctl->tfull[b], use, p.timeout_ns, s_abort)) {
         if (lane == 0) {
           raise_status(p.status, MOE_DEV_TIMEOUT);
           *s_abort = 1;
@@ -340,47 +421,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + b * C::ACC_COLS;
-      if (MODE == 0) {
-        uint16_t* dst = p.out0 + (t.out_row + row) * p.ld_out + (int64_t)t.n * 128;
-#pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 16) {
-          uint32_t gr[16], ur[16];
-          tmem_ld16(taddr + c0, gr);
-          tmem_ld16(taddr + 128 + c0, ur);
-          tmem_ld_wait();
-          uint32_t hw[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float h0 = silu_f(__uint_as_float(gr[2 * i])) * __uint_as_float(ur[2 * i]);
-            const float h1 = silu_f(__uint_as_float(gr[2 * i + 1])) * __uint_as_float(ur[2 * i + 1]);
-            hw[i] = pack_bf16x2(h0, h1);
-          }
-          st_v4(dst + c0, make_uint4(hw[0], hw[1], hw[2], hw[3]));
-          st_v4(dst + c0 + 8, make_uint4(hw[4], hw[5], hw[6], hw[7]));
-        }
-      } else {
-        const bool shared = t.g >= p.E;
-        uint16_t* base = shared ? p.out1 : p.out0;
-        uint16_t* dst = base + (t.out_row + row) * p.ld_out + (int64_t)t.n * BN;
-        const bool live = row < t.valid;
-#pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-          uint32_t vr[16];
-          tmem_ld16(taddr + c0, vr);
-          tmem_ld_wait();
-          if (live) {
-            uint32_t hw[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) hw[i] = pack_bf16x2(__uint_as_float(vr[2 * i]), __uint_as_float(vr[2 * i + 1]));
-            st_v4(dst + c0, make_uint4(hw[0], hw[1], hw[2], hw[3]));
-            st_v4(dst + c0 + 8, make_uint4(hw[4], hw[5], hw[6], hw[7]));
-          }
-        }
-      }
+      epilogue_row<MODE, BN>(p, t, tmem_base + ((uint32_t)(q * 32) << 16) + b * C::ACC_COLS, q * 32 + lane);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[b]);
+      if (lane == 0) mbar_arrive(&ctl->tempty[b]);
     }
   }
 
@@ -389,6 +433,241 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+/* ================= CTA-pair tiles (256 x 256, cta_group::2) ================= */
+
+struct PairCfg {
+  static constexpr int STAGES = 6;
+  static constexpr uint32_t STAGE_BYTES = 2 * HALF_TILE;       /* per CTA: 128 rows of A + 128 rows of B */
+  static constexpr uint32_t STAGE_TX = 2 * STAGE_BYTES;        /* bytes landing per stage in both CTAs */
+  static constexpr uint32_t ACC_COLS = 256;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t IDESC = umma_idesc_bf16(256, 256);
+  static constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Ctrl);
+};
+
+/* A cluster of two CTAs (ranks 0 and 1) works on one 256-row x 256-column tile:
+ * rank r stages A rows [r*128, r*128+128) of the tile and B rows
+ * [r*128, r*128+128) of the 256 (GEMM1: r = 0 the gate rows, r = 1 the up rows),
+ * and holds accumulator rows [r*128, r*128+128) in its own TMEM. Rank 0 arms the
+ * stage barrier for the bytes of both CTAs and issues the MMAs; its commits
+ * arrive on the barriers of both CTAs; rank 1's epilogue releases accumulators
+ * on rank 0's barrier. */
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    ffn_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                         const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+                         const FfnParams p) {
+  using C = PairCfg;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * HALF_TILE;
+  Ctrl* ctl = reinterpret_cast<Ctrl*>(sB + STAGES * HALF_TILE);
+  volatile int* s_abort = &ctl->abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctl->tfull[b], 1);
+      mbar_init(&ctl->tempty[b], 8); /* 4 epilogue warps in each CTA */
+    }
+    mbar_init(&ctl->drain, 1);
+    ctl->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA0);
+    tma_prefetch_desc(&tmA1);
+    tma_prefetch_desc(&tmB0);
+    tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&ctl->tmem_slot, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  if (warp == 2) {
+    const bool ok = build_schedule<256>(p, ctl->off, ctl->mpref, ctl->hpref, lane);
+    if (lane == 0) ctl->ok = ok ? 1 : 0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync(); /* both CTAs' barriers are initialised before any remote arrive */
+  tc_fence_after();
+
+  const uint32_t tmem_base = ctl->tmem_slot;
+  const int G = p.E + p.n_shared;
+  int64_t total = (int64_t)ctl->mpref[G] * p.n_tiles_n;
+  if (!ctl->ok) {
+    total = 0;
+    if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(p.status, MOE_DEV_COUNT_MISMATCH);
+  }
+  const int KB = p.K / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      /* ---------------- TMA producer (both CTAs) ---------------- */
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed_phase[STAGES];
+      bool armed[STAGES];
+#pragma unroll
+      for (int s = 0; s < STAGES; ++s) {
+        armed[s] = false;
+        armed_phase[s] = 0;
+      }
+      bool abort = false;
+      for (int64_t L = pair; L < total && !abort; L += npairs) {
+        const Tile t = decode_tile<MODE, 256, 256>(L, p, ctl->off, ctl->mpref, ctl->hpref);
+        const bool shared = t.g >= p.E;
+        const CUtensorMap* mA = shared ? &tmA1 : &tmA0;
+        const CUtensorMap* mB = shared ? &tmB1 : &tmB0;
+        const int a_row = t.a_row + (int)rank * 128;
+        const int b_row = (MODE == 0) ? t.b_row + (int)rank * p.f : t.b_row + (int)rank * 128;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, p.timeout_ns, s_abort)) {
+            abort = true;
+            break;
+          }
+          const bool stall = p.stall_first_stage && L == pair && kb == 0;
+          if (leader) {
+            mbar_arrive_expect_tx(&ctl->full[stage], C::STAGE_TX);
+            armed[stage] = !stall;
+            armed_phase[stage] = phase;
+          }
+          if (stall) {
+            /* test hook: this stage's bytes never arrive, so the MMA's bounded wait runs out */
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            continue;
+          }
+          const uint32_t full_leader = mapa_shared(smem_u32(&ctl->full[stage]), 0);
+          tma_load_2d_pair(sA + stage * HALF_TILE, mA, full_leader, kb * BK, a_row);
+          tma_load_2d_pair(sB + stage * HALF_TILE, mB, full_leader, kb * BK, b_row);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!abort) {
+        /* wait until the MMAs have released every stage this CTA filled, so no
+         * commit is still on its way to this CTA's barriers when it exits */
+        for (int i = 0; i < STAGES; ++i) {
+          if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, p.timeout_ns, s_abort)) {
+            abort = true;
+            break;
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (abort) {
+        raise_status(p.status, MOE_DEV_TIMEOUT);
+        *s_abort = 1;
+      }
+      /* the leader's stage barriers count both CTAs' copies: wait for them to land */
+      for (int s = 0; s < STAGES; ++s)
+        if (armed[s]) mbar_wait(&ctl->full[s], armed_phase[s], kDrainNs, nullptr);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      /* ---------------- MMA issuer (rank 0) ---------------- */
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t acc = 0;
+      bool abort = false;
+      for (int64_t L = pair; L < total && !abort; L += npairs, ++acc) {
+        const uint32_t b = acc & 1u, use = (acc >> 1) & 1u;
+        if (!mbar_wait(&ctl->tempty[b], use ^ 1u, p.timeout_ns, s_abort)) {
+          abort = true;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + b * C::ACC_COLS;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&ctl->full[stage], phase, p.timeout_ns, s_abort)) {
+            abort = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * HALF_TILE);
+          const uint32_t b_addr = smem_u32(sB + stage * HALF_TILE);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            umma_bf16_pair(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32), C::IDESC,
+                           (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit_pair_mc(&ctl->empty[stage], 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (abort) break;
+        umma_commit_pair_mc(&ctl->tfull[b], 0x3);
+      }
+      if (!abort) {
+        /* both CTAs' epilogues have released both accumulators (so no remote
+         * arrive is still on its way to this CTA) */
+        for (int i = 0; i < 2; ++i, ++acc) {
+          if (!mbar_wait(&ctl->tempty[acc & 1u], ((acc >> 1) & 1u) ^ 1u, p.timeout_ns, s_abort)) {
+            abort = true;
+            break;
+          }
+        }
+      }
+      if (abort) {
+        raise_status(p.status, MOE_DEV_TIMEOUT);
+        *s_abort = 1;
+      }
+      umma_commit_pair(&ctl->drain);
+      mbar_wait(&ctl->drain, 0, kDrainNs, nullptr);
+    }
+  } else {
+    /* ---------------- epilogue (warps 2..5 of both CTAs) ---------------- */
+    const int q = warp & 3;
+    uint32_t acc = 0;
+    for (int64_t L = pair; L < total; L += npairs, ++acc) {
+      const Tile t = decode_tile<MODE, 256, 256>(L, p, ctl->off, ctl->mpref, ctl->hpref);
+      const uint32_t b = acc & 1u, use = (acc >> 1) & 1u;
+      if (!mbar_wait(&ctl->tfull[b], use, p.timeout_ns, s_abort)) {
+        if (lane == 0) {
+          raise_status(p.status, MOE_DEV_TIMEOUT);
+          *s_abort = 1;
+        }
+        break;
+      }
+      tc_fence_after();
+      epilogue_row<MODE, 256>(p, t, tmem_base + ((uint32_t)(q * 32) << 16) + b * C::ACC_COLS,
+                              (int)rank * 128 + q * 32 + lane);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&ctl->tempty[b]), 0));
+    }
+  }
+
+  __syncthreads();
+  cluster_sync(); /* neither CTA releases TMEM or exits while its peer still works */
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
   }
 }
 
@@ -422,18 +701,89 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uin
 }
 
 template <int MODE, int BN>
-cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0, const CUtensorMap& b1,
-                        const FfnParams& p, cudaStream_t stream) {
-  using C = Cfg<MODE, BN>;
+cudaError_t launch_single(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0, const CUtensorMap& b1,
+                          const FfnParams& p, cudaStream_t stream) {
+  using C = SingleCfg<MODE, BN>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(grouped_ffn_gemm_kernel<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr_err = cudaFuncSetAttribute(ffn_gemm_single_kernel<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  grouped_ffn_gemm_kernel<MODE, BN><<<num_sms(), kThreads, C::SMEM_BYTES, stream>>>(a0, a1, b0, b1, p);
+  ffn_gemm_single_kernel<MODE, BN><<<num_sms(), kThreads, C::SMEM_BYTES, stream>>>(a0, a1, b0, b1, p);
   return cudaGetLastError();
+}
+
+/* Number of CTA pairs that can be resident at once (per device, cached). */
+template <int MODE>
+int pair_clusters() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * (unsigned)num_sms(), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = PairCfg::SMEM_BYTES;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaOccupancyMaxActiveClusters(&n, ffn_gemm_pair_kernel<MODE>, &cfg) != cudaSuccess) n = 0;
+  if (n > num_sms() / 2) n = num_sms() / 2;
+  if (n > 0) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+template <int MODE>
+cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0, const CUtensorMap& b1,
+                        const FfnParams& p, cudaStream_t stream, bool* launched) {
+  *launched = false;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(ffn_gemm_pair_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)PairCfg::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const int clusters = pair_clusters<MODE>();
+  if (debug_log()) std::fprintf(stderr, "[moe] pair GEMM%d: %d resident clusters of 2 CTAs\n", MODE + 1, clusters);
+  if (clusters <= 0) return cudaSuccess; /* caller falls back to single-CTA tiles */
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * (unsigned)clusters, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = PairCfg::SMEM_BYTES;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, ffn_gemm_pair_kernel<MODE>, a0, a1, b0, b1, p);
+  if (e == cudaSuccess) *launched = true;
+  return e;
+}
+
+FfnParams base_params(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const int32_t* expert_offsets) {
+  FfnParams p;
+  p.expert_offsets = expert_offsets;
+  p.E = s.E;
+  p.n_shared = s.n_shared;
+  p.T = s.T;
+  p.A = L.A;
+  p.f = s.f;
+  p.d = s.d;
+  p.status = reinterpret_cast<uint32_t*>(ws + L.status);
+  p.timeout_ns = wait_timeout_ns();
+  p.stall_first_stage = test_stall() ? 1 : 0;
+  return p;
 }
 
 }  // namespace
@@ -443,29 +793,28 @@ cudaError_t launch_gate_up(const moe_shape_t& s, const WsLayout& L, uint8_t* ws,
                            const uint16_t* w13s, cudaStream_t stream) {
   if (s.T == 0) return cudaSuccess;
   const bool sh = s.n_shared != 0;
+  /* 128-row single-CTA tiles pad small experts less and measured faster for this GEMM's
+   * short K; CTA-pair tiles only on request */
+  const bool pair = gemm_policy() == kGemmPair;
   CUtensorMap a0, a1, b0, b1;
   /* A = x_perm [A, d] (routed) / x [T, d] (shared); B = w13 [E*2f, d] / w13s [2f, d] */
-  if (!make_map(&a0, x_perm, (uint64_t)L.A, s.d, BM)) return cudaErrorInvalidValue;
-  if (!make_map(&a1, sh ? x : x_perm, sh ? (uint64_t)s.T : (uint64_t)L.A, s.d, BM)) return cudaErrorInvalidValue;
+  if (!make_map(&a0, x_perm, (uint64_t)L.A, s.d, 128)) return cudaErrorInvalidValue;
+  if (!make_map(&a1, sh ? x : x_perm, sh ? (uint64_t)s.T : (uint64_t)L.A, s.d, 128)) return cudaErrorInvalidValue;
   if (!make_map(&b0, w13, (uint64_t)s.E * 2 * s.f, s.d, 128)) return cudaErrorInvalidValue;
   if (!make_map(&b1, sh ? w13s : w13, sh ? (uint64_t)2 * s.f : (uint64_t)s.E * 2 * s.f, s.d, 128))
     return cudaErrorInvalidValue;
-  FfnParams p;
-  p.expert_offsets = expert_offsets;
-  p.E = s.E;
-  p.n_shared = s.n_shared;
-  p.T = s.T;
-  p.A = L.A;
-  p.f = s.f;
-  p.d = s.d;
-  p.status = reinterpret_cast<uint32_t*>(ws + L.status);
-  p.timeout_ns = wait_timeout_ns();
+  FfnParams p = base_params(s, L, ws, expert_offsets);
   p.K = s.d;
   p.n_tiles_n = s.f / 128;
   p.out0 = reinterpret_cast<uint16_t*>(ws + L.h);
   p.out1 = nullptr;
   p.ld_out = s.f;
-  return launch_gemm<0, 256>(a0, a1, b0, b1, p, stream);
+  if (pair) {
+    bool launched = false;
+    const cudaError_t e = launch_pair<0>(a0, a1, b0, b1, p, stream, &launched);
+    if (e != cudaSuccess || launched) return e;
+  }
+  return launch_single<0, 256>(a0, a1, b0, b1, p, stream);
 }
 
 cudaError_t launch_down(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const int32_t* expert_offsets,
@@ -474,28 +823,32 @@ cudaError_t launch_down(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, co
   if (s.T == 0) return cudaSuccess;
   const bool sh = s.n_shared != 0;
   const bool bn256 = (s.d % 256) == 0;
+  /* CTA-pair tiles when every expert averages >= 1024 rows (little 256-row padding) */
+  const bool pair = bn256 && (gemm_policy() == kGemmPair ||
+                              (gemm_policy() == kGemmAuto && L.A >= (int64_t)1024 * s.E));
   const uint32_t bn = bn256 ? 256 : 128;
+  const uint32_t b_box = pair ? 128 : bn;
   CUtensorMap a0, b0, b1;
   /* A = h [h_rows, f] (workspace); B = w2 [E*d, f] / w2s [d, f] */
-  if (!make_map(&a0, ws + L.h, (uint64_t)L.h_rows, s.f, BM)) return cudaErrorInvalidValue;
-  if (!make_map(&b0, w2, (uint64_t)s.E * s.d, s.f, bn)) return cudaErrorInvalidValue;
-  if (!make_map(&b1, sh ? w2s : w2, sh ? (uint64_t)s.d : (uint64_t)s.E * s.d, s.f, bn)) return cudaErrorInvalidValue;
-  FfnParams p;
-  p.expert_offsets = expert_offsets;
-  p.E = s.E;
-  p.n_shared = s.n_shared;
-  p.T = s.T;
-  p.A = L.A;
-  p.f = s.f;
-  p.d = s.d;
-  p.status = reinterpret_cast<uint32_t*>(ws + L.status);
-  p.timeout_ns = wait_timeout_ns();
+  if (!make_map(&a0, ws + L.h, (uint64_t)L.h_rows, s.f, 128)) return cudaErrorInvalidValue;
+  if (!make_map(&b0, w2, (uint64_t)s.E * s.d, s.f, b_box)) return cudaErrorInvalidValue;
+  if (!make_map(&b1, sh ? w2s : w2, sh ? (uint64_t)s.d : (uint64_t)s.E * s.d, s.f, b_box))
+    return cudaErrorInvalidValue;
+  FfnParams p = base_params(s, L, ws, expert_offsets);
   p.K = s.f;
   p.n_tiles_n = s.d / (int)bn;
   p.out0 = y_perm;
   p.out1 = sh ? y_shared : nullptr;
   p.ld_out = s.d;
-  return bn256 ? launch_gemm<1, 256>(a0, a0, b0, b1, p, stream) : launch_gemm<1, 128>(a0, a0, b0, b1, p, stream);
+  if (pair) {
+    bool launched = false;
+    const cudaError_t e = launch_pair<1>(a0, a0, b0, b1, p, stream, &launched);
+    if (e != cudaSuccess || launched) return e;
+    if (!make_map(&b0, w2, (uint64_t)s.E * s.d, s.f, bn)) return cudaErrorInvalidValue;
+    if (!make_map(&b1, sh ? w2s : w2, sh ? (uint64_t)s.d : (uint64_t)s.E * s.d, s.f, bn))
+      return cudaErrorInvalidValue;
+  }
+  return bn256 ? launch_single<1, 256>(a0, a0, b0, b1, p, stream) : launch_single<1, 128>(a0, a0, b0, b1, p, stream);
 }
 
 }  // namespace moe

@@ -6,6 +6,7 @@
  */
 #include <atomic>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 
 #include "moe_internal.h"
@@ -16,6 +17,8 @@ namespace {
 
 thread_local char g_last_cuda_error[256] = "";
 std::atomic<uint64_t> g_wait_timeout_ns{kDefaultWaitNs};
+std::atomic<int> g_gemm_policy{kGemmAuto};
+std::atomic<int> g_test_stall{0};
 
 }  // namespace
 
@@ -57,8 +60,9 @@ WsLayout ws_layout(const moe_shape_t& s) {
   L.A = (int64_t)s.T * s.k;
   L.tok_per_chunk = s.k > 0 ? (kChunkAssign / s.k > 0 ? kChunkAssign / s.k : 1) : 1;
   L.n_chunks = (s.T + L.tok_per_chunk - 1) / L.tok_per_chunk;
-  L.mt_routed_max = L.A / kTileM + (L.A < s.E ? L.A : s.E);
-  L.h_rows = (int64_t)kTileM * (L.mt_routed_max + (s.n_shared ? (s.T + kTileM - 1) / kTileM : 0));
+  /* sum_e ceil(n_e / 256) <= floor(A / 256) + (number of non-empty experts) */
+  L.mt_routed_max = L.A / kHPadRows + (L.A < s.E ? L.A : s.E);
+  L.h_rows = (int64_t)kHPadRows * (L.mt_routed_max + (s.n_shared ? (s.T + kHPadRows - 1) / kHPadRows : 0));
   size_t off = 256;
   L.status = 0;
   L.chunk = off;
@@ -85,6 +89,18 @@ int num_sms() {
 }
 
 uint64_t wait_timeout_ns() { return g_wait_timeout_ns.load(std::memory_order_relaxed); }
+
+int gemm_policy() { return g_gemm_policy.load(std::memory_order_relaxed); }
+
+bool test_stall() { return g_test_stall.load(std::memory_order_relaxed) != 0; }
+
+bool debug_log() {
+  static const bool on = [] {
+    const char* v = std::getenv("MOE_DEBUG");
+    return v && *v && *v != '0';
+  }();
+  return on;
+}
 
 }  // namespace moe
 
@@ -256,6 +272,13 @@ const char* moe_status_string(moe_status_t status) {
 }
 
 const char* moe_last_cuda_error(void) { return g_last_cuda_error; }
+
+int moe_set_gemm_policy(int policy) {
+  if (policy != kGemmAuto && policy != kGemmSingle && policy != kGemmPair) return -1;
+  return g_gemm_policy.exchange(policy, std::memory_order_relaxed);
+}
+
+int moe_set_test_stall(int enable) { return g_test_stall.exchange(enable ? 1 : 0, std::memory_order_relaxed); }
 
 uint64_t moe_set_wait_timeout_ns(uint64_t ns) {
   return g_wait_timeout_ns.exchange(ns ? ns : kDefaultWaitNs, std::memory_order_relaxed);

@@ -8,13 +8,16 @@
 #include <stddef.h>
 #include <stdint.h>
 
-#include "../../include/moe.h"
+#include "moe.h" /* include/ is on the include path */
 
 namespace moe {
 
 constexpr int kMaxE = 256;
 constexpr int kMaxK = 8;
-constexpr int kTileM = 128;           /* rows per grouped-GEMM tile (tcgen05 M) */
+constexpr int kHPadRows = 256;        /* h rows of each expert group are padded to a multiple of this */
+constexpr int kGemmAuto = 0;          /* grouped GEMM: tile shape chosen per GEMM from the shape */
+constexpr int kGemmSingle = 1;        /* grouped GEMM: single-CTA 128-row tiles only */
+constexpr int kGemmPair = 2;          /* grouped GEMM: CTA-pair 256-row tiles wherever they apply */
 constexpr int kChunkAssign = 2048;    /* assignments per dispatch histogram chunk */
 constexpr uint64_t kDefaultWaitNs = 2000000000ull; /* bounded-wait limit of the GEMM pipeline */
 
@@ -28,7 +31,7 @@ struct WsLayout {
   int64_t A = 0;          /* T * k */
   int64_t tok_per_chunk = 1;
   int64_t n_chunks = 0;
-  int64_t mt_routed_max = 0; /* upper bound of sum_e ceil(count_e / 128) */
+  int64_t mt_routed_max = 0; /* upper bound of sum_e ceil(count_e / 256) */
   int64_t h_rows = 0;
 };
 
@@ -44,6 +47,15 @@ moe_status_t cuda_fail(cudaError_t e);
 int num_sms();
 
 uint64_t wait_timeout_ns();
+
+/* Tile-shape policy of the grouped GEMM (kGemmAuto, kGemmSingle or kGemmPair). */
+int gemm_policy();
+
+/* Test hook: grouped-GEMM producers leave their first stage unloaded (see moe_set_test_stall). */
+bool test_stall();
+
+/* MOE_DEBUG set in the environment: launch configuration notes on stderr. */
+bool debug_log();
 
 cudaError_t launch_route(const float* logits, int32_t* topk_idx, float* topk_gate, int64_t T, int E, int k,
                          uint32_t* status, cudaStream_t stream);

@@ -229,6 +229,23 @@ const char* moe_last_cuda_error(void);
  * Returns the previous value. */
 uint64_t moe_set_wait_timeout_ns(uint64_t ns);
 
+/* Diagnostic knob: tile shape of the grouped GEMM for launches made after the
+ * call, process-wide. 0 (default) = chosen per GEMM from the shape: 128-row
+ * single-CTA tiles, except 256 x 256 tiles computed by a cluster of two CTAs on
+ * neighbouring SMs (cta_group::2) for the down GEMM when d % 256 == 0 and the
+ * experts average at least 1024 rows; 1 = 128-row single-CTA tiles only; 2 =
+ * CTA-pair tiles wherever they apply. Results are the same up to fp32 summation
+ * order. Returns the previous value, or -1 for an unknown policy (unchanged). */
+int moe_set_gemm_policy(int policy);
+
+/* Test hook for the bounded-wait path: while enabled (non-zero), every CTA of
+ * the grouped-GEMM launches made after the call arms its first pipeline stage
+ * but never loads it, so the MMA's wait on that stage runs out after the
+ * moe_set_wait_timeout_ns limit: MOE_DEV_TIMEOUT is set, the kernel drains its
+ * real copies and MMAs, frees its tensor memory and returns; outputs are
+ * incomplete. Never enable it outside tests. Returns the previous value. */
+int moe_set_test_stall(int enable);
+
 #ifdef __cplusplus
 }
 #endif

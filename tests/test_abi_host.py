@@ -37,12 +37,12 @@ def test_workspace_bytes_layout():
     n = moe.workspace_bytes(TINY)
     A = TINY.T * TINY.k
     chunks = -(-TINY.T // (2048 // TINY.k))
-    h_rows = 128 * (A // 128 + min(TINY.E, A))
+    h_rows = 256 * (A // 256 + min(TINY.E, A))
     expect = 256 + (-(-chunks * TINY.E * 4 // 256) * 256) + (-(-A * 4 // 256) * 256) + (-(-h_rows * TINY.f * 2 // 256) * 256)
     assert n == expect
     # shared expert adds its padded hidden rows
     sh = moe.Shape(T=256, d=512, E=8, k=2, f=1024, R=2, n_shared=1)
-    assert moe.workspace_bytes(sh) == n + 256 * TINY.f * 2
+    assert moe.workspace_bytes(sh) == n + 256 * TINY.f * 2   # ceil(256 / 256) blocks of 256 rows
     # empty batch still has the status header
     assert moe.workspace_bytes(moe.Shape(T=0, d=512, E=8, k=2, f=1024, R=2)) >= 256
     for bad in (moe.Shape(-1, 512, 8, 2, 1024, 2), moe.Shape(8, 512, 8, 9, 1024, 2), moe.Shape(8, 512, 8, 2, 1024, 3),
@@ -101,3 +101,9 @@ def test_status_strings_and_timeout_knob():
     assert old == 2_000_000_000
     assert lib.moe_set_wait_timeout_ns(0) == 12345
     assert lib.moe_set_wait_timeout_ns(0) == 2_000_000_000
+    assert lib.moe_set_gemm_policy(1) == 0
+    assert lib.moe_set_gemm_policy(7) == -1
+    assert lib.moe_set_gemm_policy(2) == 1
+    assert lib.moe_set_gemm_policy(0) == 2
+    assert lib.moe_set_test_stall(1) == 0
+    assert lib.moe_set_test_stall(0) == 1

@@ -1,0 +1,53 @@
+"""bench.py's multi-rank logic on CPU: world-size-2 gloo ranks (no GPU).
+
+With N GPUs the benchmark runs N independent replicas of the layer ("replicas
+only": the single-GPU path has no cross-GPU exchange). Each rank times its own
+steps; the reported value is all ranks' tokens over the slowest rank's time.
+"""
+import os
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _worker(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        local_ms = [250.0, 400.0][rank]            # rank 1 is the slower replica
+        mx = bench.max_over_ranks(local_ms, world)
+        value = bench.aggregate_throughput(4096, 20, world, mx / 1e3)
+        q.put((rank, mx, value, bench.replica_seed(0, rank)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_report_max_time_and_total_tokens():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + (os.getpid() % 1000)
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    for rank, mx, value, seed in res:
+        assert mx == 400.0                          # the slowest rank sets the time
+        assert value == pytest.approx(2 * 4096 * 20 / 0.4)
+        assert seed == rank                         # each replica gets its own batch
+
+
+def test_single_rank_is_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.5, 1) == 3.5
+    assert bench.aggregate_throughput(128, 10, 1, 2.0) == 640.0

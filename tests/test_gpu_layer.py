@@ -119,6 +119,15 @@ def test_layer_full_size_sampled_parity(name, n_tokens):
     torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("policy", [moe.GEMM_SINGLE, moe.GEMM_PAIR], ids=["single_tiles", "pair_tiles"])
+def test_layer_mixtral_sampled_parity_other_tiles(policy):
+    old = moe.set_gemm_policy(policy)
+    try:
+        test_layer_full_size_sampled_parity("mixtral_prefill", 4)
+    finally:
+        moe.set_gemm_policy(old)
+
+
 def test_empty_batch_is_a_no_op():
     wl = moe_synth.workload("tiny").with_(T=0)
     dv, layer, outs, status = _run_layer(wl)

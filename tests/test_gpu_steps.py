@@ -279,7 +279,15 @@ def _ffn_case(wl, idx=None):
         close(f64(bits(ys)), ys_ref, "y_shared")
 
 
-def test_expert_ffn_tiny():
+@pytest.fixture(params=[moe.GEMM_AUTO, moe.GEMM_SINGLE, moe.GEMM_PAIR], ids=["auto_tiles", "single_tiles",
+                                                                           "pair_tiles"])
+def gemm_policy(request):
+    old = moe.set_gemm_policy(request.param)
+    yield request.param
+    moe.set_gemm_policy(old)
+
+
+def test_expert_ffn_tiny(gemm_policy):
     _ffn_case(moe_synth.workload("tiny"))
 
 
@@ -293,11 +301,11 @@ def test_expert_ffn_tiny():
     # many experts, few rows each (decode-like)
     moe_synth.Workload("decode", T=16, d=256, E=64, k=8, f=256, R=8, n_shared=1, bias_kind="zipf", zipf_s=1.2),
 ])
-def test_expert_ffn_shapes(wl):
+def test_expert_ffn_shapes(wl, gemm_policy):
     _ffn_case(wl)
 
 
-def test_expert_ffn_with_empty_and_full_experts():
+def test_expert_ffn_with_empty_and_full_experts(gemm_policy):
     wl = moe_synth.Workload("emp", T=257, d=128, E=5, k=1, f=256, R=1)
     idx = np.zeros((257, 1), np.int32)
     idx[200:, 0] = 3          # experts 1, 2, 4 empty; expert 0 has 200 rows, expert 3 57
