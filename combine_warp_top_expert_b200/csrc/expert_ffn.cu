@@ -173,45 +173,111 @@ __device__ __forceinline__ Tile decode_tile(int64_t L, const FfnParams& p, const
 
 __device__ __forceinline__ float silu_f(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
 
-/* Epilogue of one accumulator row held by this thread: `taddr` addresses this
- * warp's TMEM lane quarter at the accumulator's first column, `r` is the row
- * inside the tile. GEMM1: h = silu(gate) * up -> bf16, 128 columns (always
- * stored: h is padded). GEMM2: bf16 of BN columns, stored if r < valid. */
+/* Per-warp epilogue staging: 32 rows x 64 bf16 (4 KB) in the 128-byte swizzled
+ * layout a TMA store with a {64, 32} box expects (16-byte chunk c of row r at
+ * chunk position c ^ (r % 8)). */
+constexpr uint32_t kStageBytesPerWarp = 32 * 128;
+constexpr uint32_t kEpiStagingBytes = 4 * kStageBytesPerWarp;
+
+__device__ __forceinline__ void stage_row_chunk(uint32_t sbase, int lane, int chunk, uint32_t a, uint32_t b,
+                                                uint32_t c, uint32_t d) {
+  st_shared_v4(sbase + (uint32_t)lane * 128u + ((uint32_t)(chunk ^ (lane & 7)) << 4), a, b, c, d);
+}
+
+/* Hand the warp's staged 32 x 64 block to TMA: all lanes' shared writes are made
+ * visible to the async proxy, then lane 0 issues the store. */
+__device__ __forceinline__ void store_staged_block(const CUtensorMap* map, uint8_t* stage, int32_t x, int32_t y,
+                                                   int lane) {
+  fence_proxy_async_shared();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(map, stage, x, y);
+    bulk_commit_group();
+  }
+}
+
+/* Before a warp overwrites its staging buffer, its previous TMA store must have read it. */
+__device__ __forceinline__ void staging_reusable(int lane) {
+  if (lane == 0) bulk_wait_read_all();
+  __syncwarp();
+}
+
+/* Epilogue of this warp's 32 accumulator rows. `taddr` addresses the warp's TMEM
+ * lane quarter at the accumulator's first column; `row0` is the warp's first row
+ * inside the tile (this thread's row is row0 + lane).
+ * GEMM1: h = silu(gate) * up -> bf16, 128 columns, always stored (h is padded),
+ *        as two TMA-stored 32 x 64 blocks.
+ * GEMM2: bf16 of BN columns; a warp whose 32 rows are all real stores TMA blocks,
+ *        a warp holding the expert's ragged end stores its real rows directly. */
 template <int MODE, int BN>
-__device__ __forceinline__ void epilogue_row(const FfnParams& p, const Tile& t, uint32_t taddr, int r) {
+__device__ __forceinline__ void epilogue_warp(const FfnParams& p, const Tile& t, uint32_t taddr, int row0, int lane,
+                                              uint8_t* stage, const CUtensorMap* out0, const CUtensorMap* out1) {
+  const uint32_t sbase = smem_u32(stage);
+  const int32_t grow = (int32_t)(t.out_row + row0); /* output row of lane 0 */
   if (MODE == 0) {
-    uint16_t* dst = p.out0 + (t.out_row + r) * p.ld_out + (int64_t)t.n * 128;
 #pragma unroll 1
-    for (int c0 = 0; c0 < 128; c0 += 16) {
-      uint32_t gr[16], ur[16];
-      tmem_ld16(taddr + c0, gr);
-      tmem_ld16(taddr + 128 + c0, ur);
-      tmem_ld_wait();
-      uint32_t hw[8];
+    for (int j = 0; j < 2; ++j) {
+      staging_reusable(lane);
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {
+        const int c = j * 64 + hh * 32;
+        uint32_t g0[16], g1[16], u0[16], u1[16];
+        tmem_ld16(taddr + c, g0);
+        tmem_ld16(taddr + c + 16, g1);
+        tmem_ld16(taddr + 128 + c, u0);
+        tmem_ld16(taddr + 128 + c + 16, u1);
+        tmem_ld_wait();
+        uint32_t w[16];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float h0 = silu_f(__uint_as_float(gr[2 * i])) * __uint_as_float(ur[2 * i]);
-        const float h1 = silu_f(__uint_as_float(gr[2 * i + 1])) * __uint_as_float(ur[2 * i + 1]);
-        hw[i] = pack_bf16x2(h0, h1);
+        for (int i = 0; i < 8; ++i) {
+          w[i] = pack_bf16x2(silu_f(__uint_as_float(g0[2 * i])) * __uint_as_float(u0[2 * i]),
+                             silu_f(__uint_as_float(g0[2 * i + 1])) * __uint_as_float(u0[2 * i + 1]));
+          w[8 + i] = pack_bf16x2(silu_f(__uint_as_float(g1[2 * i])) * __uint_as_float(u1[2 * i]),
+                                 silu_f(__uint_as_float(g1[2 * i + 1])) * __uint_as_float(u1[2 * i + 1]));
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          stage_row_chunk(sbase, lane, hh * 4 + q, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
       }
-      st_v4(dst + c0, make_uint4(hw[0], hw[1], hw[2], hw[3]));
-      st_v4(dst + c0 + 8, make_uint4(hw[4], hw[5], hw[6], hw[7]));
+      store_staged_block(out0, stage, t.n * 128 + j * 64, grow, lane);
     }
   } else {
     const bool shared = t.g >= p.E;
-    uint16_t* dst = (shared ? p.out1 : p.out0) + (t.out_row + r) * p.ld_out + (int64_t)t.n * BN;
-    const bool live = r < t.valid;
+    const CUtensorMap* map = shared ? out1 : out0;
+    const bool whole = row0 + 32 <= t.valid; /* warp-uniform */
+    const bool live = row0 + lane < t.valid;
+    uint16_t* dst = (shared ? p.out1 : p.out0) + (t.out_row + row0 + lane) * p.ld_out + (int64_t)t.n * BN;
 #pragma unroll 1
-    for (int c0 = 0; c0 < BN; c0 += 16) {
-      uint32_t vr[16];
-      tmem_ld16(taddr + c0, vr);
-      tmem_ld_wait();
-      if (live) {
-        uint32_t hw[8];
+    for (int j = 0; j < BN / 64; ++j) {
+      uint32_t v[4][16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) hw[i] = pack_bf16x2(__uint_as_float(vr[2 * i]), __uint_as_float(vr[2 * i + 1]));
-        st_v4(dst + c0, make_uint4(hw[0], hw[1], hw[2], hw[3]));
-        st_v4(dst + c0 + 8, make_uint4(hw[4], hw[5], hw[6], hw[7]));
+      for (int q = 0; q < 4; ++q) tmem_ld16(taddr + j * 64 + q * 16, v[q]);
+      tmem_ld_wait();
+      if (whole) {
+        staging_reusable(lane);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const uint32_t* r = &v[q][hf * 8];
+            stage_row_chunk(sbase, lane, q * 2 + hf, pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
+                            pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
+                            pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
+                            pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
+          }
+        store_staged_block(map, stage, t.n * BN + j * 64, grow, lane);
+      } else if (live) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const uint32_t* r = &v[q][hf * 8];
+            st_v4(dst + j * 64 + q * 16 + hf * 8,
+                  make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
+                             pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
+                             pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
+                             pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7]))));
+          }
       }
     }
   }
@@ -243,14 +309,16 @@ struct SingleCfg {
   static constexpr uint32_t ACC_COLS = B_ROWS;
   static constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
   static constexpr uint32_t IDESC = umma_idesc_bf16(128, B_ROWS);
-  static constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Ctrl);
+  static constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + kEpiStagingBytes + sizeof(Ctrl);
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 template <int MODE, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     ffn_gemm_single_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                            const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+                           const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
                            const FfnParams p) {
   using C = SingleCfg<MODE, BN>;
   constexpr int STAGES = C::STAGES;
@@ -259,7 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * HALF_TILE;
-  Ctrl* ctl = reinterpret_cast<Ctrl*>(sB + STAGES * C::B_BYTES);
+  uint8_t* sEpi = sB + STAGES * C::B_BYTES;
+  Ctrl* ctl = reinterpret_cast<Ctrl*>(sEpi + kEpiStagingBytes);
   volatile int* s_abort = &ctl->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -282,6 +351,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmA1);
     tma_prefetch_desc(&tmB0);
     tma_prefetch_desc(&tmB1);
+    tma_prefetch_desc(&tmO0);
+    tma_prefetch_desc(&tmO1);
   }
   if (warp == 1) {
     tmem_alloc(&ctl->tmem_slot, C::TMEM_COLS);
@@ -421,11 +492,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      epilogue_row<MODE, BN>(p, t, tmem_base + ((uint32_t)(q * 32) << 16) + b * C::ACC_COLS, q * 32 + lane);
+      epilogue_warp<MODE, BN>(p, t, tmem_base + ((uint32_t)(q * 32) << 16) + b * C::ACC_COLS, q * 32, lane,
+                              sEpi + q * kStageBytesPerWarp, &tmO0, &tmO1);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->tempty[b]);
     }
+    if (lane == 0) bulk_wait_all(); /* this warp's TMA stores are complete */
   }
 
   __syncthreads();
@@ -445,7 +518,8 @@ struct PairCfg {
   static constexpr uint32_t ACC_COLS = 256;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t IDESC = umma_idesc_bf16(256, 256);
-  static constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Ctrl);
+  static constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + kEpiStagingBytes + sizeof(Ctrl);
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 /* A cluster of two CTAs (ranks 0 and 1) works on one 256-row x 256-column tile:
@@ -459,6 +533,7 @@ template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     ffn_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                          const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+                         const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
                          const FfnParams p) {
   using C = PairCfg;
   constexpr int STAGES = C::STAGES;
@@ -466,7 +541,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * HALF_TILE;
-  Ctrl* ctl = reinterpret_cast<Ctrl*>(sB + STAGES * HALF_TILE);
+  uint8_t* sEpi = sB + STAGES * HALF_TILE;
+  Ctrl* ctl = reinterpret_cast<Ctrl*>(sEpi + kEpiStagingBytes);
   volatile int* s_abort = &ctl->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -492,6 +568,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmA1);
     tma_prefetch_desc(&tmB0);
     tma_prefetch_desc(&tmB1);
+    tma_prefetch_desc(&tmO0);
+    tma_prefetch_desc(&tmO1);
   }
   if (warp == 1) {
     tmem_alloc_pair(&ctl->tmem_slot, C::TMEM_COLS);
@@ -654,12 +732,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      epilogue_row<MODE, 256>(p, t, tmem_base + ((uint32_t)(q * 32) << 16) + b * C::ACC_COLS,
-                              (int)rank * 128 + q * 32 + lane);
+      epilogue_warp<MODE, 256>(p, t, tmem_base + ((uint32_t)(q * 32) << 16) + b * C::ACC_COLS,
+                               (int)rank * 128 + q * 32, lane, sEpi + q * kStageBytesPerWarp, &tmO0, &tmO1);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&ctl->tempty[b]), 0));
     }
+    if (lane == 0) bulk_wait_all(); /* this warp's TMA stores are complete */
   }
 
   __syncthreads();
@@ -702,7 +781,7 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uin
 
 template <int MODE, int BN>
 cudaError_t launch_single(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0, const CUtensorMap& b1,
-                          const FfnParams& p, cudaStream_t stream) {
+                          const CUtensorMap& o0, const CUtensorMap& o1, const FfnParams& p, cudaStream_t stream) {
   using C = SingleCfg<MODE, BN>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -711,7 +790,7 @@ cudaError_t launch_single(const CUtensorMap& a0, const CUtensorMap& a1, const CU
                                     (int)C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  ffn_gemm_single_kernel<MODE, BN><<<num_sms(), kThreads, C::SMEM_BYTES, stream>>>(a0, a1, b0, b1, p);
+  ffn_gemm_single_kernel<MODE, BN><<<num_sms(), kThreads, C::SMEM_BYTES, stream>>>(a0, a1, b0, b1, o0, o1, p);
   return cudaGetLastError();
 }
 
@@ -742,7 +821,8 @@ int pair_clusters() {
 
 template <int MODE>
 cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0, const CUtensorMap& b1,
-                        const FfnParams& p, cudaStream_t stream, bool* launched) {
+                        const CUtensorMap& o0, const CUtensorMap& o1, const FfnParams& p, cudaStream_t stream,
+                        bool* launched) {
   *launched = false;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -766,7 +846,7 @@ cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, ffn_gemm_pair_kernel<MODE>, a0, a1, b0, b1, p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, ffn_gemm_pair_kernel<MODE>, a0, a1, b0, b1, o0, o1, p);
   if (e == cudaSuccess) *launched = true;
   return e;
 }
@@ -803,6 +883,8 @@ cudaError_t launch_gate_up(const moe_shape_t& s, const WsLayout& L, uint8_t* ws,
   if (!make_map(&b0, w13, (uint64_t)s.E * 2 * s.f, s.d, 128)) return cudaErrorInvalidValue;
   if (!make_map(&b1, sh ? w13s : w13, sh ? (uint64_t)2 * s.f : (uint64_t)s.E * 2 * s.f, s.d, 128))
     return cudaErrorInvalidValue;
+  CUtensorMap o0; /* h [h_rows, f], stored as 32 x 64 blocks */
+  if (!make_map(&o0, ws + L.h, (uint64_t)L.h_rows, s.f, 32)) return cudaErrorInvalidValue;
   FfnParams p = base_params(s, L, ws, expert_offsets);
   p.K = s.d;
   p.n_tiles_n = s.f / 128;
@@ -811,10 +893,10 @@ cudaError_t launch_gate_up(const moe_shape_t& s, const WsLayout& L, uint8_t* ws,
   p.ld_out = s.f;
   if (pair) {
     bool launched = false;
-    const cudaError_t e = launch_pair<0>(a0, a1, b0, b1, p, stream, &launched);
+    const cudaError_t e = launch_pair<0>(a0, a1, b0, b1, o0, o0, p, stream, &launched);
     if (e != cudaSuccess || launched) return e;
   }
-  return launch_single<0, 256>(a0, a1, b0, b1, p, stream);
+  return launch_single<0, 256>(a0, a1, b0, b1, o0, o0, p, stream);
 }
 
 cudaError_t launch_down(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const int32_t* expert_offsets,
@@ -834,6 +916,9 @@ cudaError_t launch_down(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, co
   if (!make_map(&b0, w2, (uint64_t)s.E * s.d, s.f, b_box)) return cudaErrorInvalidValue;
   if (!make_map(&b1, sh ? w2s : w2, sh ? (uint64_t)s.d : (uint64_t)s.E * s.d, s.f, b_box))
     return cudaErrorInvalidValue;
+  CUtensorMap o0, o1; /* y_perm [A, d] and y_shared [T, d], stored as 32 x 64 blocks */
+  if (!make_map(&o0, y_perm, (uint64_t)L.A, s.d, 32)) return cudaErrorInvalidValue;
+  if (!make_map(&o1, sh ? y_shared : y_perm, sh ? (uint64_t)s.T : (uint64_t)L.A, s.d, 32)) return cudaErrorInvalidValue;
   FfnParams p = base_params(s, L, ws, expert_offsets);
   p.K = s.f;
   p.n_tiles_n = s.d / (int)bn;
@@ -842,13 +927,14 @@ cudaError_t launch_down(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, co
   p.ld_out = s.d;
   if (pair) {
     bool launched = false;
-    const cudaError_t e = launch_pair<1>(a0, a0, b0, b1, p, stream, &launched);
+    const cudaError_t e = launch_pair<1>(a0, a0, b0, b1, o0, o1, p, stream, &launched);
     if (e != cudaSuccess || launched) return e;
     if (!make_map(&b0, w2, (uint64_t)s.E * s.d, s.f, bn)) return cudaErrorInvalidValue;
     if (!make_map(&b1, sh ? w2s : w2, sh ? (uint64_t)s.d : (uint64_t)s.E * s.d, s.f, bn))
       return cudaErrorInvalidValue;
   }
-  return bn256 ? launch_single<1, 256>(a0, a0, b0, b1, p, stream) : launch_single<1, 128>(a0, a0, b0, b1, p, stream);
+  return bn256 ? launch_single<1, 256>(a0, a0, b0, b1, o0, o1, p, stream)
+               : launch_single<1, 128>(a0, a0, b0, b1, o0, o1, p, stream);
 }
 
 }  // namespace moe
