@@ -3,10 +3,11 @@
  *
  * Page "Expert Parallelism" (learning-materials IX.05) §4 COMBINE: "Send the
  * results back to the originating GPUs, in the original order. Weighted-sum the
- * k expert outputs per token." One warp per token: the k row indices and gates
- * are loaded once by lanes 0..k-1 and broadcast by shuffle; each lane then
- * streams 16-byte vectors of the k expert rows (+ the shared-expert row),
- * accumulates in fp32 in j order and stores one bf16 vector.
+ * k expert outputs per token." One warp per (token, column slice): the k row
+ * indices and gates are loaded by lanes 0..k-1 and broadcast by shuffle; each
+ * lane then streams 16-byte vectors of the k expert rows (+ the shared-expert
+ * row), accumulates in fp32 in j order and stores one bf16 vector. Slices keep
+ * every SM busy when T is small.
  *
  * Bytes per token: k*d*2 + (shared) d*2 read, d*2 written, k*8 of indices.
  */
@@ -16,18 +17,23 @@ namespace moe {
 
 namespace {
 
-template <int U>
-__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ y_perm,
+/* U vectors per lane per step, rows of up to KMAX experts in flight together. */
+template <int U, int KMAX>
+__global__ void __launch_bounds__(256, 2) combine_kernel(const uint16_t* __restrict__ y_perm,
                                                       const int32_t* __restrict__ assign_row,
                                                       const float* __restrict__ topk_gate,
                                                       const uint16_t* __restrict__ y_shared,
                                                       uint16_t* __restrict__ out, int64_t T, int d, int k,
-                                                      int64_t A, uint32_t* status) {
+                                                      int64_t A, int slices, int vps, uint32_t* status) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int nv = d >> 3;
+  const int64_t items = T * slices;
   bool bad = false;
-  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
+  for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < items; w += warps) {
+    const int64_t t = w / slices;
+    const int sl = (int)(w - t * slices);
+    const int v_end = min(nv, (sl + 1) * vps);
     int row = -1;
     float g = 0.0f;
     if (lane < k) {
@@ -38,67 +44,58 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
         row = -1;
       }
     }
-    int64_t src[kMaxK];
-    float gs[kMaxK];
+    int64_t src[KMAX];
+    float gs[KMAX];
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
+    for (int j = 0; j < KMAX; ++j) {
       const int r = __shfl_sync(0xFFFFFFFFu, row, j);
       gs[j] = __shfl_sync(0xFFFFFFFFu, g, j);
       src[j] = (j < k && r >= 0) ? (int64_t)r * d : -1;
     }
     const uint16_t* ysh = y_shared ? y_shared + t * d : nullptr;
     uint16_t* o = out + t * d;
-    for (int v0 = lane; v0 < nv; v0 += 32 * U) {
-      float acc[U][8];
+    for (int v0 = sl * vps + lane; v0 < v_end; v0 += 32 * U) {
+      uint4 wv[KMAX][U];
+      uint4 sv[U];
 #pragma unroll
-      for (int u = 0; u < U; ++u)
-#pragma unroll
-        for (int q = 0; q < 8; ++q) acc[u][q] = 0.0f;
-#pragma unroll
-      for (int j = 0; j < kMaxK; ++j) {
-        if (src[j] < 0) continue;
-        uint4 w[U];
+      for (int j = 0; j < KMAX; ++j)
 #pragma unroll
         for (int u = 0; u < U; ++u) {
           const int v = v0 + 32 * u;
-          if (v < nv) w[u] = ld_nc_v4(y_perm + src[j] + (int64_t)v * 8);
+          wv[j][u] = (src[j] >= 0 && v < v_end) ? ld_nc_v4(y_perm + src[j] + (int64_t)v * 8) : make_uint4(0, 0, 0, 0);
         }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const uint32_t ww[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            acc[u][2 * q] = fmaf(gs[j], bf16lo(ww[q]), acc[u][2 * q]);
-            acc[u][2 * q + 1] = fmaf(gs[j], bf16hi(ww[q]), acc[u][2 * q + 1]);
-          }
-        }
-      }
-      if (ysh) {
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int v = v0 + 32 * u;
-          if (v < nv) {
-            const uint4 w = ld_nc_v4(ysh + (int64_t)v * 8);
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              acc[u][2 * q] += bf16lo(ww[q]);
-              acc[u][2 * q + 1] += bf16hi(ww[q]);
-            }
-          }
-        }
-      }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int v = v0 + 32 * u;
-        if (v < nv) {
-          uint4 r;
-          r.x = pack_bf16x2(acc[u][0], acc[u][1]);
-          r.y = pack_bf16x2(acc[u][2], acc[u][3]);
-          r.z = pack_bf16x2(acc[u][4], acc[u][5]);
-          r.w = pack_bf16x2(acc[u][6], acc[u][7]);
-          st_v4(o + (int64_t)v * 8, r);
+        sv[u] = (ysh && v < v_end) ? ld_nc_v4(ysh + (int64_t)v * 8) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        float acc[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+          if (src[j] < 0) continue;
+          const uint32_t ww[4] = {wv[j][u].x, wv[j][u].y, wv[j][u].z, wv[j][u].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            acc[2 * q] = fmaf(gs[j], bf16lo(ww[q]), acc[2 * q]);
+            acc[2 * q + 1] = fmaf(gs[j], bf16hi(ww[q]), acc[2 * q + 1]);
+          }
         }
+        if (ysh) {
+          const uint32_t ss[4] = {sv[u].x, sv[u].y, sv[u].z, sv[u].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            acc[2 * q] += bf16lo(ss[q]);
+            acc[2 * q + 1] += bf16hi(ss[q]);
+          }
+        }
+        const int v = v0 + 32 * u;
+        if (v < v_end)
+          st_v4(o + (int64_t)v * 8, make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                               pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7])));
       }
     }
   }
@@ -111,12 +108,17 @@ cudaError_t launch_combine(const moe_shape_t& s, const uint16_t* y_perm, const i
                            const float* topk_gate, const uint16_t* y_shared, uint16_t* out, uint32_t* status,
                            cudaStream_t stream) {
   if (s.T == 0) return cudaSuccess;
-  const int threads = 256;
-  int64_t blocks = ((int64_t)s.T + 7) / 8;
-  const int64_t cap = (int64_t)num_sms() * 8;
-  if (blocks > cap) blocks = cap;
-  combine_kernel<2><<<(unsigned)blocks, threads, 0, stream>>>(y_perm, assign_row, topk_gate, y_shared, out, s.T,
-                                                              s.d, s.k, (int64_t)s.T * s.k, status);
+  const RowSlices rs = row_slices(s.T, s.d);
+  const int64_t A = (int64_t)s.T * s.k;
+  if (s.k <= 2)
+    combine_kernel<4, 2><<<(unsigned)rs.blocks, 256, 0, stream>>>(y_perm, assign_row, topk_gate, y_shared, out, s.T,
+                                                                   s.d, s.k, A, rs.slices, rs.vps, status);
+  else if (s.k <= 4)
+    combine_kernel<2, 4><<<(unsigned)rs.blocks, 256, 0, stream>>>(y_perm, assign_row, topk_gate, y_shared, out, s.T,
+                                                                   s.d, s.k, A, rs.slices, rs.vps, status);
+  else
+    combine_kernel<1, 8><<<(unsigned)rs.blocks, 256, 0, stream>>>(y_perm, assign_row, topk_gate, y_shared, out, s.T,
+                                                                   s.d, s.k, A, rs.slices, rs.vps, status);
   return cudaGetLastError();
 }
 

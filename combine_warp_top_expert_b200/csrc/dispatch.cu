@@ -8,13 +8,15 @@
  *
  * Assignment a = t*k + j goes to row offsets[e] + (number of earlier
  * assignments to e): a stable counting sort, bit-exact and deterministic (no
- * atomics decide a position). Three kernels:
- *   hist    one CTA per chunk of ~2048 assignments: per-warp histograms with
- *           __match_any_sync, giving each assignment its rank inside the chunk;
- *   scan    one CTA: expert totals, exclusive scan, per-(chunk, expert) base
- *           rows, logical-rank counts/offsets, imbalance ratios;
- *   permute one warp per token: writes row_src/assign_row and copies the
- *           token's row (16-byte vectors, read once) to its k destinations.
+ * atomic decides a position). Two kernels:
+ *   count   one CTA per chunk of ~2048 assignments: per-warp histograms with
+ *           __match_any_sync give each assignment its rank inside the chunk;
+ *           the CTA that finishes last (atomic ticket) runs the scan: expert
+ *           totals, exclusive scan, per-(chunk, expert) base rows, logical-rank
+ *           counts/offsets and the imbalance ratios;
+ *   permute one warp per (token, column slice): writes row_src/assign_row and
+ *           copies its slice of the token's row (16-byte vectors, read once)
+ *           to the k destinations; slices keep every SM busy at small T.
  * Bytes: T*d*2 read + T*k*d*2 written by the permute, plus ~T*k*16 of indices.
  */
 #include "moe_device.cuh"
@@ -25,16 +27,117 @@ namespace {
 
 constexpr int kHistThreads = 512;
 constexpr int kHistWarps = kHistThreads / 32;
-constexpr int kScanThreads = 1024;
+constexpr int kScanThreads = 512;
 
-__global__ void __launch_bounds__(kHistThreads) dispatch_hist_kernel(const int32_t* __restrict__ topk_idx, int64_t A,
-                                                                     int E, int64_t chunk_assign,
-                                                                     int32_t* __restrict__ chunk_cnt,
-                                                                     int32_t* __restrict__ local_rank,
-                                                                     uint32_t* status) {
+/* Scan over the per-chunk counts (run by one whole CTA of kScanThreads threads):
+ * expert totals and offsets, chunk counts -> chunk base rows (in place), rank
+ * counts/offsets, imbalance; row_src of rows beyond the placed total = -1. */
+__device__ void scan_chunks(int32_t* chunk, int64_t C, int E, int R, int64_t A, int32_t* expert_counts,
+                            int32_t* expert_offsets, int32_t* rank_counts, int32_t* rank_offsets, float* imbalance,
+                            int32_t* row_src) {
+  __shared__ int32_t part[kScanThreads]; /* [G][E] partial sums over chunk ranges */
+  __shared__ int32_t cnt[kMaxE];
+  __shared__ int32_t off[kMaxE + 1];
+  __shared__ int32_t s_max[2];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = max(1, kScanThreads / E);
+  const int e = tid % E, g = tid / E;
+  const bool active = g < G;
+  const int64_t c_begin = active ? (C * g) / G : 0, c_end = active ? (C * (g + 1)) / G : 0;
+  int32_t s = 0;
+  for (int64_t c = c_begin; c < c_end; ++c) s += __ldcg(chunk + c * E + e);
+  if (active) part[g * E + e] = s;
+  __syncthreads();
+  if (tid < E) {
+    int run = 0;
+    for (int q = 0; q < G; ++q) {
+      const int v = part[q * E + tid];
+      part[q * E + tid] = run;
+      run += v;
+    }
+    cnt[tid] = run;
+  }
+  __syncthreads();
+  /* exclusive scan of cnt[0..E) by warp 0: each lane owns a contiguous slice */
+  if (warp == 0) {
+    const int per = (E + 31) / 32;
+    const int b = min(E, lane * per), en = min(E, b + per);
+    int local = 0;
+    for (int i = b; i < en; ++i) local += cnt[i];
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - local;
+    for (int i = b; i < en; ++i) {
+      off[i] = run;
+      run += cnt[i];
+    }
+    if (lane == 31) off[E] = incl;
+  }
+  __syncthreads();
+  const int total = off[E];
+  /* chunk base rows, in place */
+  if (active) {
+    int32_t base = off[e] + part[g * E + e];
+    for (int64_t c = c_begin; c < c_end; ++c) {
+      const int32_t v = __ldcg(chunk + c * E + e);
+      chunk[c * E + e] = base;
+      base += v;
+    }
+  }
+  if (tid < E) {
+    expert_counts[tid] = cnt[tid];
+    expert_offsets[tid] = off[tid];
+  }
+  if (tid == 0) expert_offsets[E] = total;
+  const int per_rank = E / R;
+  for (int r = tid; r < R; r += blockDim.x) {
+    rank_offsets[r] = off[r * per_rank];
+    rank_counts[r] = off[(r + 1) * per_rank] - off[r * per_rank];
+  }
+  if (tid == 0) rank_offsets[R] = total;
+  /* maxima over ranks and experts (warp 0) */
+  if (warp == 0) {
+    int me = 0, mr = 0;
+    for (int i = lane; i < E; i += 32) me = max(me, cnt[i]);
+    for (int r = lane; r < R; r += 32) mr = max(mr, off[(r + 1) * per_rank] - off[r * per_rank]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      me = max(me, __shfl_xor_sync(0xFFFFFFFFu, me, o));
+      mr = max(mr, __shfl_xor_sync(0xFFFFFFFFu, mr, o));
+    }
+    if (lane == 0) {
+      s_max[0] = mr;
+      s_max[1] = me;
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    /* max / mean = (max * R) / total: exact integers, one correctly rounded
+     * double quotient, rounded once to fp32 (exact result for total < 2^28) */
+    if (total == 0) {
+      imbalance[0] = 1.0f;
+      imbalance[1] = 1.0f;
+    } else {
+      imbalance[0] = (float)((double)((int64_t)s_max[0] * R) / (double)total);
+      imbalance[1] = (float)((double)((int64_t)s_max[1] * E) / (double)total);
+    }
+  }
+  for (int64_t p = total + tid; p < A; p += blockDim.x) row_src[p] = -1;
+}
+
+__global__ void __launch_bounds__(kHistThreads) dispatch_count_kernel(
+    const int32_t* __restrict__ topk_idx, int64_t A, int E, int R, int64_t chunk_assign, int64_t n_chunks,
+    int32_t* __restrict__ chunk_cnt, int32_t* __restrict__ local_rank, uint32_t* status, uint32_t* ticket,
+    int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts, int32_t* rank_offsets, float* imbalance,
+    int32_t* row_src) {
   extern __shared__ int32_t sh[];
-  int32_t* hist = sh;                         /* [kHistWarps][E] */
-  int32_t* lrank = sh + kHistWarps * E;       /* [chunk_assign] */
+  __shared__ int s_last;
+  int32_t* hist = sh;                   /* [kHistWarps][E] */
+  int32_t* lrank = sh + kHistWarps * E; /* [chunk_assign] */
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t a0 = (int64_t)blockIdx.x * chunk_assign;
   const int64_t rem = A - a0;
@@ -85,125 +188,48 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_hist_kernel(const int32
     local_rank[a0 + i] = out;
   }
   if (bad) raise_status(status, MOE_DEV_BOUNDS);
+
+  /* the last chunk to finish scans all chunk counts */
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(ticket, 1u) == (uint32_t)(n_chunks - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  scan_chunks(chunk_cnt, n_chunks, E, R, A, expert_counts, expert_offsets, rank_counts, rank_offsets, imbalance,
+              row_src);
+  if (threadIdx.x == 0) *ticket = 0; /* ready for the next call on this workspace */
 }
 
-__global__ void __launch_bounds__(kScanThreads) dispatch_scan_kernel(
-    int32_t* __restrict__ chunk, int64_t C, int E, int R, int64_t A, int32_t* __restrict__ expert_counts,
-    int32_t* __restrict__ expert_offsets, int32_t* __restrict__ rank_counts, int32_t* __restrict__ rank_offsets,
-    float* __restrict__ imbalance, int32_t* __restrict__ row_src) {
-  __shared__ int32_t part[kScanThreads]; /* [G][E] partial sums over chunk ranges */
-  __shared__ int32_t cnt[kMaxE];
-  __shared__ int32_t off[kMaxE + 1];
-  __shared__ int32_t s_max[2];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int G = max(1, kScanThreads / E);
-  const int e = tid % E, g = tid / E;
-  const bool active = g < G;
-  const int64_t c_begin = active ? (C * g) / G : 0, c_end = active ? (C * (g + 1)) / G : 0;
-  int32_t s = 0;
-  for (int64_t c = c_begin; c < c_end; ++c) s += chunk[c * E + e];
-  if (active) part[g * E + e] = s;
-  __syncthreads();
-  if (tid < E) {
-    int run = 0;
-    for (int q = 0; q < G; ++q) {
-      const int v = part[q * E + tid];
-      part[q * E + tid] = run;
-      run += v;
-    }
-    cnt[tid] = run;
-  }
-  __syncthreads();
-  /* exclusive scan of cnt[0..E) by warp 0: each lane owns a contiguous slice */
-  if (warp == 0) {
-    const int per = (E + 31) / 32;
-    const int b = min(E, lane * per), en = min(E, b + per);
-    int local = 0;
-    for (int i = b; i < en; ++i) local += cnt[i];
-    int incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int run = incl - local;
-    for (int i = b; i < en; ++i) {
-      off[i] = run;
-      run += cnt[i];
-    }
-    if (lane == 31) off[E] = incl;
-  }
-  __syncthreads();
-  const int total = off[E];
-  /* chunk base rows, in place */
-  if (active) {
-    int32_t base = off[e] + part[g * E + e];
-    for (int64_t c = c_begin; c < c_end; ++c) {
-      const int32_t v = chunk[c * E + e];
-      chunk[c * E + e] = base;
-      base += v;
-    }
-  }
-  if (tid < E) {
-    expert_counts[tid] = cnt[tid];
-    expert_offsets[tid] = off[tid];
-  }
-  if (tid == 0) expert_offsets[E] = total;
-  const int per_rank = E / R;
-  if (tid < R) {
-    rank_offsets[tid] = off[tid * per_rank];
-    rank_counts[tid] = off[(tid + 1) * per_rank] - off[tid * per_rank];
-  }
-  if (tid == 0) rank_offsets[R] = total;
-  /* maxima over ranks and experts (warp 0) */
-  if (warp == 0) {
-    int me = 0, mr = 0;
-    for (int i = lane; i < E; i += 32) me = max(me, cnt[i]);
-    for (int r = lane; r < R; r += 32) mr = max(mr, off[(r + 1) * per_rank] - off[r * per_rank]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      me = max(me, __shfl_xor_sync(0xFFFFFFFFu, me, o));
-      mr = max(mr, __shfl_xor_sync(0xFFFFFFFFu, mr, o));
-    }
-    if (lane == 0) {
-      s_max[0] = mr;
-      s_max[1] = me;
-    }
-  }
-  __syncthreads();
-  if (tid == 0) {
-    /* max / mean = (max * R) / total: exact integers, one correctly rounded
-     * double quotient, rounded once to fp32 (exact result for total < 2^28) */
-    if (total == 0) {
-      imbalance[0] = 1.0f;
-      imbalance[1] = 1.0f;
-    } else {
-      imbalance[0] = (float)((double)((int64_t)s_max[0] * R) / (double)total);
-      imbalance[1] = (float)((double)((int64_t)s_max[1] * E) / (double)total);
-    }
-  }
-  for (int64_t p = total + tid; p < A; p += blockDim.x) row_src[p] = -1;
+/* Empty batch: zero counts, imbalance {1, 1}. */
+__global__ void __launch_bounds__(kScanThreads) dispatch_empty_kernel(int E, int R, int32_t* expert_counts,
+                                                                      int32_t* expert_offsets, int32_t* rank_counts,
+                                                                      int32_t* rank_offsets, float* imbalance) {
+  scan_chunks(nullptr, 0, E, R, 0, expert_counts, expert_offsets, rank_counts, rank_offsets, imbalance, nullptr);
 }
 
 template <int U>
 __global__ void __launch_bounds__(256) dispatch_permute_kernel(
     const uint16_t* __restrict__ x, const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ chunk_base,
-    const int32_t* __restrict__ local_rank, int64_t T, int d, int E, int k, int64_t tok_per_chunk,
-    int32_t* __restrict__ row_src, int32_t* __restrict__ assign_row, uint16_t* __restrict__ x_perm) {
+    const int32_t* __restrict__ local_rank, int64_t T, int d, int E, int k, int64_t tok_per_chunk, int slices,
+    int vps, int32_t* __restrict__ row_src, int32_t* __restrict__ assign_row, uint16_t* __restrict__ x_perm) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int nv = d >> 3; /* 16-byte vectors per row */
-  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
+  const int64_t items = T * slices;
+  for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < items; w += warps) {
+    const int64_t t = w / slices;
+    const int sl = (int)(w - t * slices);
     int pos = -1;
     if (lane < k) {
       const int64_t a = t * k + lane;
       const int e = __ldg(topk_idx + a);
       const int lr = __ldg(local_rank + a);
-      if (e >= 0 && e < E && lr >= 0) {
-        pos = __ldg(chunk_base + (t / tok_per_chunk) * E + e) + lr;
-        row_src[pos] = (int32_t)a;
+      if (e >= 0 && e < E && lr >= 0) pos = __ldg(chunk_base + (t / tok_per_chunk) * E + e) + lr;
+      if (sl == 0) {
+        if (pos >= 0) row_src[pos] = (int32_t)a;
+        assign_row[a] = pos;
       }
-      assign_row[a] = pos;
     }
     int64_t dst[kMaxK];
 #pragma unroll
@@ -212,12 +238,13 @@ __global__ void __launch_bounds__(256) dispatch_permute_kernel(
       dst[j] = (j < k && p >= 0) ? (int64_t)p * d : -1;
     }
     const uint16_t* src = x + t * d;
-    for (int v0 = lane; v0 < nv; v0 += 32 * U) {
+    const int v_end = min(nv, (sl + 1) * vps);
+    for (int v0 = sl * vps + lane; v0 < v_end; v0 += 32 * U) {
       uint4 buf[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int v = v0 + 32 * u;
-        if (v < nv) buf[u] = ld_nc_v4(src + (int64_t)v * 8);
+        if (v < v_end) buf[u] = ld_nc_v4(src + (int64_t)v * 8);
       }
 #pragma unroll
       for (int j = 0; j < kMaxK; ++j) {
@@ -225,7 +252,7 @@ __global__ void __launch_bounds__(256) dispatch_permute_kernel(
 #pragma unroll
         for (int u = 0; u < U; ++u) {
           const int v = v0 + 32 * u;
-          if (v < nv) st_v4(x_perm + dst[j] + (int64_t)v * 8, buf[u]);
+          if (v < v_end) st_v4(x_perm + dst[j] + (int64_t)v * 8, buf[u]);
         }
       }
     }
@@ -234,30 +261,47 @@ __global__ void __launch_bounds__(256) dispatch_permute_kernel(
 
 }  // namespace
 
+RowSlices row_slices(int64_t T, int d) {
+  const int nv = d / 8;
+  const int64_t target = (int64_t)num_sms() * 32; /* warps: 4 CTAs of 8 warps per SM */
+  int64_t s = T > 0 ? (target + T - 1) / T : 1;
+  const int max_s = (nv + 31) / 32;
+  if (s > max_s) s = max_s;
+  if (s < 1) s = 1;
+  int vps = (int)((nv + s - 1) / s);
+  vps = (vps + 31) / 32 * 32;
+  RowSlices r;
+  r.vps = vps;
+  r.slices = (nv + vps - 1) / vps;
+  const int64_t items = T * r.slices;
+  int64_t blocks = (items + 7) / 8;
+  const int64_t cap = (int64_t)num_sms() * 8;
+  r.blocks = (int)(blocks > cap ? cap : (blocks < 1 ? 1 : blocks));
+  return r;
+}
+
 cudaError_t launch_dispatch(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const uint16_t* x,
                             const int32_t* topk_idx, int32_t* expert_counts, int32_t* expert_offsets,
                             int32_t* rank_counts, int32_t* rank_offsets, int32_t* row_src, int32_t* assign_row,
                             uint16_t* x_perm, float* imbalance, cudaStream_t stream) {
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+  uint32_t* ticket = reinterpret_cast<uint32_t*>(ws + L.status + kTicketOffset);
   int32_t* chunk = reinterpret_cast<int32_t*>(ws + L.chunk);
   int32_t* lrank = reinterpret_cast<int32_t*>(ws + L.local_rank);
   const int64_t chunk_assign = L.tok_per_chunk * s.k;
-  if (L.n_chunks > 0) {
-    const size_t smem = (size_t)(kHistWarps * s.E + chunk_assign) * sizeof(int32_t);
-    dispatch_hist_kernel<<<(unsigned)L.n_chunks, kHistThreads, smem, stream>>>(topk_idx, L.A, s.E, chunk_assign,
-                                                                              chunk, lrank, status);
+  if (L.n_chunks == 0) {
+    dispatch_empty_kernel<<<1, kScanThreads, 0, stream>>>(s.E, s.R, expert_counts, expert_offsets, rank_counts,
+                                                          rank_offsets, imbalance);
+    return cudaGetLastError();
   }
-  dispatch_scan_kernel<<<1, kScanThreads, 0, stream>>>(chunk, L.n_chunks, s.E, s.R, L.A, expert_counts,
-                                                       expert_offsets, rank_counts, rank_offsets, imbalance,
-                                                       row_src);
-  if (s.T > 0) {
-    const int threads = 256;
-    int64_t blocks = ((int64_t)s.T + 7) / 8;
-    const int64_t cap = (int64_t)num_sms() * 8;
-    if (blocks > cap) blocks = cap;
-    dispatch_permute_kernel<4><<<(unsigned)blocks, threads, 0, stream>>>(
-        x, topk_idx, chunk, lrank, s.T, s.d, s.E, s.k, L.tok_per_chunk, row_src, assign_row, x_perm);
-  }
+  const size_t smem = (size_t)(kHistWarps * s.E + chunk_assign) * sizeof(int32_t);
+  dispatch_count_kernel<<<(unsigned)L.n_chunks, kHistThreads, smem, stream>>>(
+      topk_idx, L.A, s.E, s.R, chunk_assign, L.n_chunks, chunk, lrank, status, ticket, expert_counts,
+      expert_offsets, rank_counts, rank_offsets, imbalance, row_src);
+  const RowSlices rs = row_slices(s.T, s.d);
+  dispatch_permute_kernel<4><<<(unsigned)rs.blocks, 256, 0, stream>>>(x, topk_idx, chunk, lrank, s.T, s.d, s.E, s.k,
+                                                                     L.tok_per_chunk, rs.slices, rs.vps, row_src,
+                                                                     assign_row, x_perm);
   return cudaGetLastError();
 }
 

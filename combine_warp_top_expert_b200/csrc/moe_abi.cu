@@ -115,7 +115,7 @@ size_t moe_workspace_bytes(const moe_shape_t* shape) {
 
 moe_status_t moe_clear_status(void* ws, size_t ws_bytes, void* stream) {
   if (!ws || !aligned(ws, 256) || ws_bytes < 256) return MOE_ERR_WORKSPACE;
-  const cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(uint32_t), (cudaStream_t)stream);
+  const cudaError_t e = cudaMemsetAsync(ws, 0, 256, (cudaStream_t)stream); /* status word and dispatch ticket */
   return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }
 

@@ -20,6 +20,16 @@ constexpr int kGemmSingle = 1;        /* grouped GEMM: single-CTA 128-row tiles 
 constexpr int kGemmPair = 2;          /* grouped GEMM: CTA-pair 256-row tiles wherever they apply */
 constexpr int kChunkAssign = 2048;    /* assignments per dispatch histogram chunk */
 constexpr uint64_t kDefaultWaitNs = 2000000000ull; /* bounded-wait limit of the GEMM pipeline */
+constexpr size_t kTicketOffset = 64; /* uint32 in the workspace header: dispatch's last-chunk ticket */
+
+/* Work split of the row-copy kernels (permute, combine): one warp per (token,
+ * slice of `vps` 16-byte vectors), `blocks` CTAs of 8 warps (grid-stride). */
+struct RowSlices {
+  int slices = 1;
+  int vps = 32;
+  int blocks = 1;
+};
+RowSlices row_slices(int64_t T, int d);
 
 /* Byte offsets into the caller's workspace (all 256-byte aligned). */
 struct WsLayout {

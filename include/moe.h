@@ -79,7 +79,8 @@ typedef struct moe_shape {
 /* Bytes of workspace the entry points need for `shape` (0 if the shape is invalid). */
 size_t moe_workspace_bytes(const moe_shape_t* shape);
 
-/* Zero the device status word in `ws` (asynchronous on `stream`). */
+/* Zero the 256-byte header of `ws` (status word and internal counters),
+ * asynchronously on `stream`. Call once on a new workspace before first use. */
 moe_status_t moe_clear_status(void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, then copy the device status word (MOE_DEV_* bits) to *bits.
