@@ -335,68 +335,51 @@ class MoELayer:
     def __call__(self, logits, x, stream=None) -> dict:
         return moe_layer(self.shape, logits, x, self.w13, self.w2, self.w13s, self.w2s, self.outs, self.ws, stream)
 
-    def forward_host(self, logits_host, x_host, out_host, stream=None, chunks=None):
-        """End-to-end call with HOST tensors (pinned, for asynchronous copies).
+    def forward_host(self, logits_host, x_host, out_host, stream=None):
+        """Asynchronous end-to-end call with HOST tensors (pinned, for DMA).
 
-        The batch is cut into token chunks (`chunks`: a list of sizes summing to T;
-        default `default_host_chunks(T)`). Each chunk's inputs are copied to the
-        device on one stream, the layer runs on `stream`, and the chunk's `out` is
-        copied back on a third stream, so copies overlap the other chunks' compute.
-        Every token's result is the same as in one call (the layer is token-wise);
-        the routing statistics (counts, imbalance) are per chunk. Returns out_host;
-        `stream` waits for the last copy."""
+        Enqueues, and returns without waiting: the copy of this batch's logits and x
+        to the device (on a copy-in stream), the layer (on `stream`), and the copy of
+        `out` back into out_host (on a copy-out stream). Call sync_host() (or
+        torch.cuda.synchronize()) before reading out_host. Successive calls rotate
+        between two device staging slots, so one batch's copies overlap its
+        neighbours' compute, as in a serving loop; a slot is reused only after its
+        previous compute and copy-out have finished (CUDA events)."""
         import torch
-        T = self.shape.T
-        sizes = list(chunks) if chunks is not None else default_host_chunks(T)
-        if sum(sizes) != T or any(c <= 0 for c in sizes):
-            raise ValueError(f"chunk sizes {sizes} do not cover T={T}")
         s_comp = stream or torch.cuda.current_stream(self.ws.device)
-        key = tuple(sizes)
-        if getattr(self, "_pipe_key", None) != key:
+        if not hasattr(self, "_slots"):
             dev = self.ws.device
-            self._pipe_key = key
-            self._pipe = []
-            shapes = [Shape(c, self.shape.d, self.shape.E, self.shape.k, self.shape.f, self.shape.R,
-                            self.shape.n_shared) for c in sizes]
-            self._pipe_ws = torch.zeros(max(workspace_bytes(sh) for sh in shapes), dtype=torch.uint8, device=dev)
-            for sh in shapes:
-                self._pipe.append(dict(
-                    shape=sh, outs=alloc_layer_outputs(sh, dev),
-                    x=torch.empty((sh.T, sh.d), dtype=torch.bfloat16, device=dev),
-                    logits=torch.empty((sh.T, sh.E), dtype=torch.float32, device=dev),
-                    ev_in=torch.cuda.Event(), ev_done=torch.cuda.Event()))
+            self._slots = [dict(outs=alloc_layer_outputs(self.shape, dev),
+                                x=torch.empty((self.shape.T, self.shape.d), dtype=torch.bfloat16, device=dev),
+                                logits=torch.empty((self.shape.T, self.shape.E), dtype=torch.float32, device=dev),
+                                ev_in=torch.cuda.Event(), ev_done=torch.cuda.Event(), ev_out=torch.cuda.Event(),
+                                used=False) for _ in range(2)]
             self._s_in = torch.cuda.Stream(dev)
             self._s_out = torch.cuda.Stream(dev)
-            self._ev_last = torch.cuda.Event()
-        self._s_in.wait_stream(s_comp)   # earlier work on the chunk buffers has finished
-        self._s_out.wait_stream(s_comp)
-        t0 = 0
-        for c in self._pipe:
-            t1 = t0 + c["shape"].T
-            with torch.cuda.stream(self._s_in):
-                c["logits"].copy_(logits_host[t0:t1], non_blocking=True)
-                c["x"].copy_(x_host[t0:t1], non_blocking=True)
-                c["ev_in"].record(self._s_in)
-            s_comp.wait_event(c["ev_in"])
-            moe_layer(c["shape"], c["logits"], c["x"], self.w13, self.w2, self.w13s, self.w2s, c["outs"],
-                      self._pipe_ws, s_comp)
-            c["ev_done"].record(s_comp)
-            self._s_out.wait_event(c["ev_done"])
-            with torch.cuda.stream(self._s_out):
-                out_host[t0:t1].copy_(c["outs"]["out"], non_blocking=True)
-            t0 = t1
-        self._ev_last.record(self._s_out)
-        s_comp.wait_event(self._ev_last)
+            self._slot = 0
+        c = self._slots[self._slot]
+        self._slot ^= 1
+        if c["used"]:
+            self._s_in.wait_event(c["ev_done"])   # the slot's inputs were consumed by its last compute
+            s_comp.wait_event(c["ev_out"])        # the slot's last out has been copied back
+        else:
+            self._s_in.wait_stream(s_comp)
+        c["used"] = True
+        with torch.cuda.stream(self._s_in):
+            c["logits"].copy_(logits_host, non_blocking=True)
+            c["x"].copy_(x_host, non_blocking=True)
+            c["ev_in"].record(self._s_in)
+        s_comp.wait_event(c["ev_in"])
+        moe_layer(self.shape, c["logits"], c["x"], self.w13, self.w2, self.w13s, self.w2s, c["outs"], self.ws, s_comp)
+        c["ev_done"].record(s_comp)
+        self._s_out.wait_event(c["ev_done"])
+        with torch.cuda.stream(self._s_out):
+            out_host.copy_(c["outs"]["out"], non_blocking=True)
+            c["ev_out"].record(self._s_out)
+        self._last_out = c["ev_out"]
         return out_host
 
-
-def default_host_chunks(T: int):
-    """Token chunks for host-buffer calls: big enough that each chunk's grouped GEMM
-    stays compute-bound (every chunk re-reads the experts' weights), small at the
-    ends so that only a little copying is left exposed."""
-    if T >= 4096:
-        q = T // 4
-        return [q, T - 2 * q, q]
-    if T >= 2048:
-        return [T // 2, T - T // 2]
-    return [T]
+    def sync_host(self):
+        """Block until the last forward_host's copy-out has landed in host memory."""
+        if getattr(self, "_last_out", None) is not None:
+            self._last_out.synchronize()

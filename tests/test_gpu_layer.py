@@ -152,29 +152,26 @@ def test_inconsistent_offsets_are_reported_not_hung():
     assert status == 0
 
 
-@pytest.mark.parametrize("chunks", [None, [1], [100, 156], [64, 64, 64, 64]])
-def test_host_buffer_pipeline_equals_device_call(chunks):
-    """forward_host (host tensors, chunked copies overlapping compute) gives every
-    token the same result as one device call."""
+def test_host_buffer_calls_overlap_and_match_device_calls():
+    """forward_host (host tensors; copies on side streams, two rotating staging
+    slots) gives each batch exactly the result of a device call, across calls in a
+    row whose copies overlap each other's compute."""
     import torch
-    wl = moe_synth.workload("tiny")
-    dv, layer, outs, status = _run_layer(wl)
-    want = outs["out"].clone()
-    if chunks == [1]:
-        chunks = [wl.T]
-    x_h = dv["x"].cpu().pin_memory()
-    lg_h = dv["logits"].cpu().pin_memory()
-    out_h = torch.zeros((wl.T, wl.d), dtype=torch.bfloat16).pin_memory()
-    layer.forward_host(lg_h, x_h, out_h, chunks=chunks)
-    torch.cuda.current_stream().synchronize()
-    close(f64(bits(out_h)), f64(bits(want)), "out (host pipeline)")
-    # bit-identical when the grouped GEMM runs the same tile shape for every chunk
     old = moe.set_gemm_policy(moe.GEMM_SINGLE)
     try:
-        layer(dv["logits"], dv["x"])
-        want = layer.outs["out"].clone()
-        layer.forward_host(lg_h, x_h, out_h, chunks=chunks)
-        torch.cuda.current_stream().synchronize()
-        assert torch.equal(out_h.view(torch.int16), want.cpu().view(torch.int16))
+        wl = moe_synth.workload("tiny")
+        batches = [moe_synth.device_inputs(wl.with_(seed=s), weights=(s == 0)) for s in range(3)]
+        dv = batches[0]
+        layer = moe.MoELayer(_shape(wl), dv["w13"], dv["w2"])
+        want = []
+        for b in batches:
+            want.append(layer(b["logits"], b["x"])["out"].clone())
+        hosts = [(b["logits"].cpu().pin_memory(), b["x"].cpu().pin_memory(),
+                  torch.zeros((wl.T, wl.d), dtype=torch.bfloat16).pin_memory()) for b in batches]
+        for lg_h, x_h, out_h in hosts:
+            layer.forward_host(lg_h, x_h, out_h)
+        torch.cuda.synchronize()
+        for (_, _, out_h), w in zip(hosts, want):
+            assert torch.equal(out_h.view(torch.int16), w.cpu().view(torch.int16))
     finally:
         moe.set_gemm_policy(old)
