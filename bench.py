@@ -39,18 +39,20 @@ DEFAULT_CONFIG = "mixtral_prefill"
 # ---------------------------------------------------------------------------
 
 def algorithmic(wl, counts):
-    """Per-step algorithmic bytes and flops of each step (padding excluded)."""
-    T, d, E, k, f, A = wl.T, wl.d, wl.E, wl.k, wl.f, wl.T * wl.k
+    """Per-step algorithmic bytes and flops of each step (padding excluded). `counts` are the
+    rows each expert actually processes (after any capacity drops)."""
+    T, d, E, k, f = wl.T, wl.d, wl.E, wl.k, wl.f
+    A = int(sum(counts))  # placed assignments
     n_act = int(sum(1 for c in counts if c > 0))
     sh = wl.n_shared
     w = {}
-    w["route"] = dict(bytes=T * E * 4 + A * 8, flops=0)
-    w["dispatch"] = dict(bytes=T * d * 2 + A * d * 2 + A * 8, flops=0)
+    w["route"] = dict(bytes=T * E * 4 + T * k * 8, flops=0)
+    w["dispatch"] = dict(bytes=T * d * 2 + A * d * 2 + T * k * 8, flops=0)
     w["gate_up"] = dict(flops=4 * A * d * f + sh * 4 * T * d * f,
                         bytes=(n_act + sh) * 2 * d * f * 2 + A * d * 2 + sh * T * d * 2)
     w["down"] = dict(flops=2 * A * d * f + sh * 2 * T * d * f,
                      bytes=(n_act + sh) * d * f * 2 + A * d * 2 + sh * T * d * 2)
-    w["combine"] = dict(bytes=A * d * 2 + A * 8 + T * d * 2 + sh * T * d * 2, flops=0)
+    w["combine"] = dict(bytes=A * d * 2 + T * k * 8 + T * d * 2 + sh * T * d * 2, flops=0)
     w["_n_act"] = n_act
     return w
 
@@ -258,7 +260,8 @@ def run_gpu(args, wl, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     moe.set_gemm_policy({"auto": moe.GEMM_AUTO, "single": moe.GEMM_SINGLE, "pair": moe.GEMM_PAIR}[args.gemm_policy])
     wl_r = wl.with_(seed=replica_seed(wl.seed, rank))
-    shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, n_shared=wl.n_shared)
+    cap = moe.capacity_for(args.capacity_factor, wl.T, wl.k, wl.E) if args.capacity_factor else 0
+    shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, n_shared=wl.n_shared, capacity=cap)
     dv = moe_synth.device_inputs(wl_r, device=dev)
     layer = moe.MoELayer(shape, dv["w13"], dv["w2"], dv.get("w13s"), dv.get("w2s"), device=dev)
     o = layer.outs
@@ -365,6 +368,8 @@ def run_gpu(args, wl, rank, world, local_rank):
                    "n_shared": wl.n_shared, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "flushed between steps (512 MiB write, outside the step's events)",
                    "gemm_tiles": args.gemm_policy,
+                   "capacity_factor": args.capacity_factor, "capacity": cap,
+                   "dropped_fraction": 1.0 - sum(counts) / float(wl.T * wl.k) if wl.T else 0.0,
                    "experts_active": work["_n_act"], "imbalance_rank_expert": imbalance,
                    "layer_roofline_frac": t_roof / (max_ms / args.steps / 1e3),
                    "per_step_ms": {n: round(v, 4) for n, v in kern_ms.items()},
@@ -400,6 +405,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gemm-policy", default="auto", choices=["auto", "single", "pair"],
                     help="grouped-GEMM tiles: per-GEMM choice (auto), single-CTA 128-row, or CTA-pair 256x256")
+    ap.add_argument("--capacity-factor", type=float, default=None,
+                    help="per-expert capacity ceil(C*T*k/E); excess assignments are dropped (default: none)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the workload's batch size T (smaller cases for profiling)")
     args = ap.parse_args()

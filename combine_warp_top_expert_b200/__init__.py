@@ -36,7 +36,7 @@ class MoEError(RuntimeError):
 
 
 class moe_shape_t(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int32) for n in ("T", "d", "E", "k", "f", "R", "n_shared")]
+    _fields_ = [(n, ctypes.c_int32) for n in ("T", "d", "E", "k", "f", "R", "n_shared", "capacity")]
 
 
 class moe_layer_buffers_t(ctypes.Structure):
@@ -114,13 +114,21 @@ class Shape:
     f: int
     R: int
     n_shared: int = 0
+    capacity: int = 0  # per-expert assignment limit, 0 = none
 
     @property
     def A(self) -> int:
         return self.T * self.k
 
     def c(self) -> moe_shape_t:
-        return moe_shape_t(self.T, self.d, self.E, self.k, self.f, self.R, self.n_shared)
+        return moe_shape_t(self.T, self.d, self.E, self.k, self.f, self.R, self.n_shared, self.capacity)
+
+
+def capacity_for(C: float, T: int, k: int, E: int) -> int:
+    """Per-expert capacity of a capacity factor C: ceil(C * T * k / E) assignments."""
+    from fractions import Fraction
+    q = Fraction(C).limit_denominator(1 << 20) * T * k / E
+    return int(-(-q.numerator // q.denominator))
 
 
 def _ptr(t) -> Optional[int]:

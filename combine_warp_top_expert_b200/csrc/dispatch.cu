@@ -12,8 +12,8 @@
  *   count   one CTA per chunk of ~2048 assignments: per-warp histograms with
  *           __match_any_sync give each assignment its rank inside the chunk;
  *           the CTA that finishes last (atomic ticket) runs the scan: expert
- *           totals, exclusive scan, per-(chunk, expert) base rows, logical-rank
- *           counts/offsets and the imbalance ratios;
+ *           demand, kept counts (capacity), exclusive scan, per-(chunk, expert)
+ *           rank bases, logical-rank counts/offsets and the imbalance ratios;
  *   permute one warp per (token, column slice): writes row_src/assign_row and
  *           copies its slice of the token's row (16-byte vectors, read once)
  *           to the k destinations; slices keep every SM busy at small T.
@@ -30,9 +30,10 @@ constexpr int kHistWarps = kHistThreads / 32;
 constexpr int kScanThreads = 512;
 
 /* Scan over the per-chunk counts (run by one whole CTA of kScanThreads threads):
- * expert totals and offsets, chunk counts -> chunk base rows (in place), rank
- * counts/offsets, imbalance; row_src of rows beyond the placed total = -1. */
-__device__ void scan_chunks(int32_t* chunk, int64_t C, int E, int R, int64_t A, int32_t* expert_counts,
+ * each expert keeps min(demand, cap) rows; offsets over the kept counts; chunk
+ * counts -> rank bases (the expert-local rank of each chunk's first assignment,
+ * in place); rank counts/offsets, imbalance; row_src beyond the kept total = -1. */
+__device__ void scan_chunks(int32_t* chunk, int64_t C, int E, int R, int64_t A, int32_t cap, int32_t* expert_counts,
                             int32_t* expert_offsets, int32_t* rank_counts, int32_t* rank_offsets, float* imbalance,
                             int32_t* row_src) {
   __shared__ int32_t part[kScanThreads]; /* [G][E] partial sums over chunk ranges */
@@ -55,7 +56,7 @@ __device__ void scan_chunks(int32_t* chunk, int64_t C, int E, int R, int64_t A, 
       part[q * E + tid] = run;
       run += v;
     }
-    cnt[tid] = run;
+    cnt[tid] = min(run, cap); /* kept rows */
   }
   __syncthreads();
   /* exclusive scan of cnt[0..E) by warp 0: each lane owns a contiguous slice */
@@ -79,9 +80,9 @@ __device__ void scan_chunks(int32_t* chunk, int64_t C, int E, int R, int64_t A, 
   }
   __syncthreads();
   const int total = off[E];
-  /* chunk base rows, in place */
+  /* chunk rank bases, in place */
   if (active) {
-    int32_t base = off[e] + part[g * E + e];
+    int32_t base = part[g * E + e];
     for (int64_t c = c_begin; c < c_end; ++c) {
       const int32_t v = __ldcg(chunk + c * E + e);
       chunk[c * E + e] = base;
@@ -130,7 +131,7 @@ __device__ void scan_chunks(int32_t* chunk, int64_t C, int E, int R, int64_t A, 
 }
 
 __global__ void __launch_bounds__(kHistThreads) dispatch_count_kernel(
-    const int32_t* __restrict__ topk_idx, int64_t A, int E, int R, int64_t chunk_assign, int64_t n_chunks,
+    const int32_t* __restrict__ topk_idx, int64_t A, int E, int R, int32_t cap, int64_t chunk_assign, int64_t n_chunks,
     int32_t* __restrict__ chunk_cnt, int32_t* __restrict__ local_rank, uint32_t* status, uint32_t* ticket,
     int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts, int32_t* rank_offsets, float* imbalance,
     int32_t* row_src) {
@@ -196,7 +197,7 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_count_kernel(
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  scan_chunks(chunk_cnt, n_chunks, E, R, A, expert_counts, expert_offsets, rank_counts, rank_offsets, imbalance,
+  scan_chunks(chunk_cnt, n_chunks, E, R, A, cap, expert_counts, expert_offsets, rank_counts, rank_offsets, imbalance,
               row_src);
   if (threadIdx.x == 0) *ticket = 0; /* ready for the next call on this workspace */
 }
@@ -205,14 +206,16 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_count_kernel(
 __global__ void __launch_bounds__(kScanThreads) dispatch_empty_kernel(int E, int R, int32_t* expert_counts,
                                                                       int32_t* expert_offsets, int32_t* rank_counts,
                                                                       int32_t* rank_offsets, float* imbalance) {
-  scan_chunks(nullptr, 0, E, R, 0, expert_counts, expert_offsets, rank_counts, rank_offsets, imbalance, nullptr);
+  scan_chunks(nullptr, 0, E, R, 0, 0x7FFFFFFF, expert_counts, expert_offsets, rank_counts, rank_offsets, imbalance,
+              nullptr);
 }
 
 template <int U>
 __global__ void __launch_bounds__(256) dispatch_permute_kernel(
     const uint16_t* __restrict__ x, const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ chunk_base,
-    const int32_t* __restrict__ local_rank, int64_t T, int d, int E, int k, int64_t tok_per_chunk, int slices,
-    int vps, int32_t* __restrict__ row_src, int32_t* __restrict__ assign_row, uint16_t* __restrict__ x_perm) {
+    const int32_t* __restrict__ local_rank, const int32_t* __restrict__ expert_offsets, int64_t T, int d, int E,
+    int k, int32_t cap, int64_t tok_per_chunk, int slices, int vps, int32_t* __restrict__ row_src,
+    int32_t* __restrict__ assign_row, uint16_t* __restrict__ x_perm) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int nv = d >> 3; /* 16-byte vectors per row */
@@ -225,7 +228,10 @@ __global__ void __launch_bounds__(256) dispatch_permute_kernel(
       const int64_t a = t * k + lane;
       const int e = __ldg(topk_idx + a);
       const int lr = __ldg(local_rank + a);
-      if (e >= 0 && e < E && lr >= 0) pos = __ldg(chunk_base + (t / tok_per_chunk) * E + e) + lr;
+      if (e >= 0 && e < E && lr >= 0) {
+        const int rank = __ldg(chunk_base + (t / tok_per_chunk) * E + e) + lr; /* among e's assignments */
+        if (rank < cap) pos = __ldg(expert_offsets + e) + rank;                /* else dropped */
+      }
       if (sl == 0) {
         if (pos >= 0) row_src[pos] = (int32_t)a;
         assign_row[a] = pos;
@@ -295,13 +301,14 @@ cudaError_t launch_dispatch(const moe_shape_t& s, const WsLayout& L, uint8_t* ws
     return cudaGetLastError();
   }
   const size_t smem = (size_t)(kHistWarps * s.E + chunk_assign) * sizeof(int32_t);
+  const int32_t cap = s.capacity > 0 ? s.capacity : 0x7FFFFFFF;
   dispatch_count_kernel<<<(unsigned)L.n_chunks, kHistThreads, smem, stream>>>(
-      topk_idx, L.A, s.E, s.R, chunk_assign, L.n_chunks, chunk, lrank, status, ticket, expert_counts,
+      topk_idx, L.A, s.E, s.R, cap, chunk_assign, L.n_chunks, chunk, lrank, status, ticket, expert_counts,
       expert_offsets, rank_counts, rank_offsets, imbalance, row_src);
   const RowSlices rs = row_slices(s.T, s.d);
-  dispatch_permute_kernel<4><<<(unsigned)rs.blocks, 256, 0, stream>>>(x, topk_idx, chunk, lrank, s.T, s.d, s.E, s.k,
-                                                                     L.tok_per_chunk, rs.slices, rs.vps, row_src,
-                                                                     assign_row, x_perm);
+  dispatch_permute_kernel<4><<<(unsigned)rs.blocks, 256, 0, stream>>>(
+      x, topk_idx, chunk, lrank, expert_offsets, s.T, s.d, s.E, s.k, cap, L.tok_per_chunk, rs.slices, rs.vps,
+      row_src, assign_row, x_perm);
   return cudaGetLastError();
 }
 

@@ -39,6 +39,7 @@ moe_status_t validate_shape(const moe_shape_t* s) {
   if (!s) return MOE_ERR_INVALID_ARG;
   if (s->T < 0 || s->d < 1 || s->f < 1 || s->E < 1 || s->k < 1 || s->R < 1) return MOE_ERR_INVALID_ARG;
   if (s->k > s->E || s->E % s->R != 0 || (s->n_shared != 0 && s->n_shared != 1)) return MOE_ERR_INVALID_ARG;
+  if (s->capacity < 0) return MOE_ERR_INVALID_ARG;
   if (s->E > kMaxE || s->k > kMaxK) return MOE_ERR_UNSUPPORTED;
   if ((int64_t)s->T * s->k > (int64_t(1) << 27)) return MOE_ERR_UNSUPPORTED;
   if (s->d % 128 != 0 || s->f % 128 != 0 || s->d > 65536 || s->f > 65536) return MOE_ERR_UNSUPPORTED;

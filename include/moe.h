@@ -38,7 +38,7 @@
  *
  * Supported shapes: 0 <= T, T*k <= 2^27; 1 <= E <= 256; 1 <= k <= min(E, 8);
  * 1 <= R, E % R == 0; d % 128 == 0 and f % 128 == 0 (128 <= d, f <= 65536);
- * n_shared in {0, 1}.
+ * n_shared in {0, 1}; capacity >= 0.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -74,6 +74,7 @@ typedef struct moe_shape {
   int32_t f;        /* expert FFN width (SwiGLU hidden size) */
   int32_t R;        /* logical expert-parallel ranks */
   int32_t n_shared; /* shared experts applied to every token: 0 or 1 */
+  int32_t capacity; /* per-expert limit on assignments, 0 = none (see moe_dispatch) */
 } moe_shape_t;
 
 /* Bytes of workspace the entry points need for `shape` (0 if the shape is invalid). */
@@ -113,8 +114,14 @@ moe_status_t moe_route(const moe_shape_t* shape, const float* logits, int32_t* t
  *   x_perm         [T*k, d] bf16 out: x_perm[assign_row[a]] = x[a / k]; rows are
  *                  expert-contiguous (expert e at [off[e], off[e+1])), so rank-major;
  *                  inside an expert, rows keep assignment order (stable).
- *   imbalance      [2] fp32 out: [0] = max_r rank_counts[r] / mean (= *R / (T*k)),
- *                  [1] = max_e expert_counts[e] / mean; {1, 1} when T = 0. */
+ *   imbalance      [2] fp32 out: [0] = max_r rank_counts[r] / mean (= *R / total),
+ *                  [1] = max_e expert_counts[e] / mean; {1, 1} when nothing is placed.
+ * Capacity (page §5 "Mitigations", capacity factor): with shape->capacity = c > 0
+ * an expert keeps only its first c assignments in assignment order; the others
+ * are dropped: assign_row = -1, no row, nothing added by moe_combine ("skip the
+ * expert, pass through the residual"). Counts, offsets, ranks and imbalance then
+ * describe the kept rows; T*k - expert_offsets[E] assignments were dropped.
+ * c = ceil(C * T * k / E) gives the page's capacity factor C. */
 moe_status_t moe_dispatch(const moe_shape_t* shape, const moe_bf16_t* x, const int32_t* topk_idx,
                           int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
                           int32_t* rank_offsets, int32_t* row_src, int32_t* assign_row, moe_bf16_t* x_perm,

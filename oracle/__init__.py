@@ -43,6 +43,8 @@ def lib():
         L.oracle_route.argtypes = [i64, i32, i32, vp, vp, vp]
         L.oracle_dispatch.restype = i64
         L.oracle_dispatch.argtypes = [i64, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.oracle_dispatch_capacity.restype = i64
+        L.oracle_dispatch_capacity.argtypes = [i64, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.oracle_permute_rows.restype = None
         L.oracle_permute_rows.argtypes = [i64, i32, i32, vp, vp, vp]
         L.oracle_swiglu.restype = None
@@ -72,7 +74,8 @@ def route(logits: np.ndarray, k: int):
     return idx, gate, int(n)
 
 
-def dispatch(topk_idx: np.ndarray, E: int, R: int) -> dict:
+def dispatch(topk_idx: np.ndarray, E: int, R: int, capacity: int = 0) -> dict:
+    """capacity > 0: each expert keeps only its first `capacity` assignments."""
     topk_idx, ip = _c(topk_idx, np.int32)
     T, k = topk_idx.shape
     A = T * k
@@ -80,9 +83,12 @@ def dispatch(topk_idx: np.ndarray, E: int, R: int) -> dict:
                rank_counts=np.empty(R, np.int32), rank_offsets=np.empty(R + 1, np.int32),
                row_src=np.empty(A, np.int32), assign_row=np.empty(A, np.int32),
                imbalance=np.empty(2, np.float32))
-    bad = lib().oracle_dispatch(T, E, k, R, ip, *(out[n].ctypes.data for n in (
-        "expert_counts", "expert_offsets", "rank_counts", "rank_offsets", "row_src", "assign_row", "imbalance")))
+    dropped = ctypes.c_int64(0)
+    bad = lib().oracle_dispatch_capacity(T, E, k, R, capacity, ip, *(out[n].ctypes.data for n in (
+        "expert_counts", "expert_offsets", "rank_counts", "rank_offsets", "row_src", "assign_row", "imbalance")),
+        ctypes.addressof(dropped))
     out["skipped"] = int(bad)
+    out["dropped"] = int(dropped.value)
     return out
 
 
@@ -165,11 +171,11 @@ def naive_token_loop(x, topk_idx, gate, w13, w2, w13s=None, w2s=None) -> np.ndar
     return out
 
 
-def layer(x, logits, w13, w2, k, R, w13s=None, w2s=None) -> dict:
+def layer(x, logits, w13, w2, k, R, w13s=None, w2s=None, capacity: int = 0) -> dict:
     """The whole layer: route -> dispatch -> permute -> expert FFN -> combine."""
     E = w13.shape[0]
     idx, gate, nan = route(logits, k)
-    disp = dispatch(idx, E, R)
+    disp = dispatch(idx, E, R, capacity)
     x_perm = permute_rows(x, disp["row_src"], k)
     y_perm, y_shared = expert_ffn(x_perm, disp["expert_offsets"], w13, w2, x, w13s, w2s)
     out = combine(y_perm, disp["assign_row"], gate, y_shared)

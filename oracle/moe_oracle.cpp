@@ -91,10 +91,14 @@ int64_t oracle_route(int64_t T, int32_t E, int32_t k, const float* logits, int32
  * and §1 (experts placed on GPUs in contiguous blocks: GPU 0 holds 0-15, ...).
  *   Assignment a = t*k + j goes to expert e = topk_idx[a] (entries outside
  *   [0, E) are skipped, counted, and get assign_row = -1).
- *   counts[e] = #{a : topk_idx[a] = e}; offsets = exclusive scan, offsets[E] = total.
  *   Rows are handed out in assignment order: a takes row offsets[e] + (number of
  *   earlier assignments to e). [reading] the page says "sort" without an order
  *   inside an expert; keeping assignment order is the plainest stable reading.
+ *   Capacity, page §5 "Mitigations" 1 (capacity factor): when capacity > 0 an
+ *   expert keeps only its first `capacity` assignments in that order; the rest
+ *   are dropped (assign_row = -1: "skip the expert, pass through the residual").
+ *   counts[e] = assignments kept by e; offsets = exclusive scan of counts,
+ *   offsets[E] = total kept.
  *   Logical rank r owns experts [r*E/R, (r+1)*E/R): rank_counts[r] = sum of its
  *   experts' counts, rank_offsets[r] = offsets[r*E/R].
  *   Imbalance, page §5: the most loaded GPU against the ideal, 140/64 in the
@@ -102,31 +106,43 @@ int64_t oracle_route(int64_t T, int32_t E, int32_t k, const float* logits, int32
  *   imbalance[1] = max_e counts[e] / (total / E), each computed as
  *   (double)(max * R) / (double)total rounded once to fp32 (exact integers, so
  *   this is the correctly rounded quotient for total < 2^28); {1, 1} if total = 0.
- * Returns the number of skipped (out-of-range) entries.
+ * Returns the number of skipped (out-of-range) entries; *dropped (if not null)
+ * receives the number of assignments dropped by the capacity.
  */
-int64_t oracle_dispatch(int64_t T, int32_t E, int32_t k, int32_t R, const int32_t* topk_idx, int32_t* counts,
-                        int32_t* offsets, int32_t* rank_counts, int32_t* rank_offsets, int32_t* row_src,
-                        int32_t* assign_row, float* imbalance) {
+int64_t oracle_dispatch_capacity(int64_t T, int32_t E, int32_t k, int32_t R, int32_t capacity,
+                                 const int32_t* topk_idx, int32_t* counts, int32_t* offsets, int32_t* rank_counts,
+                                 int32_t* rank_offsets, int32_t* row_src, int32_t* assign_row, float* imbalance,
+                                 int64_t* dropped) {
   const int64_t A = T * (int64_t)k;
-  int64_t bad = 0;
-  for (int32_t e = 0; e < E; ++e) counts[e] = 0;
+  int64_t bad = 0, drop = 0;
+  /* first pass: which assignments each expert keeps, in assignment order */
+  std::vector<int32_t> seen(E, 0);
+  std::vector<char> keep(A, 0);
   for (int64_t a = 0; a < A; ++a) {
     const int32_t e = topk_idx[a];
     if (e < 0 || e >= E) {
       ++bad;
       continue;
     }
-    counts[e] += 1;
+    if (capacity > 0 && seen[e] >= capacity) {
+      ++drop;
+    } else {
+      keep[a] = 1;
+    }
+    seen[e] += 1;
   }
+  for (int32_t e = 0; e < E; ++e) counts[e] = 0;
+  for (int64_t a = 0; a < A; ++a)
+    if (keep[a]) counts[topk_idx[a]] += 1;
   offsets[0] = 0;
   for (int32_t e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
   std::vector<int32_t> cursor(E, 0);
   for (int64_t a = 0; a < A; ++a) {
-    const int32_t e = topk_idx[a];
-    if (e < 0 || e >= E) {
+    if (!keep[a]) {
       assign_row[a] = -1;
       continue;
     }
+    const int32_t e = topk_idx[a];
     const int32_t p = offsets[e] + cursor[e]++;
     row_src[p] = (int32_t)a;
     assign_row[a] = p;
@@ -151,7 +167,16 @@ int64_t oracle_dispatch(int64_t T, int32_t E, int32_t k, int32_t R, const int32_
     imbalance[0] = (float)((double)(max_r * R) / (double)total);
     imbalance[1] = (float)((double)(max_e * E) / (double)total);
   }
+  if (dropped) *dropped = drop;
   return bad;
+}
+
+/* Dispatch with no capacity limit. */
+int64_t oracle_dispatch(int64_t T, int32_t E, int32_t k, int32_t R, const int32_t* topk_idx, int32_t* counts,
+                        int32_t* offsets, int32_t* rank_counts, int32_t* rank_offsets, int32_t* row_src,
+                        int32_t* assign_row, float* imbalance) {
+  return oracle_dispatch_capacity(T, E, k, R, 0, topk_idx, counts, offsets, rank_counts, rank_offsets, row_src,
+                                  assign_row, imbalance, nullptr);
 }
 
 /* Dispatch data movement, page §4 DISPATCH step 3 ("exchange the token data"):

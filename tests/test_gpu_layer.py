@@ -175,3 +175,20 @@ def test_host_buffer_calls_overlap_and_match_device_calls():
             assert torch.equal(out_h.view(torch.int16), w.cpu().view(torch.int16))
     finally:
         moe.set_gemm_policy(old)
+
+
+def test_layer_with_capacity_matches_oracle():
+    import torch
+    wl = moe_synth.Workload("capl", T=300, d=256, E=8, k=2, f=256, R=4, bias_kind="zipf", zipf_s=1.0)
+    cap = moe.capacity_for(1.25, wl.T, wl.k, wl.E)
+    shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, capacity=cap)
+    dv = moe_synth.device_inputs(wl)
+    layer = moe.MoELayer(shape, dv["w13"], dv["w2"])
+    outs = layer(dv["logits"], dv["x"])
+    assert moe.get_status(layer.ws) == 0
+    res = oracle.layer(moe_synth.host_x(wl), moe_synth.host_logits(wl), moe_synth.host_w13(wl),
+                       moe_synth.host_w2(wl), wl.k, wl.R, capacity=cap)
+    assert res["dropped"] > 0
+    for n in ("expert_counts", "expert_offsets", "row_src", "assign_row"):
+        assert np.array_equal(np_i32(outs[n]), res[n]), n
+    close(f64(bits(outs["out"])), res["out"], "out with capacity")

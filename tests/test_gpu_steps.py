@@ -310,3 +310,18 @@ def test_expert_ffn_with_empty_and_full_experts(gemm_policy):
     idx = np.zeros((257, 1), np.int32)
     idx[200:, 0] = 3          # experts 1, 2, 4 empty; expert 0 has 200 rows, expert 3 57
     _ffn_case(wl, idx)
+
+
+@pytest.mark.parametrize("name,C", [("mixtral_prefill", 1.0), ("mixtral_prefill", 1.25), ("qwen3_mixed", 1.5),
+                                    ("dsv3_skewed_prefill", 1.0), ("tiny", 2.0)])
+def test_dispatch_with_capacity_matches_oracle(name, C):
+    wl = moe_synth.workload(name)
+    cap = moe.capacity_for(C, wl.T, wl.k, wl.E)
+    shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, capacity=cap)
+    ridx, _, _ = oracle.route(moe_synth.host_logits(wl), wl.k)
+    ref = oracle.dispatch(ridx, wl.E, wl.R, capacity=cap)
+    x_dev = moe_synth.device_inputs(wl, weights=False)["x"]
+    o = _gpu_dispatch(shape, x_dev, ridx)
+    assert o["status"] == 0
+    _check_dispatch(o, ref, moe_synth.host_x(wl) if wl.T * wl.d <= (1 << 24) else None, wl.k)
+    assert wl.T * wl.k - int(o["expert_offsets"][-1].item()) == ref["dropped"]

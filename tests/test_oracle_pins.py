@@ -292,3 +292,53 @@ def test_sorted_path_equals_naive_per_token_loop():
     res = oracle.layer(x, lg, w13, w2, wl.k, wl.R, w13s, w2s)
     naive = oracle.naive_token_loop(x, res["topk_idx"], res["topk_gate"], w13, w2, w13s, w2s)
     assert np.max(np.abs(res["out"] - naive)) <= 1e-12 * np.max(np.abs(naive))
+
+
+# ---------------------------------------------------------------------------
+# capacity factor (§5 "Mitigations" 1): keep the first `capacity` per expert
+# ---------------------------------------------------------------------------
+
+def test_capacity_on_the_worked_example():
+    """C = 1.25 ("typical" on the page): capacity = 1.25 * 512 / 8 = 80 per expert."""
+    g = json.load(open(os.path.join(GOLDEN, "expert_parallelism_s5_imbalance.json")))
+    counts = np.array(g["counts"])
+    idx, _, _ = oracle.route(_onehot_logits(counts, 7), 1)
+    cap = math.ceil(1.25 * g["T"] / g["E"])
+    assert cap == 80
+    d = oracle.dispatch(idx, g["E"], g["E"], capacity=cap)
+    kept = np.minimum(counts, cap)
+    assert list(d["expert_counts"]) == kept.tolist() == [80, 80, 78, 62, 48, 40, 31, 18]
+    assert d["dropped"] == int((counts - kept).sum()) == 75
+    # the capacity bounds the imbalance: 80 * 8 / 437 instead of 140 * 8 / 512
+    assert d["imbalance"][1] == np.float32(640 / 437)
+    assert d["imbalance"][1] < np.float32(2.1875)
+
+
+@pytest.mark.parametrize("T,E,k,cap", [(300, 8, 2, 50), (257, 16, 4, 1), (64, 5, 3, 1000), (129, 64, 8, 7)])
+def test_capacity_keeps_the_first_assignments_in_order(T, E, k, cap):
+    idx = np.random.default_rng(T + cap).integers(0, E, size=(T, k)).astype(np.int32)
+    d = oracle.dispatch(idx, E, 1, capacity=cap)
+    flat = idx.reshape(-1)
+    keep = np.zeros(T * k, bool)
+    for e in range(E):                       # brute force: the first `cap` of each expert, in order
+        keep[np.flatnonzero(flat == e)[:cap]] = True
+    assert np.array_equal(d["assign_row"] >= 0, keep)
+    assert d["dropped"] == int((~keep).sum())
+    assert list(d["row_src"][:keep.sum()]) == sorted(np.flatnonzero(keep), key=lambda a: (flat[a], a))
+    assert np.all(d["row_src"][keep.sum():] == -1)
+    if cap >= max(np.bincount(flat, minlength=E)):   # a capacity nobody reaches changes nothing
+        free = oracle.dispatch(idx, E, 1)
+        for n in ("expert_counts", "row_src", "assign_row"):
+            assert np.array_equal(d[n], free[n])
+
+
+def test_capacity_layer_equals_naive_loop_without_dropped_assignments():
+    wl = moe_synth.Workload("cap", T=40, d=32, E=4, k=2, f=48, R=2, bias_kind="hot", n_hot=1, beta=2.0)
+    x, lg = moe_synth.host_x(wl), moe_synth.host_logits(wl)
+    w13, w2 = moe_synth.host_w13(wl), moe_synth.host_w2(wl)
+    res = oracle.layer(x, lg, w13, w2, wl.k, wl.R, capacity=12)
+    assert res["dropped"] > 0
+    idx = res["topk_idx"].copy()
+    idx.reshape(-1)[res["assign_row"] < 0] = -1          # a dropped assignment adds nothing
+    naive = oracle.naive_token_loop(x, idx, res["topk_gate"], w13, w2)
+    assert np.max(np.abs(res["out"] - naive)) <= 1e-12 * np.max(np.abs(naive))
