@@ -395,6 +395,87 @@ def run_gpu(args, wl, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# regime sweep: per-expert cost against activated experts and tokens per expert
+# ---------------------------------------------------------------------------
+
+def fit_max_affine(G, N, t, iters=50):
+    """Fit t = max(a + b*G, c + beta*N) by alternating least squares over the two
+    regimes (weight streaming: cost per activated expert; compute: cost per token)."""
+    import numpy as np
+    G, N, t = (np.asarray(v, dtype=np.float64) for v in (G, N, t))
+    n = N / np.maximum(G, 1)
+    regime = n >= np.median(n)  # True: compute
+    params = None
+    for _ in range(iters):
+        if regime.all() or (~regime).all():
+            regime = n >= np.median(n)
+        A1 = np.stack([np.ones((~regime).sum()), G[~regime]], 1)
+        A2 = np.stack([np.ones(regime.sum()), N[regime]], 1)
+        (a, b), *_ = np.linalg.lstsq(A1, t[~regime], rcond=None)
+        (c, beta), *_ = np.linalg.lstsq(A2, t[regime], rcond=None)
+        new = (c + beta * N) > (a + b * G)
+        params = (a, b, c, beta)
+        if (new == regime).all():
+            break
+        regime = new
+    a, b, c, beta = params
+    pred = np.maximum(a + b * G, c + beta * N)
+    return dict(a=a, b=b, c=c, beta=beta, n_star=b / beta if beta > 0 else None,
+                rel_rms=float(np.sqrt(np.mean(((pred - t) / t) ** 2))))
+
+
+def run_regime_sweep(args):
+    """Expert FFN time of G experts with n tokens each (d, f of a DeepSeek-V3 expert), through
+    moe_expert_ffn; fits the max-affine model and reports the crossover n* = b / beta."""
+    import statistics
+
+    import torch
+
+    import combine_warp_top_expert_b200 as moe
+    import moe_synth
+    d, f = args.regime_d, args.regime_f
+    Gs = [1, 8, 32, 64, 148, 256]
+    ns = [1, 8, 16, 32, 64, 96, 128, 160, 192, 224, 256, 320, 384, 512, 768, 1024]
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    rows = []
+    for G in Gs:
+        wl = moe_synth.Workload("regime", T=1, d=d, E=G, k=1, f=f, R=1)
+        dvw = moe_synth.device_inputs(wl)
+        for n in ns:
+            A = G * n
+            shape = moe.Shape(T=A, d=d, E=G, k=1, f=f, R=1)
+            xw = moe_synth.device_inputs(wl.with_(T=A, seed=1), weights=False)["x"]
+            offs = (torch.arange(G + 1, dtype=torch.int32, device="cuda") * n).contiguous()
+            y = torch.empty((A, d), dtype=torch.bfloat16, device="cuda")
+            ws = moe.new_workspace(shape)
+            ts = []
+            for rep in range(3 + 5):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                moe.moe_expert_ffn(shape, xw, offs, dvw["w13"], dvw["w2"], None, None, None, y, None, ws)
+                e1.record()
+                torch.cuda.synchronize()
+                if rep >= 3:
+                    ts.append(e0.elapsed_time(e1))
+            ms = statistics.median(ts)
+            assert moe.get_status(ws) == 0
+            rows.append(dict(G=G, n=n, N=A, ms=ms, tflops=6.0 * A * d * f / (ms * 1e-3) / 1e12,
+                             weight_gbs=G * 3 * d * f * 2 / (ms * 1e-3) / 1e9))
+            print(json.dumps(dict(regime_point=rows[-1])), flush=True)
+            del xw, y, ws
+        del dvw
+        torch.cuda.empty_cache()
+    full = [r for r in rows if r["G"] >= 32]  # enough experts to occupy every SM
+    for name, key in (("tokens", lambda r: r["N"]), ("tile_rounded_tokens", lambda r: r["G"] * -(-r["n"] // 128) * 128)):
+        fit = fit_max_affine([r["G"] for r in full], [key(r) for r in full], [r["ms"] for r in full])
+        fit.update(d=d, f=f, unit="ms", N=name, model="t = max(a + b*G, c + beta*N), G >= 32",
+                   b_gbs=3 * d * f * 2 / (fit["b"] * 1e-3) / 1e9,
+                   beta_tflops=6.0 * d * f / (fit["beta"] * 1e-3) / 1e12)
+        print(json.dumps(dict(regime_fit=fit)), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -407,12 +488,19 @@ def main():
                     help="grouped-GEMM tiles: per-GEMM choice (auto), single-CTA 128-row, or CTA-pair 256x256")
     ap.add_argument("--capacity-factor", type=float, default=None,
                     help="per-expert capacity ceil(C*T*k/E); excess assignments are dropped (default: none)")
+    ap.add_argument("--regime-sweep", action="store_true",
+                    help="sweep activated experts x tokens per expert and fit t = max(a + b*G, c + beta*N)")
+    ap.add_argument("--regime-d", type=int, default=7168)
+    ap.add_argument("--regime-f", type=int, default=2048)
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the workload's batch size T (smaller cases for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
 
+    if args.regime_sweep:
+        run_regime_sweep(args)
+        return
     import moe_synth
     wl = moe_synth.workload(args.config)
     if args.tokens is not None:

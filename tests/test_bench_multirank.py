@@ -51,3 +51,18 @@ def test_single_rank_is_identity():
     import bench
     assert bench.max_over_ranks(3.5, 1) == 3.5
     assert bench.aggregate_throughput(128, 10, 1, 2.0) == 640.0
+
+
+def test_max_affine_fit_recovers_known_regimes():
+    """The regime fit of bench.py --regime-sweep recovers a known max-affine profile."""
+    sys.path.insert(0, ROOT)
+    import bench
+    G, N, t = [], [], []
+    for g in (1, 8, 32, 64, 148, 256):
+        for n in (1, 8, 16, 32, 64, 128, 192, 256, 384, 512, 1024):
+            G.append(g)
+            N.append(g * n)
+            t.append(max(0.01 + 0.0135 * g, 0.02 + 6.3e-5 * g * n))
+    fit = bench.fit_max_affine(G, N, t)
+    assert fit["b"] == pytest.approx(0.0135) and fit["beta"] == pytest.approx(6.3e-5)
+    assert fit["n_star"] == pytest.approx(0.0135 / 6.3e-5) and fit["rel_rms"] < 1e-9
