@@ -312,6 +312,15 @@ def test_expert_ffn_with_empty_and_full_experts(gemm_policy):
     _ffn_case(wl, idx)
 
 
+@pytest.mark.parametrize("rows", [1, 15, 16, 17, 31, 32, 33, 63, 96, 127, 128, 129, 240, 255, 256, 257])
+def test_expert_ffn_tail_sizes(rows, gemm_policy):
+    """Ragged ends of every size class around the 32-row store blocks and the 128/256-row tiles."""
+    wl = moe_synth.Workload("tail", T=rows + 40, d=256, E=3, k=1, f=256, R=1, n_shared=1)
+    idx = np.full((wl.T, 1), 2, np.int32)
+    idx[:rows, 0] = 0          # expert 0: `rows` rows, expert 1 empty, expert 2: 40 rows
+    _ffn_case(wl, idx)
+
+
 @pytest.mark.parametrize("name,C", [("mixtral_prefill", 1.0), ("mixtral_prefill", 1.25), ("qwen3_mixed", 1.5),
                                     ("dsv3_skewed_prefill", 1.0), ("tiny", 2.0)])
 def test_dispatch_with_capacity_matches_oracle(name, C):
