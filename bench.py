@@ -263,7 +263,7 @@ def run_gpu(args, wl, rank, world, local_rank):
     cap = moe.capacity_for(args.capacity_factor, wl.T, wl.k, wl.E) if args.capacity_factor else 0
     shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, n_shared=wl.n_shared, capacity=cap)
     dv = moe_synth.device_inputs(wl_r, device=dev)
-    layer = moe.MoELayer(shape, dv["w13"], dv["w2"], dv.get("w13s"), dv.get("w2s"), device=dev)
+    layer = moe.MoELayer(shape, dv["w13"], dv["w2"], dv.get("w13s"), dv.get("w2s"), device=dev, gather=args.gather)
     o = layer.outs
     ws = layer.ws
     stream = torch.cuda.current_stream(dev)
@@ -276,8 +276,12 @@ def run_gpu(args, wl, rank, world, local_rank):
         moe.moe_dispatch(shape, dv["x"], o["topk_idx"], o["expert_counts"], o["expert_offsets"], o["rank_counts"],
                          o["rank_offsets"], o["row_src"], o["assign_row"], o["x_perm"], o["imbalance"], ws, stream)
         evs[2].record(stream)
-        moe.moe_expert_gate_up(shape, o["x_perm"], o["expert_offsets"], dv["w13"], dv["x"], dv.get("w13s"), ws,
-                               stream)
+        if args.gather:
+            moe.moe_expert_gate_up_gather(shape, dv["x"], o["row_src"], o["expert_offsets"], dv["w13"],
+                                          dv.get("w13s"), ws, stream)
+        else:
+            moe.moe_expert_gate_up(shape, o["x_perm"], o["expert_offsets"], dv["w13"], dv["x"], dv.get("w13s"), ws,
+                                   stream)
         evs[3].record(stream)
         moe.moe_expert_down(shape, o["expert_offsets"], dv["w2"], dv.get("w2s"), o["y_perm"], o.get("y_shared"), ws,
                             stream)
@@ -368,6 +372,7 @@ def run_gpu(args, wl, rank, world, local_rank):
                    "n_shared": wl.n_shared, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "flushed between steps (512 MiB write, outside the step's events)",
                    "gemm_tiles": args.gemm_policy,
+                   "x_perm": "not materialised (rows gathered in the gate/up GEMM)" if args.gather else "materialised",
                    "capacity_factor": args.capacity_factor, "capacity": cap,
                    "dropped_fraction": 1.0 - sum(counts) / float(wl.T * wl.k) if wl.T else 0.0,
                    "experts_active": work["_n_act"], "imbalance_rank_expert": imbalance,
@@ -492,6 +497,8 @@ def main():
                     help="sweep activated experts x tokens per expert and fit t = max(a + b*G, c + beta*N)")
     ap.add_argument("--regime-d", type=int, default=7168)
     ap.add_argument("--regime-f", type=int, default=2048)
+    ap.add_argument("--gather", action="store_true",
+                    help="no x_perm: dispatch writes indices only and the gate/up GEMM gathers rows of x itself")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the workload's batch size T (smaller cases for profiling)")
     args = ap.parse_args()

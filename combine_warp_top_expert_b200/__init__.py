@@ -24,7 +24,7 @@ ABI_FUNCTIONS = (
     "moe_workspace_bytes", "moe_clear_status", "moe_get_status", "moe_route", "moe_dispatch", "moe_expert_ffn",
     "moe_combine", "moe_layer", "moe_status_string", "moe_last_cuda_error", "moe_set_wait_timeout_ns",
     "moe_expert_gate_up", "moe_expert_down", "moe_dispatch_static", "moe_set_gemm_policy",
-    "moe_set_test_stall",
+    "moe_set_test_stall", "moe_expert_gate_up_gather",
 )
 GEMM_AUTO, GEMM_SINGLE, GEMM_PAIR = 0, 1, 2
 
@@ -76,6 +76,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     L.moe_expert_ffn.argtypes = [shp] + [vp] * 9 + [vp, sz, vp]
     L.moe_expert_gate_up.restype = st
     L.moe_expert_gate_up.argtypes = [shp] + [vp] * 5 + [vp, sz, vp]
+    L.moe_expert_gate_up_gather.restype = st
+    L.moe_expert_gate_up_gather.argtypes = [shp] + [vp] * 5 + [vp, sz, vp]
     L.moe_expert_down.restype = st
     L.moe_expert_down.argtypes = [shp] + [vp] * 5 + [vp, sz, vp]
     L.moe_combine.restype = st
@@ -217,7 +219,7 @@ def moe_dispatch(shape: Shape, x, topk_idx, expert_counts, expert_offsets, rank_
     _dev(rank_offsets, i32, (shape.R + 1,), "rank_offsets")
     _dev(row_src, i32, (shape.A,), "row_src")
     _dev(assign_row, i32, (shape.A,), "assign_row")
-    _dev(x_perm, bf, (shape.A, shape.d), "x_perm")
+    _dev(x_perm, bf, (shape.A, shape.d), "x_perm")  # None: indices only
     _dev(imbalance, torch.float32, (2,), "imbalance")
     _check("moe_dispatch", load().moe_dispatch(
         ctypes.byref(shape.c()), _ptr(x), _ptr(topk_idx), _ptr(expert_counts), _ptr(expert_offsets),
@@ -258,6 +260,21 @@ def moe_expert_gate_up(shape: Shape, x_perm, expert_offsets, w13, x, w13s, ws, s
         ws.numel(), _stream(stream)))
 
 
+def moe_expert_gate_up_gather(shape: Shape, x, row_src, expert_offsets, w13, w13s, ws, stream=None):
+    """GEMM1 + SwiGLU gathering its rows from x through row_src (no x_perm)."""
+    import torch
+    bf = torch.bfloat16
+    _dev(x, bf, (shape.T, shape.d), "x")
+    _dev(row_src, torch.int32, (shape.A,), "row_src")
+    _dev(expert_offsets, torch.int32, (shape.E + 1,), "expert_offsets")
+    _dev(w13, bf, (shape.E, 2 * shape.f, shape.d), "w13")
+    if shape.n_shared:
+        _dev(w13s, bf, (2 * shape.f, shape.d), "w13s")
+    _check("moe_expert_gate_up_gather", load().moe_expert_gate_up_gather(
+        ctypes.byref(shape.c()), _ptr(x), _ptr(row_src), _ptr(expert_offsets), _ptr(w13), _ptr(w13s), _ptr(ws),
+        ws.numel(), _stream(stream)))
+
+
 def moe_expert_down(shape: Shape, expert_offsets, w2, w2s, y_perm, y_shared, ws, stream=None):
     """GEMM2 from the workspace's hidden rows (second half of moe_expert_ffn)."""
     import torch
@@ -290,8 +307,9 @@ _LAYER_OUTPUTS = ("topk_idx", "topk_gate", "expert_counts", "expert_offsets", "r
                   "row_src", "assign_row", "x_perm", "imbalance", "y_perm", "y_shared", "out")
 
 
-def alloc_layer_outputs(shape: Shape, device="cuda") -> dict:
-    """Device buffers for every output of moe_layer."""
+def alloc_layer_outputs(shape: Shape, device="cuda", x_perm: bool = True) -> dict:
+    """Device buffers for every output of moe_layer (x_perm=False: the layer gathers
+    rows of x inside the grouped GEMM and x_perm is not materialised)."""
     import torch
     i32, f32, bf = torch.int32, torch.float32, torch.bfloat16
     T, k, E, R, d, A = shape.T, shape.k, shape.E, shape.R, shape.d, shape.A
@@ -304,7 +322,7 @@ def alloc_layer_outputs(shape: Shape, device="cuda") -> dict:
         rank_offsets=torch.empty((R + 1,), dtype=i32, device=device),
         row_src=torch.empty((A,), dtype=i32, device=device),
         assign_row=torch.empty((A,), dtype=i32, device=device),
-        x_perm=torch.empty((A, d), dtype=bf, device=device),
+        x_perm=torch.empty((A, d), dtype=bf, device=device) if x_perm else None,
         imbalance=torch.empty((2,), dtype=f32, device=device),
         y_perm=torch.empty((A, d), dtype=bf, device=device),
         y_shared=torch.empty((T, d), dtype=bf, device=device) if shape.n_shared else None,
@@ -334,11 +352,13 @@ def moe_layer(shape: Shape, logits, x, w13, w2, w13s, w2s, outs: dict, ws, strea
 class MoELayer:
     """Weights resident on the device plus a reusable workspace and output set."""
 
-    def __init__(self, shape: Shape, w13, w2, w13s=None, w2s=None, device="cuda"):
+    def __init__(self, shape: Shape, w13, w2, w13s=None, w2s=None, device="cuda", gather: bool = False):
+        """gather=True: no x_perm; the grouped GEMM gathers the dispatched rows of x itself."""
         self.shape = shape
         self.w13, self.w2, self.w13s, self.w2s = w13, w2, w13s, w2s
+        self.gather = gather
         self.ws = new_workspace(shape, device)
-        self.outs = alloc_layer_outputs(shape, device)
+        self.outs = alloc_layer_outputs(shape, device, x_perm=not gather)
 
     def __call__(self, logits, x, stream=None) -> dict:
         return moe_layer(self.shape, logits, x, self.w13, self.w2, self.w13s, self.w2s, self.outs, self.ws, stream)
@@ -357,7 +377,7 @@ class MoELayer:
         s_comp = stream or torch.cuda.current_stream(self.ws.device)
         if not hasattr(self, "_slots"):
             dev = self.ws.device
-            self._slots = [dict(outs=alloc_layer_outputs(self.shape, dev),
+            self._slots = [dict(outs=alloc_layer_outputs(self.shape, dev, x_perm=not self.gather),
                                 x=torch.empty((self.shape.T, self.shape.d), dtype=torch.bfloat16, device=dev),
                                 logits=torch.empty((self.shape.T, self.shape.E), dtype=torch.float32, device=dev),
                                 ev_in=torch.cuda.Event(), ev_done=torch.cuda.Event(), ev_out=torch.cuda.Event(),

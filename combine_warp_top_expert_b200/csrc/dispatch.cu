@@ -237,6 +237,7 @@ __global__ void __launch_bounds__(256) dispatch_permute_kernel(
         assign_row[a] = pos;
       }
     }
+    if (x_perm == nullptr) continue; /* index-only dispatch */
     int64_t dst[kMaxK];
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) {
@@ -305,7 +306,13 @@ cudaError_t launch_dispatch(const moe_shape_t& s, const WsLayout& L, uint8_t* ws
   dispatch_count_kernel<<<(unsigned)L.n_chunks, kHistThreads, smem, stream>>>(
       topk_idx, L.A, s.E, s.R, cap, chunk_assign, L.n_chunks, chunk, lrank, status, ticket, expert_counts,
       expert_offsets, rank_counts, rank_offsets, imbalance, row_src);
-  const RowSlices rs = row_slices(s.T, s.d);
+  RowSlices rs = row_slices(s.T, s.d);
+  if (x_perm == nullptr) { /* indices only: one warp per token */
+    rs.slices = 1;
+    rs.vps = s.d / 8;
+    const int64_t blocks = ((int64_t)s.T + 7) / 8, cap = (int64_t)num_sms() * 8;
+    rs.blocks = (int)(blocks > cap ? cap : blocks);
+  }
   dispatch_permute_kernel<4><<<(unsigned)rs.blocks, 256, 0, stream>>>(
       x, topk_idx, chunk, lrank, expert_offsets, s.T, s.d, s.E, s.k, cap, L.tok_per_chunk, rs.slices, rs.vps,
       row_src, assign_row, x_perm);

@@ -77,6 +77,9 @@ struct FfnParams {
   uint32_t* status;
   uint64_t timeout_ns;
   int stall_first_stage; /* test hook: arm the first stage of each CTA's first tile but never load it */
+  const int32_t* row_src;   /* GEMM1 gathering A from x: row_src of dispatch (null: A is x_perm) */
+  const uint16_t* gather_x; /* x [T, d] rows to gather from */
+  int k;                    /* experts per token (token of assignment a = a / k) */
 };
 
 struct Tile {
@@ -314,7 +317,7 @@ struct SingleCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-template <int MODE, int BN>
+template <int MODE, int BN, bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
     ffn_gemm_single_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                            const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
@@ -333,9 +336,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  static_assert(!GATHER || MODE == 0, "only GEMM1 gathers its A rows");
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&ctl->full[s], 1);
+      /* gathering: lane 0's expect_tx arrival + one arrival per producer lane */
+      mbar_init(&ctl->full[s], GATHER ? 33 : 1);
       mbar_init(&ctl->empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -376,8 +381,73 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int KB = p.K / BK;
 
   if (warp == 0) {
-    if (lane == 0) {
-      /* ---------------- TMA producer ---------------- */
+    if constexpr (!GATHER) {
+      if (lane == 0) {
+        /* ---------------- TMA producer ---------------- */
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t armed_phase[STAGES];
+        bool armed[STAGES];
+  #pragma unroll
+        for (int s = 0; s < STAGES; ++s) {
+          armed[s] = false;
+          armed_phase[s] = 0;
+        }
+        bool abort = false;
+        for (int64_t L = blockIdx.x; L < total && !abort; L += gridDim.x) {
+          const Tile t = decode_tile<MODE, 128, BN>(L, p, ctl->off, ctl->mpref, ctl->hpref);
+          const bool shared = t.g >= p.E;
+          const CUtensorMap* mA = shared ? &tmA1 : &tmA0;
+          const CUtensorMap* mB = shared ? &tmB1 : &tmB0;
+          for (int kb = 0; kb < KB; ++kb) {
+            if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, p.timeout_ns, s_abort)) {
+              abort = true;
+              break;
+            }
+            mbar_arrive_expect_tx(&ctl->full[stage], C::STAGE_BYTES);
+            if (p.stall_first_stage && L == blockIdx.x && kb == 0) {
+              /* test hook: this stage's bytes never arrive, so the MMA's bounded wait runs out */
+              if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1u;
+              }
+              continue;
+            }
+            armed[stage] = true;
+            armed_phase[stage] = phase;
+            uint8_t* a_dst = sA + stage * HALF_TILE;
+            uint8_t* b_dst = sB + stage * C::B_BYTES;
+            tma_load_2d(a_dst, mA, &ctl->full[stage], kb * BK, t.a_row);
+            if (MODE == 0) {
+              tma_load_2d(b_dst, mB, &ctl->full[stage], kb * BK, t.b_row);
+              tma_load_2d(b_dst + HALF_TILE, mB, &ctl->full[stage], kb * BK, t.b_row + p.f);
+            } else {
+              tma_load_2d(b_dst, mB, &ctl->full[stage], kb * BK, t.b_row);
+            }
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+        if (abort) {
+          raise_status(p.status, MOE_DEV_TIMEOUT);
+          *s_abort = 1;
+        }
+        /* every armed stage's copies must land before the CTA may exit */
+        for (int s = 0; s < STAGES; ++s)
+          if (armed[s]) mbar_wait(&ctl->full[s], armed_phase[s], kDrainNs, nullptr);
+      }
+    } else {
+      /* ---------------- producer warp, A gathered from x ----------------
+       * Lane 0 waits for free stages, arms them and TMA-loads B (and A for the
+       * shared expert, whose rows are x itself). The routed rows of GEMM1 come
+       * straight from x: row p of expert e is token row_src[p] / k. The whole warp
+       * copies them with 16-byte cp.async into the 128-byte swizzled layout of the
+       * stage: lane l moves 16-byte chunk l % 8 of rows l / 8 + 4 i (i < 32), so one
+       * instruction covers four 128-byte row segments, and each lane's byte offsets
+       * into x stay in registers for the whole tile. Every lane arrives on every
+       * stage barrier once its copies have landed (the barrier counts 32 + 1). */
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed_phase[STAGES];
@@ -388,49 +458,84 @@ __global__ void __launch_bounds__(kThreads, 1)
         armed_phase[s] = 0;
       }
       bool abort = false;
+      const int chunk = lane & 7, row0 = lane >> 3;
+      /* swizzle of rows row0 + 4 i: (row0 + 4 i) % 8 == row0 ^ (4 (i % 2)) since row0 < 4 */
+      const uint32_t sw_even = (uint32_t)(chunk ^ row0) << 4, sw_odd = (uint32_t)(chunk ^ row0 ^ 4) << 4;
+      const uint32_t row_bytes = (uint32_t)p.d * 2u; /* T * d * 2 < 2^32 is checked on the host */
+      const char* xk0 = reinterpret_cast<const char*>(p.gather_x) + chunk * 16;
       for (int64_t L = blockIdx.x; L < total && !abort; L += gridDim.x) {
         const Tile t = decode_tile<MODE, 128, BN>(L, p, ctl->off, ctl->mpref, ctl->hpref);
         const bool shared = t.g >= p.E;
-        const CUtensorMap* mA = shared ? &tmA1 : &tmA0;
-        const CUtensorMap* mB = shared ? &tmB1 : &tmB0;
+        uint32_t goff[32];
+        if (!shared) {
+          /* rows past the expert's end read token 0 (computed, never stored); a row index
+           * outside [0, T * k) reads token 0 too and raises MOE_DEV_BOUNDS */
+          const int r_end = ctl->off[t.g + 1];
+          const int r0 = ctl->off[t.g] + t.m * 128 + row0;
+          bool bad = false;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int r = r0 + 4 * i;
+            uint32_t tok = r < r_end ? (uint32_t)__ldg(p.row_src + r) / (uint32_t)p.k : 0u;
+            if (tok >= (uint32_t)p.T) {
+              bad = true;
+              tok = 0u;
+            }
+            goff[i] = tok * row_bytes;
+          }
+          if (bad) raise_status(p.status, MOE_DEV_BOUNDS);
+        }
+        const uint32_t tx_bytes = shared ? C::STAGE_BYTES : C::B_BYTES;
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, p.timeout_ns, s_abort)) {
+          int ok = 1, skip = 0;
+          uint8_t* a_dst = sA + stage * HALF_TILE;
+          uint8_t* b_dst = sB + stage * C::B_BYTES;
+          if (lane == 0) {
+            ok = mbar_wait(&ctl->empty[stage], phase ^ 1u, p.timeout_ns, s_abort) ? 1 : 0;
+            if (ok) {
+              mbar_arrive_expect_tx(&ctl->full[stage], tx_bytes);
+              if (p.stall_first_stage && L == blockIdx.x && kb == 0) {
+                skip = 1; /* test hook: this stage's bytes never arrive, so the MMA's bounded wait runs out */
+              } else {
+                armed[stage] = true;
+                armed_phase[stage] = phase;
+                /* the weights first: they come from DRAM, the rows of x mostly from L2 */
+                const CUtensorMap* mB = shared ? &tmB1 : &tmB0;
+                tma_load_2d(b_dst, mB, &ctl->full[stage], kb * BK, t.b_row);
+                tma_load_2d(b_dst + HALF_TILE, mB, &ctl->full[stage], kb * BK, t.b_row + p.f);
+                if (shared) tma_load_2d(a_dst, &tmA1, &ctl->full[stage], kb * BK, t.a_row);
+              }
+            }
+          }
+          ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+          skip = __shfl_sync(0xFFFFFFFFu, skip, 0);
+          if (!ok) {
             abort = true;
             break;
           }
-          mbar_arrive_expect_tx(&ctl->full[stage], C::STAGE_BYTES);
-          if (p.stall_first_stage && L == blockIdx.x && kb == 0) {
-            /* test hook: this stage's bytes never arrive, so the MMA's bounded wait runs out */
-            if (++stage == STAGES) {
-              stage = 0;
-              phase ^= 1u;
-            }
-            continue;
+          if (!shared && !skip) {
+            const uint32_t a_base = smem_u32(a_dst) + (uint32_t)row0 * 128u;
+            const char* xk = xk0 + (int64_t)kb * (BK * 2);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              cp_async_16(a_base + (uint32_t)i * 512u + ((i & 1) ? sw_odd : sw_even), xk + goff[i]);
           }
-          armed[stage] = true;
-          armed_phase[stage] = phase;
-          uint8_t* a_dst = sA + stage * HALF_TILE;
-          uint8_t* b_dst = sB + stage * C::B_BYTES;
-          tma_load_2d(a_dst, mA, &ctl->full[stage], kb * BK, t.a_row);
-          if (MODE == 0) {
-            tma_load_2d(b_dst, mB, &ctl->full[stage], kb * BK, t.b_row);
-            tma_load_2d(b_dst + HALF_TILE, mB, &ctl->full[stage], kb * BK, t.b_row + p.f);
-          } else {
-            tma_load_2d(b_dst, mB, &ctl->full[stage], kb * BK, t.b_row);
-          }
+          cp_async_mbar_arrive(&ctl->full[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
-      if (abort) {
-        raise_status(p.status, MOE_DEV_TIMEOUT);
-        *s_abort = 1;
+      if (lane == 0) {
+        if (abort) {
+          raise_status(p.status, MOE_DEV_TIMEOUT);
+          *s_abort = 1;
+        }
+        /* every armed stage's copies must land before the CTA may exit */
+        for (int s = 0; s < STAGES; ++s)
+          if (armed[s]) mbar_wait(&ctl->full[s], armed_phase[s], kDrainNs, nullptr);
       }
-      /* every armed stage's copies must land before the CTA may exit */
-      for (int s = 0; s < STAGES; ++s)
-        if (armed[s]) mbar_wait(&ctl->full[s], armed_phase[s], kDrainNs, nullptr);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -452,6 +557,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             abort = true;
             break;
           }
+          /* rows gathered by cp.async were written through the generic proxy: order them
+           * before the tensor core reads the stage through the async proxy */
+          if constexpr (GATHER) fence_proxy_async_shared();
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + stage * HALF_TILE);
           const uint32_t b_addr = smem_u32(sB + stage * C::B_BYTES);
@@ -779,18 +887,19 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uin
   return r == CUDA_SUCCESS;
 }
 
-template <int MODE, int BN>
+template <int MODE, int BN, bool GATHER = false>
 cudaError_t launch_single(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0, const CUtensorMap& b1,
                           const CUtensorMap& o0, const CUtensorMap& o1, const FfnParams& p, cudaStream_t stream) {
   using C = SingleCfg<MODE, BN>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(ffn_gemm_single_kernel<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)C::SMEM_BYTES);
+    attr_err = cudaFuncSetAttribute(ffn_gemm_single_kernel<MODE, BN, GATHER>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  ffn_gemm_single_kernel<MODE, BN><<<num_sms(), kThreads, C::SMEM_BYTES, stream>>>(a0, a1, b0, b1, o0, o1, p);
+  ffn_gemm_single_kernel<MODE, BN, GATHER>
+      <<<num_sms(), kThreads, C::SMEM_BYTES, stream>>>(a0, a1, b0, b1, o0, o1, p);
   return cudaGetLastError();
 }
 
@@ -863,23 +972,32 @@ FfnParams base_params(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, cons
   p.status = reinterpret_cast<uint32_t*>(ws + L.status);
   p.timeout_ns = wait_timeout_ns();
   p.stall_first_stage = test_stall() ? 1 : 0;
+  p.row_src = nullptr;
+  p.gather_x = nullptr;
+  p.k = s.k;
   return p;
 }
 
 }  // namespace
 
 cudaError_t launch_gate_up(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const uint16_t* x_perm,
-                           const int32_t* expert_offsets, const uint16_t* w13, const uint16_t* x,
-                           const uint16_t* w13s, cudaStream_t stream) {
+                           const int32_t* row_src, const int32_t* expert_offsets, const uint16_t* w13,
+                           const uint16_t* x, const uint16_t* w13s, cudaStream_t stream) {
   if (s.T == 0) return cudaSuccess;
   const bool sh = s.n_shared != 0;
+  const bool gather = x_perm == nullptr; /* A rows gathered from x through row_src */
   /* 128-row single-CTA tiles pad small experts less and measured faster for this GEMM's
-   * short K; CTA-pair tiles only on request */
-  const bool pair = gemm_policy() == kGemmPair;
+   * short K; CTA-pair tiles only on request (and never when gathering) */
+  const bool pair = !gather && gemm_policy() == kGemmPair;
   CUtensorMap a0, a1, b0, b1;
-  /* A = x_perm [A, d] (routed) / x [T, d] (shared); B = w13 [E*2f, d] / w13s [2f, d] */
-  if (!make_map(&a0, x_perm, (uint64_t)L.A, s.d, 128)) return cudaErrorInvalidValue;
-  if (!make_map(&a1, sh ? x : x_perm, sh ? (uint64_t)s.T : (uint64_t)L.A, s.d, 128)) return cudaErrorInvalidValue;
+  /* A = x_perm [A, d] (routed; rows of x gathered by the producer warp instead when x_perm is
+   * null) / x [T, d] (shared);
+   * B = w13 [E*2f, d] / w13s [2f, d] */
+  if (gather && (uint64_t)s.T * (uint64_t)s.d * 2u > 0xFFFFFFFFull) return cudaErrorInvalidValue;
+  if (!make_map(&a0, gather ? x : x_perm, gather ? (uint64_t)s.T : (uint64_t)L.A, s.d, 128))
+    return cudaErrorInvalidValue;
+  if (!make_map(&a1, sh || gather ? x : x_perm, sh || gather ? (uint64_t)s.T : (uint64_t)L.A, s.d, 128))
+    return cudaErrorInvalidValue;
   if (!make_map(&b0, w13, (uint64_t)s.E * 2 * s.f, s.d, 128)) return cudaErrorInvalidValue;
   if (!make_map(&b1, sh ? w13s : w13, sh ? (uint64_t)2 * s.f : (uint64_t)s.E * 2 * s.f, s.d, 128))
     return cudaErrorInvalidValue;
@@ -891,12 +1009,15 @@ cudaError_t launch_gate_up(const moe_shape_t& s, const WsLayout& L, uint8_t* ws,
   p.out0 = reinterpret_cast<uint16_t*>(ws + L.h);
   p.out1 = nullptr;
   p.ld_out = s.f;
+  p.row_src = gather ? row_src : nullptr;
+  p.gather_x = gather ? x : nullptr;
   if (pair) {
     bool launched = false;
     const cudaError_t e = launch_pair<0>(a0, a1, b0, b1, o0, o0, p, stream, &launched);
     if (e != cudaSuccess || launched) return e;
   }
-  return launch_single<0, 256>(a0, a1, b0, b1, o0, o0, p, stream);
+  return gather ? launch_single<0, 256, true>(a0, a1, b0, b1, o0, o0, p, stream)
+                : launch_single<0, 256>(a0, a1, b0, b1, o0, o0, p, stream);
 }
 
 cudaError_t launch_down(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const int32_t* expert_offsets,

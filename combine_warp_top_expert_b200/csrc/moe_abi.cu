@@ -31,6 +31,9 @@ namespace {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+/* GEMM1 gathering rows of x keeps each row's byte offset into x in 32 bits. */
+bool gather_fits(const moe_shape_t& s) { return (uint64_t)s.T * (uint64_t)s.d * 2u <= 0xFFFFFFFFull; }
+
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 }  // namespace
@@ -148,8 +151,8 @@ moe_status_t moe_dispatch(const moe_shape_t* shape, const moe_bf16_t* x, const i
   moe_status_t st = validate_shape(shape);
   if (st != MOE_OK) return st;
   if (!expert_counts || !expert_offsets || !rank_counts || !rank_offsets || !imbalance) return MOE_ERR_INVALID_ARG;
-  if (shape->T > 0 && (!x || !topk_idx || !row_src || !assign_row || !x_perm)) return MOE_ERR_INVALID_ARG;
-  if (shape->T > 0 && (!aligned(x, 16) || !aligned(x_perm, 16))) return MOE_ERR_INVALID_ARG;
+  if (shape->T > 0 && (!topk_idx || !row_src || !assign_row)) return MOE_ERR_INVALID_ARG;
+  if (shape->T > 0 && x_perm && (!x || !aligned(x, 16) || !aligned(x_perm, 16))) return MOE_ERR_INVALID_ARG;
   if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
   const WsLayout L = ws_layout(*shape);
   const cudaError_t e = launch_dispatch(*shape, L, (uint8_t*)ws, x, topk_idx, expert_counts, expert_offsets,
@@ -174,7 +177,8 @@ moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_bf16_t* x_perm, 
     return MOE_ERR_INVALID_ARG;
   if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
   const WsLayout L = ws_layout(*shape);
-  cudaError_t e = launch_gate_up(*shape, L, (uint8_t*)ws, x_perm, expert_offsets, w13, x, w13s, (cudaStream_t)stream);
+  cudaError_t e =
+      launch_gate_up(*shape, L, (uint8_t*)ws, x_perm, nullptr, expert_offsets, w13, x, w13s, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e);
   e = launch_down(*shape, L, (uint8_t*)ws, expert_offsets, w2, w2s, y_perm, shape->n_shared ? y_shared : nullptr,
                   (cudaStream_t)stream);
@@ -191,8 +195,23 @@ moe_status_t moe_expert_gate_up(const moe_shape_t* shape, const moe_bf16_t* x_pe
   if (shape->n_shared && shape->T > 0 && (!x || !w13s || !aligned(x, 16) || !aligned(w13s, 16)))
     return MOE_ERR_INVALID_ARG;
   if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
-  const cudaError_t e = launch_gate_up(*shape, ws_layout(*shape), (uint8_t*)ws, x_perm, expert_offsets, w13, x, w13s,
-                                       (cudaStream_t)stream);
+  const cudaError_t e = launch_gate_up(*shape, ws_layout(*shape), (uint8_t*)ws, x_perm, nullptr, expert_offsets, w13, x,
+                                       w13s, (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+moe_status_t moe_expert_gate_up_gather(const moe_shape_t* shape, const moe_bf16_t* x, const int32_t* row_src,
+                                       const int32_t* expert_offsets, const moe_bf16_t* w13, const moe_bf16_t* w13s,
+                                       void* ws, size_t ws_bytes, void* stream) {
+  moe_status_t st = validate_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!expert_offsets || !w13 || !aligned(w13, 16)) return MOE_ERR_INVALID_ARG;
+  if (shape->T > 0 && (!x || !row_src || !aligned(x, 16))) return MOE_ERR_INVALID_ARG;
+  if (shape->n_shared && shape->T > 0 && (!w13s || !aligned(w13s, 16))) return MOE_ERR_INVALID_ARG;
+  if (!gather_fits(*shape)) return MOE_ERR_UNSUPPORTED;
+  if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
+  const cudaError_t e = launch_gate_up(*shape, ws_layout(*shape), (uint8_t*)ws, nullptr, row_src, expert_offsets, w13,
+                                       x, w13s, (cudaStream_t)stream);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }
 
@@ -235,9 +254,10 @@ moe_status_t moe_layer(const moe_shape_t* shape, const moe_layer_buffers_t* b, v
       !b->imbalance)
     return MOE_ERR_INVALID_ARG;
   if (shape->T > 0 && (!b->logits || !b->x || !b->topk_idx || !b->topk_gate || !b->row_src || !b->assign_row ||
-                       !b->x_perm || !b->y_perm || !b->out))
+                       !b->y_perm || !b->out))
     return MOE_ERR_INVALID_ARG;
   if (shape->n_shared && shape->T > 0 && (!b->w13s || !b->w2s || !b->y_shared)) return MOE_ERR_INVALID_ARG;
+  if (!b->x_perm && !gather_fits(*shape)) return MOE_ERR_UNSUPPORTED;
   const void* al[] = {b->x, b->w13, b->w2, b->w13s, b->w2s, b->x_perm, b->y_perm, b->y_shared, b->out};
   for (const void* p : al)
     if (p && !aligned(p, 16)) return MOE_ERR_INVALID_ARG;
@@ -252,7 +272,8 @@ moe_status_t moe_layer(const moe_shape_t* shape, const moe_layer_buffers_t* b, v
                       b->rank_offsets, b->row_src, b->assign_row, b->x_perm, b->imbalance, s);
   if (e != cudaSuccess) return cuda_fail(e);
   const uint16_t* ysh_in = shape->n_shared ? b->y_shared : nullptr;
-  e = launch_gate_up(*shape, L, w, b->x_perm, b->expert_offsets, b->w13, b->x, b->w13s, s);
+  /* x_perm null: dispatch writes indices only and GEMM1 gathers the rows of x itself */
+  e = launch_gate_up(*shape, L, w, b->x_perm, b->row_src, b->expert_offsets, b->w13, b->x, b->w13s, s);
   if (e != cudaSuccess) return cuda_fail(e);
   e = launch_down(*shape, L, w, b->expert_offsets, b->w2, b->w2s, b->y_perm, shape->n_shared ? b->y_shared : nullptr,
                   s);

@@ -128,6 +128,17 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+/* 16-byte asynchronous copy global -> shared (L2 only). */
+__device__ __forceinline__ void cp_async_16(uint32_t smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_dst), "l"(gmem_src) : "memory");
+}
+
+/* Arrive on `bar` once all cp.async copies issued so far by this thread have landed
+ * (the arrival is counted in the barrier's expected count). */
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 /* 2D tile store shared -> global (bulk async-group of the issuing thread). The
  * shared source must be in the tensor map's swizzled layout. */
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int32_t x, int32_t y) {

@@ -75,10 +75,11 @@ cudaError_t launch_dispatch(const moe_shape_t& s, const WsLayout& L, uint8_t* ws
                             int32_t* rank_counts, int32_t* rank_offsets, int32_t* row_src, int32_t* assign_row,
                             uint16_t* x_perm, float* imbalance, cudaStream_t stream);
 
-/* GEMM1: h (workspace) = silu(A W_gate^T) * (A W_up^T) per expert group */
+/* GEMM1: h (workspace) = silu(A W_gate^T) * (A W_up^T) per expert group; A is
+ * x_perm, or (x_perm null) the rows of x gathered through row_src */
 cudaError_t launch_gate_up(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const uint16_t* x_perm,
-                           const int32_t* expert_offsets, const uint16_t* w13, const uint16_t* x,
-                           const uint16_t* w13s, cudaStream_t stream);
+                           const int32_t* row_src, const int32_t* expert_offsets, const uint16_t* w13,
+                           const uint16_t* x, const uint16_t* w13s, cudaStream_t stream);
 
 /* GEMM2: y_perm / y_shared = h W2^T per expert group */
 cudaError_t launch_down(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const int32_t* expert_offsets,

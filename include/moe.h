@@ -114,6 +114,8 @@ moe_status_t moe_route(const moe_shape_t* shape, const float* logits, int32_t* t
  *   x_perm         [T*k, d] bf16 out: x_perm[assign_row[a]] = x[a / k]; rows are
  *                  expert-contiguous (expert e at [off[e], off[e+1])), so rank-major;
  *                  inside an expert, rows keep assignment order (stable).
+ *                  May be NULL (x may then be NULL too): indices only, no row copies,
+ *                  for moe_expert_gate_up_gather.
  *   imbalance      [2] fp32 out: [0] = max_r rank_counts[r] / mean (= *R / total),
  *                  [1] = max_e expert_counts[e] / mean; {1, 1} when nothing is placed.
  * Capacity (page §5 "Mitigations", capacity factor): with shape->capacity = c > 0
@@ -184,6 +186,23 @@ moe_status_t moe_expert_down(const moe_shape_t* shape, const int32_t* expert_off
                              const moe_bf16_t* w2s, moe_bf16_t* y_perm, moe_bf16_t* y_shared, void* ws,
                              size_t ws_bytes, void* stream);
 
+/* moe_expert_gate_up without x_perm: GEMM1 gathers each row of its tiles from
+ * x itself (row p of expert e is token row_src[p] / k), so the dispatched rows
+ * never make a round trip through HBM. This is the single-GPU form of the
+ * per-expert overlap (PEO) of the page "Balancing and Beyond: Communication-
+ * Centric Optimizations in Expert Parallelism" (key idea): no exchange buffer
+ * is materialised before expert compute.
+ *   x [T, d] bf16 in, row_src [T*k] int32 in (from moe_dispatch, which may be
+ *   called with x_perm = NULL), other arguments as moe_expert_gate_up. Follow it
+ *   with moe_expert_down as usual. h is bit-identical to moe_expert_gate_up's.
+ * Returns MOE_ERR_UNSUPPORTED when T * d * 2 > 2^32 - 1 (row offsets into x are
+ * kept in 32 bits). The rows are copied by one warp with 16-byte cp.async
+ * instead of TMA tiles, which on B200 costs more GEMM time than the x_perm
+ * round trip it saves; moe_expert_gate_up stays the default. */
+moe_status_t moe_expert_gate_up_gather(const moe_shape_t* shape, const moe_bf16_t* x, const int32_t* row_src,
+                                       const int32_t* expert_offsets, const moe_bf16_t* w13, const moe_bf16_t* w13s,
+                                       void* ws, size_t ws_bytes, void* stream);
+
 /* Combine: un-permute and gate-weighted sum, back in original token order.
  * Page "Expert Parallelism" §4 COMBINE.
  *   out[t] = sum_{j<k} topk_gate[t,j] * y_perm[assign_row[t*k+j]] (+ y_shared[t])
@@ -210,7 +229,8 @@ typedef struct moe_layer_buffers {
   int32_t* rank_offsets;     /* [R+1]   out */
   int32_t* row_src;          /* [T*k]   out */
   int32_t* assign_row;       /* [T*k]   out */
-  moe_bf16_t* x_perm;        /* [T*k, d] out */
+  moe_bf16_t* x_perm;        /* [T*k, d] out; NULL: not materialised, GEMM1 gathers rows of x
+                                (as moe_expert_gate_up_gather, same limit) */
   float* imbalance;          /* [2]     out */
   moe_bf16_t* y_perm;        /* [T*k, d] out */
   moe_bf16_t* y_shared;      /* [T, d]  out (NULL if n_shared = 0) */

@@ -107,3 +107,15 @@ def test_status_strings_and_timeout_knob():
     assert lib.moe_set_gemm_policy(0) == 2
     assert lib.moe_set_test_stall(1) == 0
     assert lib.moe_set_test_stall(0) == 1
+
+
+def test_gathering_gemm_rejects_inputs_past_32_bit_row_offsets():
+    """GEMM1 that gathers rows of x keeps byte offsets into x in 32 bits: T*d*2 must fit."""
+    lib = moe.load()
+    big = moe.Shape(T=(1 << 20) + 8, d=2048, E=8, k=2, f=1024, R=2).c()   # x is 4 GiB + 32 KiB
+    assert lib.moe_expert_gate_up_gather(ctypes.byref(big), FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 62,
+                                         None) == moe.MOE_ERR_UNSUPPORTED
+    b = moe.moe_layer_buffers_t(*([FAKE] * len(moe.moe_layer_buffers_t._fields_)))
+    b.x_perm = None
+    b.w13s = b.w2s = b.y_shared = None
+    assert lib.moe_layer(ctypes.byref(big), ctypes.byref(b), FAKE, 1 << 62, None) == moe.MOE_ERR_UNSUPPORTED

@@ -192,3 +192,62 @@ def test_layer_with_capacity_matches_oracle():
     for n in ("expert_counts", "expert_offsets", "row_src", "assign_row"):
         assert np.array_equal(np_i32(outs[n]), res[n]), n
     close(f64(bits(outs["out"])), res["out"], "out with capacity")
+
+
+def _run_layer_gather(wl, capacity=0):
+    dv = moe_synth.device_inputs(wl)
+    shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, n_shared=wl.n_shared, capacity=capacity)
+    layer = moe.MoELayer(shape, dv["w13"], dv["w2"], dv.get("w13s"), dv.get("w2s"), gather=True)
+    outs = layer(dv["logits"], dv["x"])
+    return dv, layer, outs, moe.get_status(layer.ws)
+
+
+def test_layer_gathering_rows_full_parity():
+    """x_perm not materialised: the grouped GEMM gathers the dispatched rows of x itself."""
+    wl = moe_synth.Workload("gsh", T=200, d=256, E=16, k=4, f=256, R=4, n_shared=1, bias_kind="zipf", zipf_s=1.0)
+    dv, layer, outs, status = _run_layer_gather(wl)
+    assert status == 0 and outs["x_perm"] is None
+    _check_routing(wl, outs)
+    res = oracle.layer(moe_synth.host_x(wl), moe_synth.host_logits(wl), moe_synth.host_w13(wl),
+                       moe_synth.host_w2(wl), wl.k, wl.R, moe_synth.host_w13s(wl), moe_synth.host_w2s(wl))
+    close(f64(bits(outs["y_perm"])), res["y_perm"], "y_perm")
+    close(f64(bits(outs["out"])), res["out"], "out")
+
+
+@pytest.mark.parametrize("name,n_tokens", [("mixtral_prefill", 4), ("dsv3_skewed_prefill", 2), ("dsv3_decode", 4)])
+def test_layer_gathering_rows_full_size_sampled(name, n_tokens):
+    import torch
+    wl = moe_synth.workload(name)
+    dv, layer, outs, status = _run_layer_gather(wl)
+    assert status == 0
+    ridx, rgate, ref = _check_routing(wl, outs)
+    _sampled_parity(wl, outs, ridx, rgate, ref, n_tokens, seed=3)
+    del layer, outs, dv
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", ["qwen3_mixed", "dsv3_decode"])
+def test_layer_gathering_rows_is_bit_identical_to_materialised_x_perm(name):
+    """Same A rows, same MMA order: the gathering GEMM changes where rows come from, not the arithmetic."""
+    import torch
+    wl = moe_synth.workload(name)
+    dv = moe_synth.device_inputs(wl)
+    shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, n_shared=wl.n_shared)
+    a = moe.MoELayer(shape, dv["w13"], dv["w2"], dv.get("w13s"), dv.get("w2s"))(dv["logits"], dv["x"])
+    b = moe.MoELayer(shape, dv["w13"], dv["w2"], dv.get("w13s"), dv.get("w2s"), gather=True)(dv["logits"], dv["x"])
+    for n in ("row_src", "assign_row", "expert_offsets", "y_perm", "out"):
+        assert torch.equal(a[n], b[n]), n
+
+
+def test_layer_gathering_rows_with_capacity_matches_oracle():
+    wl = moe_synth.Workload("capg", T=300, d=256, E=8, k=2, f=256, R=4, n_shared=1, bias_kind="zipf", zipf_s=1.0)
+    cap = moe.capacity_for(1.25, wl.T, wl.k, wl.E)
+    dv, layer, outs, status = _run_layer_gather(wl, capacity=cap)
+    assert status == 0
+    res = oracle.layer(moe_synth.host_x(wl), moe_synth.host_logits(wl), moe_synth.host_w13(wl),
+                       moe_synth.host_w2(wl), wl.k, wl.R, moe_synth.host_w13s(wl), moe_synth.host_w2s(wl),
+                       capacity=cap)
+    assert res["dropped"] > 0
+    for n in ("expert_counts", "expert_offsets", "row_src", "assign_row"):
+        assert np.array_equal(np_i32(outs[n]), res[n]), n
+    close(f64(bits(outs["out"])), res["out"], "out with capacity, gathered rows")

@@ -334,3 +334,77 @@ def test_dispatch_with_capacity_matches_oracle(name, C):
     assert o["status"] == 0
     _check_dispatch(o, ref, moe_synth.host_x(wl) if wl.T * wl.d <= (1 << 24) else None, wl.k)
     assert wl.T * wl.k - int(o["expert_offsets"][-1].item()) == ref["dropped"]
+
+
+def _ffn_gather_case(wl, idx=None):
+    """moe_expert_gate_up_gather (rows of x gathered through row_src) + moe_expert_down against the oracle."""
+    torch = _torch()
+    shape = _shape(wl)
+    x_np = moe_synth.host_x(wl)
+    if idx is None:
+        idx, _, _ = oracle.route(moe_synth.host_logits(wl), wl.k)
+    ref = oracle.dispatch(idx, wl.E, wl.R)
+    xp_np = oracle.permute_rows(x_np, ref["row_src"], wl.k)
+    w13, w2 = moe_synth.host_w13(wl), moe_synth.host_w2(wl)
+    w13s = moe_synth.host_w13s(wl) if wl.n_shared else None
+    w2s = moe_synth.host_w2s(wl) if wl.n_shared else None
+    y_ref, ys_ref = oracle.expert_ffn(xp_np, ref["expert_offsets"], w13, w2, x_np, w13s, w2s)
+    y = torch.empty((shape.A, wl.d), dtype=torch.bfloat16, device="cuda")
+    ys = torch.empty((wl.T, wl.d), dtype=torch.bfloat16, device="cuda") if wl.n_shared else None
+    ws = moe.new_workspace(shape)
+    offs = torch.from_numpy(ref["expert_offsets"]).cuda()
+    moe.moe_expert_gate_up_gather(shape, _bf16_dev(x_np), torch.from_numpy(ref["row_src"]).cuda(), offs,
+                                  _bf16_dev(w13), _bf16_dev(w13s) if wl.n_shared else None, ws)
+    moe.moe_expert_down(shape, offs, _bf16_dev(w2), _bf16_dev(w2s) if wl.n_shared else None, y, ys, ws)
+    assert moe.get_status(ws) == 0
+    total = ref["expert_offsets"][-1]
+    for e in range(wl.E):
+        r0, r1 = ref["expert_offsets"][e], ref["expert_offsets"][e + 1]
+        if r1 > r0:
+            close(f64(bits(y))[r0:r1], y_ref[r0:r1], f"y_perm expert {e} (gathered rows)")
+    close(f64(bits(y))[:total], y_ref[:total], "y_perm (gathered rows)")
+    if wl.n_shared:
+        close(f64(bits(ys)), ys_ref, "y_shared")
+
+
+@pytest.mark.parametrize("wl", [
+    moe_synth.workload("tiny"),
+    moe_synth.Workload("skew", T=300, d=256, E=6, k=2, f=384, R=2, n_shared=1, bias_kind="hot", n_hot=1, beta=3.0),
+    moe_synth.Workload("decode", T=16, d=256, E=64, k=8, f=256, R=8, n_shared=1, bias_kind="zipf", zipf_s=1.2),
+    moe_synth.Workload("d384", T=200, d=384, E=4, k=1, f=256, R=2),
+])
+def test_expert_ffn_gathering_rows_from_x(wl, gemm_policy):
+    _ffn_gather_case(wl)
+
+
+def test_index_only_dispatch_equals_full_dispatch():
+    torch = _torch()
+    wl = moe_synth.workload("qwen3_mixed")
+    shape = _shape(wl)
+    ridx, _, _ = oracle.route(moe_synth.host_logits(wl), wl.k)
+    full = _gpu_dispatch(shape, moe_synth.device_inputs(wl, weights=False)["x"], ridx)
+    i32 = torch.int32
+    o = {n: torch.full_like(full[n], -9) for n in ("expert_counts", "expert_offsets", "rank_counts", "rank_offsets",
+                                                     "row_src", "assign_row", "imbalance")}
+    ws = moe.new_workspace(shape)
+    moe.moe_dispatch(shape, None, torch.from_numpy(ridx).cuda(), o["expert_counts"], o["expert_offsets"],
+                     o["rank_counts"], o["rank_offsets"], o["row_src"], o["assign_row"], None, o["imbalance"], ws)
+    assert moe.get_status(ws) == 0
+    for n, t in o.items():
+        assert torch.equal(t, full[n]), n
+
+
+def test_gathering_gemm_reports_a_row_index_out_of_range():
+    """A row_src entry past T*k is read as token 0 and raises MOE_DEV_BOUNDS (checked in the kernel)."""
+    torch = _torch()
+    wl = moe_synth.workload("tiny")
+    shape = _shape(wl)
+    idx, _, _ = oracle.route(moe_synth.host_logits(wl), wl.k)
+    ref = oracle.dispatch(idx, wl.E, wl.R)
+    row_src = ref["row_src"].copy()
+    row_src[5] = shape.A + 1000
+    ws = moe.new_workspace(shape)
+    moe.moe_expert_gate_up_gather(shape, _bf16_dev(moe_synth.host_x(wl)), torch.from_numpy(row_src).cuda(),
+                                  torch.from_numpy(ref["expert_offsets"]).cuda(), _bf16_dev(moe_synth.host_w13(wl)),
+                                  None, ws)
+    assert moe.get_status(ws) == moe.MOE_DEV_BOUNDS
