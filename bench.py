@@ -258,7 +258,8 @@ def run_gpu(args, wl, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    moe.set_gemm_policy({"auto": moe.GEMM_AUTO, "single": moe.GEMM_SINGLE, "pair": moe.GEMM_PAIR}[args.gemm_policy])
+    moe.set_gemm_policy({"auto": moe.GEMM_AUTO, "single": moe.GEMM_SINGLE, "pair": moe.GEMM_PAIR,
+                         "split": moe.GEMM_SPLIT}[args.gemm_policy])
     wl_r = wl.with_(seed=replica_seed(wl.seed, rank))
     cap = moe.capacity_for(args.capacity_factor, wl.T, wl.k, wl.E) if args.capacity_factor else 0
     shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, n_shared=wl.n_shared, capacity=cap)
@@ -489,8 +490,9 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--gemm-policy", default="auto", choices=["auto", "single", "pair"],
-                    help="grouped-GEMM tiles: per-GEMM choice (auto), single-CTA 128-row, or CTA-pair 256x256")
+    ap.add_argument("--gemm-policy", default="auto", choices=["auto", "single", "pair", "split"],
+                    help="grouped-GEMM tiles: chosen from the shape (auto), single-CTA 128-row, CTA-pair 256x256, "
+                         "or split (pairs for whole 256-row blocks, single CTAs for short last blocks)")
     ap.add_argument("--capacity-factor", type=float, default=None,
                     help="per-expert capacity ceil(C*T*k/E); excess assignments are dropped (default: none)")
     ap.add_argument("--regime-sweep", action="store_true",

@@ -26,7 +26,7 @@ ABI_FUNCTIONS = (
     "moe_expert_gate_up", "moe_expert_down", "moe_dispatch_static", "moe_set_gemm_policy",
     "moe_set_test_stall", "moe_expert_gate_up_gather",
 )
-GEMM_AUTO, GEMM_SINGLE, GEMM_PAIR = 0, 1, 2
+GEMM_AUTO, GEMM_SINGLE, GEMM_PAIR, GEMM_SPLIT = 0, 1, 2, 3
 
 
 class MoEError(RuntimeError):
@@ -191,7 +191,8 @@ def set_test_stall(enable: bool) -> int:
 
 
 def set_gemm_policy(policy: int) -> int:
-    """GEMM_AUTO (per-GEMM choice), GEMM_SINGLE (128-row tiles) or GEMM_PAIR (CTA-pair 256x256 tiles)."""
+    """GEMM_AUTO (chosen from the shape), GEMM_SINGLE (128-row tiles), GEMM_PAIR (CTA-pair 256x256 tiles)
+    or GEMM_SPLIT (CTA pairs for whole 256-row blocks, single CTAs for last blocks of <= 128 rows)."""
     old = load().moe_set_gemm_policy(policy)
     if old < 0:
         raise ValueError(f"unknown GEMM policy {policy}")

@@ -77,6 +77,7 @@ struct FfnParams {
   uint32_t* status;
   uint64_t timeout_ns;
   int stall_first_stage; /* test hook: arm the first stage of each CTA's first tile but never load it */
+  int part;              /* rows of each group this launch covers: kPartAll, kPartPair or kPartTail */
   const int32_t* row_src;   /* GEMM1 gathering A from x: row_src of dispatch (null: A is x_perm) */
   const uint16_t* gather_x; /* x [T, d] rows to gather from */
   int k;                    /* experts per token (token of assignment a = a / k) */
@@ -90,6 +91,28 @@ struct Tile {
   int b_row;       /* first B row (TMA coordinate); GEMM1: the gate rows */
   int64_t out_row; /* first output row */
 };
+
+/* Which rows of a group one launch covers. kPartAll: every row, in TM-row tiles.
+ * The split schedule runs a group in two launches so that its last partial block
+ * is not padded to 256 rows: kPartPair takes the 256-row CTA-pair tiles, including
+ * a last one with more than 128 real rows; kPartTail takes a last block of 1..128
+ * rows as one 128-row single-CTA tile. */
+constexpr int kPartAll = 0, kPartPair = 1, kPartTail = 2;
+
+/* m-tiles (TM rows, counted from the group's first row) of a group of `rows`
+ * rows that a launch covers: [first, first + count). */
+template <int TM>
+__device__ __forceinline__ int part_tiles(int rows, int part, int* first) {
+  const int rem = rows & 255;
+  const bool short_tail = rem > 0 && rem <= 128;
+  *first = 0;
+  if (part == kPartPair) return short_tail ? rows >> 8 : (rows + 255) >> 8;
+  if (part == kPartTail) {
+    *first = (rows - rem) / TM;
+    return short_tail ? 1 : 0;
+  }
+  return (rows + TM - 1) / TM;
+}
 
 /* Shared-memory schedule, built by one warp: s_off = expert_offsets,
  * s_mpref[g] = m-tiles (TM rows) of groups < g, s_hpref[g] = 256-row blocks of h
@@ -113,7 +136,8 @@ __device__ __forceinline__ bool build_schedule(const FfnParams& p, int32_t* s_of
     } else if (g < G) {
       rows = (int)p.T;
     }
-    int im = (rows + TM - 1) / TM, ih = (rows + kHPad - 1) / kHPad;
+    int first_m;
+    int im = part_tiles<TM>(rows, p.part, &first_m), ih = (rows + kHPad - 1) / kHPad;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int ym = __shfl_up_sync(0xFFFFFFFFu, im, o);
@@ -156,10 +180,12 @@ __device__ __forceinline__ Tile decode_tile(int64_t L, const FfnParams& p, const
   t.g = lo;
   const int mt = s_mpref[lo + 1] - s_mpref[lo];
   const int local = (int)(L - (int64_t)s_mpref[lo] * p.n_tiles_n);
-  t.n = local / mt;
-  t.m = local - t.n * mt;
   const bool shared = lo >= p.E;
   const int rows = shared ? (int)p.T : s_off[lo + 1] - s_off[lo];
+  int first_m;
+  part_tiles<TM>(rows, p.part, &first_m);
+  t.n = local / mt;
+  t.m = first_m + (local - t.n * mt);
   t.valid = min(TM, rows - t.m * TM);
   const int hrow = s_hpref[lo] * kHPad + t.m * TM;
   if (MODE == 0) {
@@ -960,6 +986,12 @@ cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   return e;
 }
 
+/* Split schedule (CTA-pair tiles for whole 256-row blocks, single-CTA tiles for
+ * last blocks of <= 128 rows) on request only: its tail launch streams the weights
+ * of every expert with a short last block from DRAM a second time, which cost more
+ * than the padding it saves on every workload measured. */
+bool split_tiles(int pol) { return pol == kGemmSplit; }
+
 FfnParams base_params(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const int32_t* expert_offsets) {
   FfnParams p;
   p.expert_offsets = expert_offsets;
@@ -972,6 +1004,7 @@ FfnParams base_params(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, cons
   p.status = reinterpret_cast<uint32_t*>(ws + L.status);
   p.timeout_ns = wait_timeout_ns();
   p.stall_first_stage = test_stall() ? 1 : 0;
+  p.part = kPartAll;
   p.row_src = nullptr;
   p.gather_x = nullptr;
   p.k = s.k;
@@ -988,7 +1021,9 @@ cudaError_t launch_gate_up(const moe_shape_t& s, const WsLayout& L, uint8_t* ws,
   const bool gather = x_perm == nullptr; /* A rows gathered from x through row_src */
   /* 128-row single-CTA tiles pad small experts less and measured faster for this GEMM's
    * short K; CTA-pair tiles only on request (and never when gathering) */
-  const bool pair = !gather && gemm_policy() == kGemmPair;
+  const int pol = gather ? kGemmSingle : gemm_policy();
+  const bool split = split_tiles(pol);
+  const bool pair = split || pol == kGemmPair;
   CUtensorMap a0, a1, b0, b1;
   /* A = x_perm [A, d] (routed; rows of x gathered by the producer warp instead when x_perm is
    * null) / x [T, d] (shared);
@@ -1013,8 +1048,10 @@ cudaError_t launch_gate_up(const moe_shape_t& s, const WsLayout& L, uint8_t* ws,
   p.gather_x = gather ? x : nullptr;
   if (pair) {
     bool launched = false;
+    p.part = split ? kPartPair : kPartAll;
     const cudaError_t e = launch_pair<0>(a0, a1, b0, b1, o0, o0, p, stream, &launched);
-    if (e != cudaSuccess || launched) return e;
+    if (e != cudaSuccess || (launched && !split)) return e;
+    p.part = launched ? kPartTail : kPartAll;
   }
   return gather ? launch_single<0, 256, true>(a0, a1, b0, b1, o0, o0, p, stream)
                 : launch_single<0, 256>(a0, a1, b0, b1, o0, o0, p, stream);
@@ -1026,9 +1063,11 @@ cudaError_t launch_down(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, co
   if (s.T == 0) return cudaSuccess;
   const bool sh = s.n_shared != 0;
   const bool bn256 = (s.d % 256) == 0;
-  /* CTA-pair tiles when every expert averages >= 1024 rows (little 256-row padding) */
-  const bool pair = bn256 && (gemm_policy() == kGemmPair ||
-                              (gemm_policy() == kGemmAuto && L.A >= (int64_t)1024 * s.E));
+  /* CTA-pair tiles (256 output columns per tile) when every expert averages >= 1024
+   * rows, so that 256-row padding stays small */
+  const int pol = bn256 ? gemm_policy() : kGemmSingle;
+  const bool split = split_tiles(pol);
+  const bool pair = split || pol == kGemmPair || (pol == kGemmAuto && L.A >= (int64_t)1024 * s.E);
   const uint32_t bn = bn256 ? 256 : 128;
   const uint32_t b_box = pair ? 128 : bn;
   CUtensorMap a0, b0, b1;
@@ -1048,8 +1087,10 @@ cudaError_t launch_down(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, co
   p.ld_out = s.d;
   if (pair) {
     bool launched = false;
+    p.part = split ? kPartPair : kPartAll;
     const cudaError_t e = launch_pair<1>(a0, a0, b0, b1, o0, o1, p, stream, &launched);
-    if (e != cudaSuccess || launched) return e;
+    if (e != cudaSuccess || (launched && !split)) return e;
+    p.part = launched ? kPartTail : kPartAll;
     if (!make_map(&b0, w2, (uint64_t)s.E * s.d, s.f, bn)) return cudaErrorInvalidValue;
     if (!make_map(&b1, sh ? w2s : w2, sh ? (uint64_t)s.d : (uint64_t)s.E * s.d, s.f, bn))
       return cudaErrorInvalidValue;

@@ -296,7 +296,7 @@ const char* moe_status_string(moe_status_t status) {
 const char* moe_last_cuda_error(void) { return g_last_cuda_error; }
 
 int moe_set_gemm_policy(int policy) {
-  if (policy != kGemmAuto && policy != kGemmSingle && policy != kGemmPair) return -1;
+  if (policy != kGemmAuto && policy != kGemmSingle && policy != kGemmPair && policy != kGemmSplit) return -1;
   return g_gemm_policy.exchange(policy, std::memory_order_relaxed);
 }
 

@@ -18,6 +18,7 @@ constexpr int kHPadRows = 256;        /* h rows of each expert group are padded 
 constexpr int kGemmAuto = 0;          /* grouped GEMM: tile shape chosen per GEMM from the shape */
 constexpr int kGemmSingle = 1;        /* grouped GEMM: single-CTA 128-row tiles only */
 constexpr int kGemmPair = 2;          /* grouped GEMM: CTA-pair 256-row tiles wherever they apply */
+constexpr int kGemmSplit = 3;         /* grouped GEMM: CTA pairs for 256-row blocks, single CTAs for short tails */
 constexpr int kChunkAssign = 2048;    /* assignments per dispatch histogram chunk */
 constexpr uint64_t kDefaultWaitNs = 2000000000ull; /* bounded-wait limit of the GEMM pipeline */
 constexpr size_t kTicketOffset = 64; /* uint32 in the workspace header: dispatch's last-chunk ticket */
@@ -58,7 +59,7 @@ int num_sms();
 
 uint64_t wait_timeout_ns();
 
-/* Tile-shape policy of the grouped GEMM (kGemmAuto, kGemmSingle or kGemmPair). */
+/* Tile-shape policy of the grouped GEMM (kGemmAuto, kGemmSingle, kGemmPair or kGemmSplit). */
 int gemm_policy();
 
 /* Test hook: grouped-GEMM producers leave their first stage unloaded (see moe_set_test_stall). */

@@ -258,12 +258,20 @@ const char* moe_last_cuda_error(void);
 uint64_t moe_set_wait_timeout_ns(uint64_t ns);
 
 /* Diagnostic knob: tile shape of the grouped GEMM for launches made after the
- * call, process-wide. 0 (default) = chosen per GEMM from the shape: 128-row
- * single-CTA tiles, except 256 x 256 tiles computed by a cluster of two CTAs on
- * neighbouring SMs (cta_group::2) for the down GEMM when d % 256 == 0 and the
- * experts average at least 1024 rows; 1 = 128-row single-CTA tiles only; 2 =
- * CTA-pair tiles wherever they apply. Results are the same up to fp32 summation
- * order. Returns the previous value, or -1 for an unknown policy (unchanged). */
+ * call, process-wide. Two tile shapes exist: 128 x 256 tiles of one CTA, and
+ * 256 x 256 tiles computed by a cluster of two CTAs on neighbouring SMs
+ * (cta_group::2; the down GEMM needs d % 256 == 0 for them).
+ *   0 (default) = single-CTA tiles, except CTA-pair tiles for the down GEMM
+ *       when the routed experts average at least 1024 rows (T*k >= 1024*E);
+ *   1 = single-CTA tiles only;
+ *   2 = CTA-pair tiles wherever they apply (every group padded to 256 rows);
+ *   3 = split: each group's whole 256-row blocks, and a last block of more than
+ *       128 rows, as CTA-pair tiles; a last block of 1..128 rows as one
+ *       single-CTA tile in a second launch (padding as with single tiles, but
+ *       the second launch reads those experts' weights again: slower on the
+ *       workloads measured).
+ * Results are the same up to fp32 summation order. Returns the previous value,
+ * or -1 for an unknown policy (unchanged). */
 int moe_set_gemm_policy(int policy);
 
 /* Test hook for the bounded-wait path: while enabled (non-zero), every CTA of

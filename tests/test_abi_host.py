@@ -104,7 +104,8 @@ def test_status_strings_and_timeout_knob():
     assert lib.moe_set_gemm_policy(1) == 0
     assert lib.moe_set_gemm_policy(7) == -1
     assert lib.moe_set_gemm_policy(2) == 1
-    assert lib.moe_set_gemm_policy(0) == 2
+    assert lib.moe_set_gemm_policy(3) == 2
+    assert lib.moe_set_gemm_policy(0) == 3
     assert lib.moe_set_test_stall(1) == 0
     assert lib.moe_set_test_stall(0) == 1
 

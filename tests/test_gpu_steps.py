@@ -279,8 +279,8 @@ def _ffn_case(wl, idx=None):
         close(f64(bits(ys)), ys_ref, "y_shared")
 
 
-@pytest.fixture(params=[moe.GEMM_AUTO, moe.GEMM_SINGLE, moe.GEMM_PAIR], ids=["auto_tiles", "single_tiles",
-                                                                           "pair_tiles"])
+@pytest.fixture(params=[moe.GEMM_AUTO, moe.GEMM_SINGLE, moe.GEMM_PAIR, moe.GEMM_SPLIT],
+                ids=["auto_tiles", "single_tiles", "pair_tiles", "split_tiles"])
 def gemm_policy(request):
     old = moe.set_gemm_policy(request.param)
     yield request.param
@@ -312,9 +312,11 @@ def test_expert_ffn_with_empty_and_full_experts(gemm_policy):
     _ffn_case(wl, idx)
 
 
-@pytest.mark.parametrize("rows", [1, 15, 16, 17, 31, 32, 33, 63, 96, 127, 128, 129, 240, 255, 256, 257])
+@pytest.mark.parametrize("rows", [1, 15, 16, 17, 31, 32, 33, 63, 96, 127, 128, 129, 240, 255, 256, 257,
+                                  383, 384, 385, 512, 513, 700])
 def test_expert_ffn_tail_sizes(rows, gemm_policy):
-    """Ragged ends of every size class around the 32-row store blocks and the 128/256-row tiles."""
+    """Ragged ends of every size class around the 32-row store blocks and the 128/256-row tiles
+    (and, for the split schedule, last blocks just under, at and over 128 rows after whole 256-row blocks)."""
     wl = moe_synth.Workload("tail", T=rows + 40, d=256, E=3, k=1, f=256, R=1, n_shared=1)
     idx = np.full((wl.T, 1), 2, np.int32)
     idx[:rows, 0] = 0          # expert 0: `rows` rows, expert 1 empty, expert 2: 40 rows
