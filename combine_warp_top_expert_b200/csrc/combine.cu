@@ -1,9 +1,9 @@
 /*
  * combine.cu -- un-permute and top-k gate-weighted sum.
  *
- * Page "Expert Parallelism" (learning-materials IX.05) §4 COMBINE: "Send the
- * results back to the originating GPUs, in the original order. Weighted-sum the
- * k expert outputs per token." One warp per (token, column slice): the k row
+ * Page "Expert Parallelism" (learning-materials IX.05) §4 COMBINE: expert
+ * outputs go back to where their tokens came from, in the original token order,
+ * and each token's k outputs are summed with its gate weights. One warp per (token, column slice): the k row
  * indices and gates are loaded by lanes 0..k-1 and broadcast by shuffle; each
  * lane then streams 16-byte vectors of the k expert rows (+ the shared-expert
  * row), accumulates in fp32 in j order and stores one bf16 vector. Slices keep

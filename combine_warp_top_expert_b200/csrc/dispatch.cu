@@ -1,10 +1,10 @@
 /*
  * dispatch.cu -- per-expert histogram, exclusive scan and stable permute.
  *
- * Page "Expert Parallelism" (learning-materials IX.05) §4 DISPATCH: "Sort
- * tokens by destination expert (and therefore by destination GPU)", "Count how
- * many tokens go to each GPU", "Each GPU now has a contiguous set of tokens for
- * each of ITS experts"; §5: the load of the busiest GPU against the ideal.
+ * Page "Expert Parallelism" (learning-materials IX.05) §4 DISPATCH: tokens are
+ * ordered by the expert they go to (which orders them by GPU too), the tokens per
+ * GPU are counted, and afterwards every GPU holds one contiguous run of tokens
+ * per expert it owns; §5: the load of the busiest GPU against the ideal.
  *
  * Assignment a = t*k + j goes to row offsets[e] + (number of earlier
  * assignments to e): a stable counting sort, bit-exact and deterministic (no

@@ -2,10 +2,10 @@
  * expert_ffn.cu -- the experts' SwiGLU FFN as two persistent grouped GEMMs on
  * the 5th-generation tensor cores (tcgen05.mma, TMEM accumulators, TMA loads).
  *
- * Page "Expert Parallelism" (learning-materials IX.05) §4 COMPUTE: "Grouped
- * GEMM: each expert processes its tokens ... many different-shaped GEMMs in one
- * launch"; §8: "A naive per-expert loop is far slower than a proper grouped
- * GEMM". The page "UltraEP ..." (thelatestinai.com/papers/2606.04101, the
+ * Page "Expert Parallelism" (learning-materials IX.05) §4 COMPUTE: every expert
+ * multiplies its own tokens, and the differently sized per-expert GEMMs run as
+ * one grouped launch; §8: looping over the experts one by one is much slower
+ * than a grouped GEMM. The page "UltraEP ..." (thelatestinai.com/papers/2606.04101, the
  * makespan-aware dispatcher abstract) notes that grouped GEMM rounds each
  * expert's tokens up to 128-row M tiles: that is the tile height here, and the
  * padding rows are masked, never counted as work.

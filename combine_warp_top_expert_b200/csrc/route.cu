@@ -2,8 +2,8 @@
  * route.cu -- router top-k and gates.
  *
  * Page "Expert Parallelism" (learning-materials IX.05) §1: each token is routed
- * to k of the E experts; §4: "Router output: for each token, which expert(s) it
- * needs". One warp per token: lane l holds the logits of experts l, l+32, ...
+ * to k of the E experts; §4: the router's output names, per token, the experts
+ * it goes to. One warp per token: lane l holds the logits of experts l, l+32, ...
  * (coalesced 128-byte loads), k rounds of a warp-shuffle arg-max select the
  * experts in descending logit order with ties to the lower index, and the gates
  * are the softmax over the k selected logits.

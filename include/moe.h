@@ -90,7 +90,7 @@ moe_status_t moe_get_status(const void* ws, size_t ws_bytes, uint32_t* bits, voi
 
 /* Router: top-k selection and gates.
  * Page "Expert Parallelism" §1 (each token is routed to k of E experts) and §4
- * ("Router output: for each token, which expert(s) it needs").
+ * (the router's output: the experts each token goes to).
  *   logits    [T, E] fp32 in
  *   topk_idx  [T, k] int32 out: the k experts with the largest logits, in
  *             descending logit order; equal logits go to the lower expert index
@@ -155,9 +155,9 @@ moe_status_t moe_dispatch_static(const moe_shape_t* shape, const moe_bf16_t* x, 
                                  float* imbalance, uint32_t* status, void* stream);
 
 /* Expert FFN: one grouped GEMM over all experts (tcgen05 tensor cores).
- * Page "Expert Parallelism" §4 COMPUTE ("each expert processes its tokens ...
- * many different-shaped GEMMs in one launch") and §1 (E expert FFNs); the FFN is
- * SwiGLU: y = W2_e (silu(W_gate,e x) * (W_up,e x)), silu(a) = a / (1 + e^-a).
+ * Page "Expert Parallelism" §4 COMPUTE (every expert multiplies its own tokens;
+ * the differently sized GEMMs run as one grouped launch) and §1 (E expert FFNs);
+ * the FFN is SwiGLU: y = W2_e (silu(W_gate,e x) * (W_up,e x)), silu(a) = a / (1 + e^-a).
  *   x_perm         [T*k, d] bf16 in (from moe_dispatch)
  *   expert_offsets [E+1]    int32 in (from moe_dispatch)
  *   w13            [E, 2f, d] bf16 in: rows [0, f) = W_gate, [f, 2f) = W_up (K = d contiguous)

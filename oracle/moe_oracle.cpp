@@ -48,13 +48,14 @@ double order_key(float l) { return std::isnan(l) ? -std::numeric_limits<double>:
 extern "C" {
 
 /*
- * Router top-k and gates. Page "Expert Parallelism" §1: "each token is routed to
- * k of them"; §4: "Router output: for each token, which expert(s) it needs".
+ * Router top-k and gates. Page "Expert Parallelism" §1: each token is routed to
+ * k of the E experts; §4: the router's output names, per token, the experts it
+ * goes to.
  *   Order the E experts of token t by (logit descending, index ascending): expert
  *   a comes before b iff l_a > l_b, or l_a == l_b and a < b (IEEE compare, so
  *   -0.0 == +0.0). topk_idx[t][j] is the j-th expert in that order.
- *   [reading] the page gives no gate formula, only "weighted-sum the k expert
- *   outputs": the gates are the softmax over the k selected logits,
+ *   [reading] the page gives no gate formula, only that combine weights the k
+ *   expert outputs: the gates are the softmax over the k selected logits,
  *   g_j = exp(l_j - l_0) / sum_i exp(l_i - l_0), in fp64, rounded to fp32;
  *   g_j = 1/k if l_0 = -inf.
  * Returns the number of NaN logits seen.
@@ -85,18 +86,19 @@ int64_t oracle_route(int64_t T, int32_t E, int32_t k, const float* logits, int32
 
 /*
  * Dispatch bookkeeping. Page "Expert Parallelism" §4 DISPATCH:
- *   1. "Sort tokens by destination expert (and therefore by destination GPU)"
- *   2. "Count how many tokens go to each GPU"
- *   4. "Each GPU now has a contiguous set of tokens for each of ITS experts"
+ *   step 1 orders the tokens by the expert they go to (and so by GPU),
+ *   step 2 counts the tokens per GPU,
+ *   step 4 leaves every GPU with one contiguous run of tokens per expert it owns
  * and §1 (experts placed on GPUs in contiguous blocks: GPU 0 holds 0-15, ...).
  *   Assignment a = t*k + j goes to expert e = topk_idx[a] (entries outside
  *   [0, E) are skipped, counted, and get assign_row = -1).
  *   Rows are handed out in assignment order: a takes row offsets[e] + (number of
- *   earlier assignments to e). [reading] the page says "sort" without an order
+ *   earlier assignments to e). [reading] the page asks for a sort without an order
  *   inside an expert; keeping assignment order is the plainest stable reading.
  *   Capacity, page §5 "Mitigations" 1 (capacity factor): when capacity > 0 an
  *   expert keeps only its first `capacity` assignments in that order; the rest
- *   are dropped (assign_row = -1: "skip the expert, pass through the residual").
+ *   are dropped (assign_row = -1: the dropped assignment skips its expert and
+ *   only the residual path carries the token).
  *   counts[e] = assignments kept by e; offsets = exclusive scan of counts,
  *   offsets[E] = total kept.
  *   Logical rank r owns experts [r*E/R, (r+1)*E/R): rank_counts[r] = sum of its
@@ -179,7 +181,7 @@ int64_t oracle_dispatch(int64_t T, int32_t E, int32_t k, int32_t R, const int32_
                                   assign_row, imbalance, nullptr);
 }
 
-/* Dispatch data movement, page §4 DISPATCH step 3 ("exchange the token data"):
+/* Dispatch data movement, page §4 DISPATCH step 3 (the token rows are exchanged):
  * x_perm[p] = x[row_src[p] / k] for every filled row p (bit copy). */
 void oracle_permute_rows(int64_t n_rows, int32_t k, int32_t d, const uint16_t* x, const int32_t* row_src,
                          uint16_t* x_perm) {
@@ -191,7 +193,7 @@ void oracle_permute_rows(int64_t n_rows, int32_t k, int32_t d, const uint16_t* x
 }
 
 /*
- * One expert's SwiGLU FFN on n rows. Page §1 ("each layer has E expert FFNs");
+ * One expert's SwiGLU FFN on n rows. Page §1 (a layer holds E expert FFNs);
  * [reading] the FFN is SwiGLU: with W_gate = w13[0:f], W_up = w13[f:2f],
  *   a = W_gate x, b = W_up x, h = silu(a) * b, silu(a) = a / (1 + e^-a), y = W2 h,
  * all in fp64 with no intermediate rounding.
@@ -230,7 +232,7 @@ void oracle_swiglu(int64_t n, int32_t d, int32_t f, const uint16_t* xrows, const
 }
 
 /*
- * Expert compute, page §4 COMPUTE ("each expert processes its tokens"): the rows
+ * Expert compute, page §4 COMPUTE (every expert multiplies its own tokens): the rows
  * [offsets[e], offsets[e+1]) of x_perm go through expert e's FFN, written to the
  * same rows of y_perm. [reading] a shared expert (n_shared = 1) applies its own
  * SwiGLU FFN to every token of x, into y_shared.
@@ -247,8 +249,8 @@ void oracle_expert_ffn(int64_t T, int32_t d, int32_t E, int32_t f, int32_t n_sha
 }
 
 /*
- * Combine, page §4 COMBINE: "Send the results back ... in the original order.
- * Weighted-sum the k expert outputs per token."
+ * Combine, page §4 COMBINE: expert outputs return in the original token order
+ * and each token's k outputs are summed with its gate weights.
  *   out[t] = sum_{j<k} gate[t][j] * y_perm[assign_row[t*k+j]] (+ y_shared[t]), fp64,
  *   j in increasing order; a skipped assignment (assign_row < 0) adds nothing.
  */
@@ -268,7 +270,7 @@ void oracle_combine(int64_t T, int32_t k, int32_t d, const double* y_perm, const
   }
 }
 
-/* The "naive per-token loop" of the page's hands-on exercise C (§10): no sort,
+/* The unsorted per-token loop of the page's hands-on exercise C (§10): no sort,
  * each token visits its k experts directly. Same result as dispatch -> FFN ->
  * combine; used as an independent cross-check of the sorted path. */
 void oracle_naive_token_loop(int64_t T, int32_t d, int32_t E, int32_t k, int32_t f, int32_t n_shared,

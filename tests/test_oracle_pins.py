@@ -121,7 +121,7 @@ def test_worked_imbalance_example_section5():
     assert d8["imbalance"][0] == np.float32(140 / 64) == np.float32(2.1875)
     assert d8["imbalance"][1] == np.float32(2.1875)
     assert round(float(d8["imbalance"][0]), 1) == 2.2            # the page prints "2.2x"
-    assert round(100.0 / float(d8["imbalance"][0])) == 46        # "effective utilization = 46%"
+    assert round(100.0 / float(d8["imbalance"][0])) == 46        # the page's 46% effective utilization
     # two logical ranks, experts {0..3} and {4..7}: 375 vs 137 against 256
     d2 = oracle.dispatch(idx, g["E"], 2)
     assert list(d2["rank_counts"]) == [375, 137]
