@@ -134,6 +134,7 @@ moe_status_t moe_get_status(const void* ws, size_t ws_bytes, uint32_t* bits, voi
 
 moe_status_t moe_route(const moe_shape_t* shape, const float* logits, int32_t* topk_idx, float* topk_gate, void* ws,
                        size_t ws_bytes, void* stream) {
+  const NvtxRange nvtx_range("moe_route");
   moe_status_t st = validate_shape(shape);
   if (st != MOE_OK) return st;
   if (shape->T > 0 && (!logits || !topk_idx || !topk_gate)) return MOE_ERR_INVALID_ARG;
@@ -148,6 +149,7 @@ moe_status_t moe_dispatch(const moe_shape_t* shape, const moe_bf16_t* x, const i
                           int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
                           int32_t* rank_offsets, int32_t* row_src, int32_t* assign_row, moe_bf16_t* x_perm,
                           float* imbalance, void* ws, size_t ws_bytes, void* stream) {
+  const NvtxRange nvtx_range("moe_dispatch");
   moe_status_t st = validate_shape(shape);
   if (st != MOE_OK) return st;
   if (!expert_counts || !expert_offsets || !rank_counts || !rank_offsets || !imbalance) return MOE_ERR_INVALID_ARG;
@@ -165,6 +167,7 @@ moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_bf16_t* x_perm, 
                             const moe_bf16_t* w13, const moe_bf16_t* w2, const moe_bf16_t* x,
                             const moe_bf16_t* w13s, const moe_bf16_t* w2s, moe_bf16_t* y_perm,
                             moe_bf16_t* y_shared, void* ws, size_t ws_bytes, void* stream) {
+  const NvtxRange nvtx_range("moe_expert_ffn");
   moe_status_t st = validate_shape(shape);
   if (st != MOE_OK) return st;
   if (!expert_offsets || !w13 || !w2) return MOE_ERR_INVALID_ARG;
@@ -188,6 +191,7 @@ moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_bf16_t* x_perm, 
 moe_status_t moe_expert_gate_up(const moe_shape_t* shape, const moe_bf16_t* x_perm, const int32_t* expert_offsets,
                                 const moe_bf16_t* w13, const moe_bf16_t* x, const moe_bf16_t* w13s, void* ws,
                                 size_t ws_bytes, void* stream) {
+  const NvtxRange nvtx_range("moe_expert_gate_up");
   moe_status_t st = validate_shape(shape);
   if (st != MOE_OK) return st;
   if (!expert_offsets || !w13 || !aligned(w13, 16)) return MOE_ERR_INVALID_ARG;
@@ -203,6 +207,7 @@ moe_status_t moe_expert_gate_up(const moe_shape_t* shape, const moe_bf16_t* x_pe
 moe_status_t moe_expert_gate_up_gather(const moe_shape_t* shape, const moe_bf16_t* x, const int32_t* row_src,
                                        const int32_t* expert_offsets, const moe_bf16_t* w13, const moe_bf16_t* w13s,
                                        void* ws, size_t ws_bytes, void* stream) {
+  const NvtxRange nvtx_range("moe_expert_gate_up_gather");
   moe_status_t st = validate_shape(shape);
   if (st != MOE_OK) return st;
   if (!expert_offsets || !w13 || !aligned(w13, 16)) return MOE_ERR_INVALID_ARG;
@@ -218,6 +223,7 @@ moe_status_t moe_expert_gate_up_gather(const moe_shape_t* shape, const moe_bf16_
 moe_status_t moe_expert_down(const moe_shape_t* shape, const int32_t* expert_offsets, const moe_bf16_t* w2,
                              const moe_bf16_t* w2s, moe_bf16_t* y_perm, moe_bf16_t* y_shared, void* ws,
                              size_t ws_bytes, void* stream) {
+  const NvtxRange nvtx_range("moe_expert_down");
   moe_status_t st = validate_shape(shape);
   if (st != MOE_OK) return st;
   if (!expert_offsets || !w2 || !aligned(w2, 16)) return MOE_ERR_INVALID_ARG;
@@ -233,6 +239,7 @@ moe_status_t moe_expert_down(const moe_shape_t* shape, const int32_t* expert_off
 moe_status_t moe_combine(const moe_shape_t* shape, const moe_bf16_t* y_perm, const int32_t* assign_row,
                          const float* topk_gate, const moe_bf16_t* y_shared, moe_bf16_t* out, void* ws,
                          size_t ws_bytes, void* stream) {
+  const NvtxRange nvtx_range("moe_combine");
   moe_status_t st = validate_shape(shape);
   if (st != MOE_OK) return st;
   if (shape->T > 0 && (!y_perm || !assign_row || !topk_gate || !out)) return MOE_ERR_INVALID_ARG;
@@ -247,6 +254,7 @@ moe_status_t moe_combine(const moe_shape_t* shape, const moe_bf16_t* y_perm, con
 
 moe_status_t moe_layer(const moe_shape_t* shape, const moe_layer_buffers_t* b, void* ws, size_t ws_bytes,
                        void* stream) {
+  const NvtxRange nvtx_range("moe_layer");
   moe_status_t st = validate_shape(shape);
   if (st != MOE_OK) return st;
   if (!b) return MOE_ERR_INVALID_ARG;
