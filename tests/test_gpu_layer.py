@@ -119,11 +119,21 @@ def test_layer_full_size_sampled_parity(name, n_tokens):
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("policy", [moe.GEMM_SINGLE, moe.GEMM_PAIR], ids=["single_tiles", "pair_tiles"])
+@pytest.mark.parametrize("policy", [moe.GEMM_SINGLE, moe.GEMM_PAIR, moe.GEMM_SPLIT],
+                         ids=["single_tiles", "pair_tiles", "split_tiles"])
 def test_layer_mixtral_sampled_parity_other_tiles(policy):
     old = moe.set_gemm_policy(policy)
     try:
         test_layer_full_size_sampled_parity("mixtral_prefill", 4)
+    finally:
+        moe.set_gemm_policy(old)
+
+
+def test_layer_skewed_prefill_sampled_parity_split_tiles():
+    """Split tiles on the skewed prefill: cold experts end in short tails, hot ones and the shared expert don't."""
+    old = moe.set_gemm_policy(moe.GEMM_SPLIT)
+    try:
+        test_layer_full_size_sampled_parity("dsv3_skewed_prefill", 3)
     finally:
         moe.set_gemm_policy(old)
 
