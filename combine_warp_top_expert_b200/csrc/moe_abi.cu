@@ -9,9 +9,21 @@
 #include <cstdlib>
 #include <cstring>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "moe_internal.h"
 
 namespace moe {
+
+/* NVTX range around one ABI call on the host, so that Nsight timelines show which
+ * entry point issued which kernels (header-only NVTX: a no-op unless a tool is
+ * attached). */
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 namespace {
 

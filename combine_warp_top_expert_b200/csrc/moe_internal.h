@@ -8,8 +8,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
-#include "moe.h"
-#include <nvtx3/nvToolsExt.h> /* include/ is on the include path */
+#include "moe.h" /* include/ is on the include path */
 
 namespace moe {
 
@@ -56,16 +55,6 @@ moe_status_t validate_shape(const moe_shape_t* s);
 moe_status_t cuda_fail(cudaError_t e);
 
 /* Device SM count of the current device (cached). */
-/* NVTX range around one ABI call on the host, so that Nsight timelines show which
- * entry point issued which kernels (header-only NVTX: a no-op unless a tool is
- * attached). */
-struct NvtxRange {
-  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
-  ~NvtxRange() { nvtxRangePop(); }
-  NvtxRange(const NvtxRange&) = delete;
-  NvtxRange& operator=(const NvtxRange&) = delete;
-};
-
 int num_sms();
 
 uint64_t wait_timeout_ns();
