@@ -144,16 +144,27 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_count_kernel(
   const int64_t rem = A - a0;
   const int n = (int)(rem < chunk_assign ? rem : chunk_assign);
   const int per_warp = (n + kHistWarps - 1) / kHistWarps;
+  const int w_begin = warp * per_warp, w_end = min(n, (warp + 1) * per_warp);
+  /* all of this warp's expert ids in flight at once, before the histogram needs them */
+  constexpr int kIters = kChunkAssign / (kHistWarps * 32);
+  static_assert(kIters * kHistWarps * 32 == kChunkAssign, "a chunk is whole 32-wide steps of every warp");
+  int ev[kIters];
+#pragma unroll
+  for (int it = 0; it < kIters; ++it) {
+    const int i = w_begin + it * 32 + lane;
+    ev[it] = i < w_end ? __ldg(topk_idx + a0 + i) : -1;
+  }
   for (int i = threadIdx.x; i < kHistWarps * E; i += blockDim.x) hist[i] = 0;
   __syncthreads();
 
   bool bad = false;
-  const int w_begin = warp * per_warp, w_end = min(n, (warp + 1) * per_warp);
   int32_t* my_hist = hist + warp * E;
-  for (int base = w_begin; base < w_end; base += 32) {
-    const int i = base + lane;
+#pragma unroll
+  for (int it = 0; it < kIters; ++it) {
+    const int i = w_begin + it * 32 + lane;
+    if (w_begin + it * 32 >= w_end) break; /* warp-uniform */
     const bool valid = i < w_end;
-    int e = valid ? __ldg(topk_idx + a0 + i) : -1;
+    int e = valid ? ev[it] : -1;
     if (valid && (e < 0 || e >= E)) {
       bad = true;
       e = -1;
@@ -190,13 +201,18 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_count_kernel(
   }
   if (bad) raise_status(status, MOE_DEV_BOUNDS);
 
-  /* the last chunk to finish scans all chunk counts */
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) s_last = atomicAdd(ticket, 1u) == (uint32_t)(n_chunks - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
+  /* the last chunk to finish scans all chunk counts (a single chunk is its own last one:
+   * its counts are visible to the whole CTA after the barrier) */
+  if (n_chunks > 1) {
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(ticket, 1u) == (uint32_t)(n_chunks - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+  } else {
+    __syncthreads();
+  }
   scan_chunks(chunk_cnt, n_chunks, E, R, A, cap, expert_counts, expert_offsets, rank_counts, rank_offsets, imbalance,
               row_src);
   if (threadIdx.x == 0) *ticket = 0; /* ready for the next call on this workspace */
