@@ -137,8 +137,7 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_count_kernel(
     int32_t* row_src) {
   extern __shared__ int32_t sh[];
   __shared__ int s_last;
-  int32_t* hist = sh;                   /* [kHistWarps][E] */
-  int32_t* lrank = sh + kHistWarps * E; /* [chunk_assign] */
+  int32_t* hist = sh; /* [kHistWarps][E] */
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t a0 = (int64_t)blockIdx.x * chunk_assign;
   const int64_t rem = A - a0;
@@ -158,6 +157,9 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_count_kernel(
   __syncthreads();
 
   bool bad = false;
+  int rv[kIters]; /* rank of each of this lane's assignments among the warp's earlier ones */
+#pragma unroll
+  for (int it = 0; it < kIters; ++it) rv[it] = -1;
   int32_t* my_hist = hist + warp * E;
 #pragma unroll
   for (int it = 0; it < kIters; ++it) {
@@ -169,13 +171,14 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_count_kernel(
       bad = true;
       e = -1;
     }
+    ev[it] = e; /* -1 for lanes past the end and for skipped entries */
     const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
     int r = -1;
     if (e >= 0) r = my_hist[e] + __popc(peers & ((1u << lane) - 1u));
     __syncwarp();
     if (e >= 0 && lane == __ffs(peers) - 1) my_hist[e] += __popc(peers);
     __syncwarp();
-    if (valid) lrank[i] = r;
+    rv[it] = r;
   }
   __syncthreads();
   /* per expert: exclusive scan over the warps; chunk total to global */
@@ -190,14 +193,12 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_count_kernel(
     chunk_cnt[(int64_t)blockIdx.x * E + e] = run;
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const int r = lrank[i];
-    int out = -1;
-    if (r >= 0) {
-      const int w = i / per_warp;
-      out = hist[w * E + __ldg(topk_idx + a0 + i)] + r;
-    }
-    local_rank[a0 + i] = out;
+  /* each lane finishes its own assignments: rank inside the chunk = the warp's base
+   * for the expert (exclusive scan over the warps) + the rank inside the warp */
+#pragma unroll
+  for (int it = 0; it < kIters; ++it) {
+    const int i = w_begin + it * 32 + lane;
+    if (i < w_end) local_rank[a0 + i] = rv[it] >= 0 ? hist[warp * E + ev[it]] + rv[it] : -1;
   }
   if (bad) raise_status(status, MOE_DEV_BOUNDS);
 
@@ -239,6 +240,17 @@ __global__ void __launch_bounds__(256) dispatch_permute_kernel(
   for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < items; w += warps) {
     const int64_t t = w / slices;
     const int sl = (int)(w - t * slices);
+    const uint16_t* src = x_perm ? x + t * d : nullptr;
+    const int v_begin = sl * vps + lane, v_end = min(nv, (sl + 1) * vps);
+    /* the first row vectors need no index: their loads go out before the index chain */
+    uint4 buf[U];
+    if (x_perm != nullptr) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int v = v_begin + 32 * u;
+        if (v < v_end) buf[u] = ld_nc_v4(src + (int64_t)v * 8);
+      }
+    }
     int pos = -1;
     if (lane < k) {
       const int64_t a = t * k + lane;
@@ -260,14 +272,13 @@ __global__ void __launch_bounds__(256) dispatch_permute_kernel(
       const int p = __shfl_sync(0xFFFFFFFFu, pos, j);
       dst[j] = (j < k && p >= 0) ? (int64_t)p * d : -1;
     }
-    const uint16_t* src = x + t * d;
-    const int v_end = min(nv, (sl + 1) * vps);
-    for (int v0 = sl * vps + lane; v0 < v_end; v0 += 32 * U) {
-      uint4 buf[U];
+    for (int v0 = v_begin; v0 < v_end; v0 += 32 * U) {
+      if (v0 != v_begin) {
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int v = v0 + 32 * u;
-        if (v < v_end) buf[u] = ld_nc_v4(src + (int64_t)v * 8);
+        for (int u = 0; u < U; ++u) {
+          const int v = v0 + 32 * u;
+          if (v < v_end) buf[u] = ld_nc_v4(src + (int64_t)v * 8);
+        }
       }
 #pragma unroll
       for (int j = 0; j < kMaxK; ++j) {
@@ -317,7 +328,7 @@ cudaError_t launch_dispatch(const moe_shape_t& s, const WsLayout& L, uint8_t* ws
                                                           rank_offsets, imbalance);
     return cudaGetLastError();
   }
-  const size_t smem = (size_t)(kHistWarps * s.E + chunk_assign) * sizeof(int32_t);
+  const size_t smem = (size_t)kHistWarps * s.E * sizeof(int32_t);
   const int32_t cap = s.capacity > 0 ? s.capacity : 0x7FFFFFFF;
   dispatch_count_kernel<<<(unsigned)L.n_chunks, kHistThreads, smem, stream>>>(
       topk_idx, L.A, s.E, s.R, cap, chunk_assign, L.n_chunks, chunk, lrank, status, ticket, expert_counts,
