@@ -72,13 +72,39 @@ KERNEL_SOURCES = ("combine_warp_top_expert_b200/csrc/expert_ffn.cu", "combine_wa
                   "combine_warp_top_expert_b200/csrc/moe_internal.h")
 
 
+def strip_c_comments(text: str) -> str:
+    """C/C++ source without comments and with runs of white space collapsed (string and
+    character literals kept as they are), so that comment edits leave the hash unchanged."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_hash() -> str:
-    """Hash of the grouped-GEMM sources; a traffic figure is valid only for the source it was taken on."""
+    """Hash of the grouped-GEMM sources' code (comments and layout ignored); a traffic
+    figure is valid only for the code it was taken on."""
     import hashlib
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+            h.update(strip_c_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -25,13 +25,21 @@
  * owns TMEM and issues tcgen05.mma from one thread, warps 2-5 drain the
  * accumulator with tcgen05.ld and run the epilogue), two TMEM accumulators of
  * 256 fp32 columns so the epilogue of tile i overlaps the main loop of tile i+1:
- *   pair   (default) a cluster of 2 CTAs on neighbouring SMs computes a 256 x 256
- *          tile with cta_group::2 MMAs: each CTA stages its own 128 rows of A
- *          and 128 of the 256 rows of B (6-stage ring of 32 KB), so each SM moves
- *          32 KB of operands per 64-deep K step instead of 48 KB;
  *   single one CTA computes a 128 x 256 (GEMM1) or 128 x BN (GEMM2) tile with
- *          cta_group::1 MMAs (4-stage ring of 48 KB); used for GEMM2 when d is
- *          not a multiple of 256.
+ *          cta_group::1 MMAs (4-stage ring of 48 KB); the default for GEMM1 and
+ *          for every workload whose experts average fewer than 1024 rows;
+ *   pair   a cluster of 2 CTAs on neighbouring SMs computes a 256 x 256 tile
+ *          with cta_group::2 MMAs: each CTA stages its own 128 rows of A and 128
+ *          of the 256 rows of B (6-stage ring of 32 KB), so each SM moves 32 KB
+ *          of operands per 64-deep K step instead of 48 KB; faster per flop but
+ *          pads every group to 256 rows, so the default only for GEMM2 when
+ *          d % 256 == 0 and the experts average at least 1024 rows.
+ * moe_set_gemm_policy forces either shape, or a split that runs each group's
+ * whole 256-row blocks as pairs and a last block of <= 128 rows in a second,
+ * single-CTA launch (FfnParams::part selects the rows a launch covers).
+ * GEMM1 can also gather its A rows straight from x through row_src instead of
+ * reading x_perm (the GATHER instantiation: a warp of cp.async copies instead of
+ * one TMA tile per stage).
  * GEMM1's B tile stacks 128 gate rows over the matching 128 up rows, so one
  * N=256 MMA yields both halves of the SwiGLU for 128 output columns and the
  * epilogue combines them before anything leaves the SM.
