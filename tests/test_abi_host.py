@@ -120,3 +120,11 @@ def test_gathering_gemm_rejects_inputs_past_32_bit_row_offsets():
     b.x_perm = None
     b.w13s = b.w2s = b.y_shared = None
     assert lib.moe_layer(ctypes.byref(big), ctypes.byref(b), FAKE, 1 << 62, None) == moe.MOE_ERR_UNSUPPORTED
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No silent fallback: without the CUDA library every entry point raises."""
+    monkeypatch.setattr(moe, "_lib", None)
+    monkeypatch.setattr(moe, "LIB_PATH", str(tmp_path / "absent" / "libmoe_b200.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        moe.load(build_if_missing=False)
