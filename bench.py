@@ -396,7 +396,7 @@ def run_gpu(args, wl, rank, world, local_rank):
         "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded generator; weights random-init, no checkpoints)",
         "config": {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "f": wl.f, "R": wl.R,
-                   "n_shared": wl.n_shared, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "n_shared": wl.n_shared, "seed": wl.seed, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "flushed between steps (512 MiB write, outside the step's events)",
                    "gemm_tiles": args.gemm_policy,
                    "x_perm": "not materialised (rows gathered in the gate/up GEMM)" if args.gather else "materialised",
@@ -412,7 +412,8 @@ def run_gpu(args, wl, rank, world, local_rank):
                      "unit": "TFLOP/s" if d["bound"] == "tensor" else "GB/s",
                      "frac": d["achieved"] / (peaks["bf16"] if d["bound"] == "tensor" else peaks["hbm"]),
                      "peak_kind": f"{peaks['source']} burst",
-                     "traffic": recorded_traffic(wl.name, f"moe_expert_{dom}") if args.tokens is None else None},
+                     "traffic": recorded_traffic(wl.name, f"moe_expert_{dom}")
+                     if args.tokens is None and args.seed is None else None},
         "clocks": clocks.summary(),
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(x_h.numel() * 2 + lg_h.numel() * 4),
                 "d2h_bytes_per_step": int(outs_h[0].numel() * 2),
@@ -527,6 +528,9 @@ def main():
     ap.add_argument("--regime-f", type=int, default=2048)
     ap.add_argument("--gather", action="store_true",
                     help="no x_perm: dispatch writes indices only and the gate/up GEMM gathers rows of x itself")
+    ap.add_argument("--seed", type=int, default=None,
+                    help="seed of the synthetic inputs (default: the workload's; the router bias is calibrated "
+                         "on the default seed)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the workload's batch size T (smaller cases for profiling)")
     args = ap.parse_args()
@@ -540,6 +544,8 @@ def main():
     wl = moe_synth.workload(args.config)
     if args.tokens is not None:
         wl = wl.with_(T=args.tokens)
+    if args.seed is not None:
+        wl = wl.with_(seed=args.seed)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
