@@ -52,3 +52,37 @@ def test_pipeline_wait_timeout_is_reported_and_context_survives(policy):
         moe.set_gemm_policy(old_policy)
     y_ref, _ = oracle.expert_ffn(xp_np, ref["expert_offsets"], moe_synth.host_w13(wl), moe_synth.host_w2(wl))
     close(f64(bits(y)), y_ref, "y_perm after timeout")
+
+
+def test_gathering_gemm_wait_timeout_is_reported_and_context_survives():
+    """The bounded-wait path of the GEMM1 variant whose producer warp gathers rows of x."""
+    import torch
+    wl = moe_synth.workload("tiny")
+    shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R)
+    dv = moe_synth.device_inputs(wl)
+    idx, _, _ = oracle.route(moe_synth.host_logits(wl), wl.k)
+    ref = oracle.dispatch(idx, wl.E, wl.R)
+    row_src = torch.from_numpy(ref["row_src"]).cuda()
+    offs = torch.from_numpy(ref["expert_offsets"]).cuda()
+    y = torch.zeros((shape.A, wl.d), dtype=torch.bfloat16, device="cuda")
+    ws = moe.new_workspace(shape)
+
+    def run():
+        moe.moe_expert_gate_up_gather(shape, dv["x"], row_src, offs, dv["w13"], None, ws)
+        moe.moe_expert_down(shape, offs, dv["w2"], None, y, None, ws)
+
+    moe.set_wait_timeout_ns(50_000_000)
+    moe.set_test_stall(True)
+    try:
+        run()
+        status = moe.get_status(ws)
+    finally:
+        moe.set_test_stall(False)
+        moe.set_wait_timeout_ns(0)
+    assert status & moe.MOE_DEV_TIMEOUT
+    moe.clear_status(ws)
+    run()
+    assert moe.get_status(ws) == 0
+    xp_np = oracle.permute_rows(moe_synth.host_x(wl), ref["row_src"], wl.k)
+    y_ref, _ = oracle.expert_ffn(xp_np, ref["expert_offsets"], moe_synth.host_w13(wl), moe_synth.host_w2(wl))
+    close(f64(bits(y)), y_ref, "y_perm after a timeout in the gathering GEMM")
