@@ -342,3 +342,65 @@ def test_capacity_layer_equals_naive_loop_without_dropped_assignments():
     idx.reshape(-1)[res["assign_row"] < 0] = -1          # a dropped assignment adds nothing
     naive = oracle.naive_token_loop(x, idx, res["topk_gate"], w13, w2)
     assert np.max(np.abs(res["out"] - naive)) <= 1e-12 * np.max(np.abs(naive))
+
+
+# ---------------------------------------------------------------------------
+# dispatch with capacity and ranks: randomised brute force (hypothesis)
+# ---------------------------------------------------------------------------
+
+def _brute_dispatch(flat, E, R, cap):
+    """Stable sort by expert keeping each expert's first `cap` assignments (cap 0: all)."""
+    A = len(flat)
+    kept = [[] for _ in range(E)]
+    for a in range(A):
+        e = int(flat[a])
+        if cap == 0 or len(kept[e]) < cap:
+            kept[e].append(a)
+    row_src = [a for e in range(E) for a in kept[e]]
+    assign_row = [-1] * A
+    for p, a in enumerate(row_src):
+        assign_row[a] = p
+    counts = [len(kept[e]) for e in range(E)]
+    per = E // R
+    rank_counts = [sum(counts[r * per:(r + 1) * per]) for r in range(R)]
+    return row_src, assign_row, counts, rank_counts
+
+
+def test_dispatch_matches_brute_force_on_random_shapes_with_capacity():
+    from hypothesis import given, settings, strategies as st
+
+    @st.composite
+    def case(draw):
+        E = draw(st.integers(1, 24))
+        k = draw(st.integers(1, min(E, 8)))
+        divisors = [r for r in range(1, E + 1) if E % r == 0]
+        R = draw(st.sampled_from(divisors))
+        T = draw(st.integers(0, 60))
+        seed = draw(st.integers(0, 2**31 - 1))
+        cap = draw(st.integers(0, max(1, T * k)))
+        return T, E, k, R, cap, seed
+
+    @settings(max_examples=80, deadline=None)
+    @given(case())
+    def check(c):
+        T, E, k, R, cap, seed = c
+        rng = np.random.default_rng(seed)
+        idx = np.array([rng.permutation(E)[:k] for _ in range(T)], np.int32).reshape(T, k)
+        d = oracle.dispatch(idx, E, R, capacity=cap)
+        flat = idx.reshape(-1)
+        row_src, assign_row, counts, rank_counts = _brute_dispatch(flat, E, R, cap)
+        total = len(row_src)
+        assert list(d["expert_counts"]) == counts
+        assert list(d["expert_offsets"]) == [sum(counts[:e]) for e in range(E + 1)]
+        assert list(d["rank_counts"]) == rank_counts
+        assert list(d["rank_offsets"]) == [sum(rank_counts[:r]) for r in range(R + 1)]
+        assert list(d["row_src"][:total]) == row_src and np.all(d["row_src"][total:] == -1)
+        assert list(d["assign_row"]) == assign_row
+        assert d["dropped"] == T * k - total
+        if total:
+            assert d["imbalance"][0] == np.float32(max(rank_counts) * R / total)
+            assert d["imbalance"][1] == np.float32(max(counts) * E / total)
+        else:
+            assert list(d["imbalance"]) == [1.0, 1.0]
+
+    check()
