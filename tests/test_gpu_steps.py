@@ -410,3 +410,33 @@ def test_gathering_gemm_reports_a_row_index_out_of_range():
                                   torch.from_numpy(ref["expert_offsets"]).cuda(), _bf16_dev(moe_synth.host_w13(wl)),
                                   None, ws)
     assert moe.get_status(ws) == moe.MOE_DEV_BOUNDS
+
+
+def _random_dispatch_cases(n=24, seed=2024):
+    rng = np.random.default_rng(seed)
+    cases = []
+    for _ in range(n):
+        E = int(rng.integers(1, 257))
+        k = int(rng.integers(1, min(E, 8) + 1))
+        divisors = [r for r in range(1, min(E, 16) + 1) if E % r == 0]
+        R = int(rng.choice(divisors))
+        T = int(rng.integers(0, 5000))
+        cap = int(rng.integers(1, max(2, T * k // E * 2))) if rng.random() < 0.4 and T else 0
+        cases.append((T, E, k, R, cap, int(rng.integers(0, 2**31 - 1))))
+    return cases
+
+
+@pytest.mark.parametrize("T,E,k,R,cap,seed", _random_dispatch_cases())
+def test_dispatch_random_shapes_bit_exact(T, E, k, R, cap, seed):
+    """Seeded random shapes (chunk boundaries, many or few experts, capacity drops) against the oracle."""
+    torch = _torch()
+    rng = np.random.default_rng(seed)
+    idx = np.array([rng.permutation(E)[:k] for _ in range(T)], np.int32).reshape(T, k)
+    shape = moe.Shape(T=T, d=128, E=E, k=k, f=128, R=R, capacity=cap)
+    x_np = rng.integers(0, 1 << 16, size=(T, 128), dtype=np.uint64).astype(np.uint16)
+    x_dev = torch.from_numpy(x_np.view(np.int16)).cuda().view(torch.bfloat16) if T else \
+        torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
+    o = _gpu_dispatch(shape, x_dev, idx)
+    assert o["status"] == 0
+    ref = oracle.dispatch(idx, E, R, capacity=cap)
+    _check_dispatch(o, ref, x_np, k)
