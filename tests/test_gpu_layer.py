@@ -261,3 +261,39 @@ def test_layer_gathering_rows_with_capacity_matches_oracle():
     for n in ("expert_counts", "expert_offsets", "row_src", "assign_row"):
         assert np.array_equal(np_i32(outs[n]), res[n]), n
     close(f64(bits(outs["out"])), res["out"], "out with capacity, gathered rows")
+
+
+def _random_layer_cases(n=12, seed=77):
+    rng = np.random.default_rng(seed)
+    cases = []
+    for i in range(n):
+        E = int(rng.integers(1, 33))
+        k = int(rng.integers(1, min(E, 8) + 1))
+        R = int(rng.choice([r for r in range(1, E + 1) if E % r == 0]))
+        T = int(rng.integers(1, 400))
+        d = int(rng.choice([128, 256, 384, 512]))
+        f = int(rng.choice([128, 256, 384]))
+        n_shared = int(rng.integers(0, 2))
+        cf = float(rng.choice([0.0, 0.0, 1.0, 1.5]))
+        wl = moe_synth.Workload(f"rnd{i}", T=T, d=d, E=E, k=k, f=f, R=R, n_shared=n_shared, bias_kind="zipf",
+                                zipf_s=float(rng.uniform(0.0, 1.5)), seed=i + 1)
+        cases.append((wl, cf))
+    return cases
+
+
+@pytest.mark.parametrize("wl,cf", _random_layer_cases(), ids=[c[0].name for c in _random_layer_cases()])
+def test_layer_random_shapes_match_oracle(wl, cf):
+    """Seeded random shapes through the whole layer (default tile policy) against the oracle."""
+    cap = moe.capacity_for(cf, wl.T, wl.k, wl.E) if cf else 0
+    shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, n_shared=wl.n_shared, capacity=cap)
+    dv = moe_synth.device_inputs(wl)
+    layer = moe.MoELayer(shape, dv["w13"], dv["w2"], dv.get("w13s"), dv.get("w2s"))
+    outs = layer(dv["logits"], dv["x"])
+    assert moe.get_status(layer.ws) == 0
+    res = oracle.layer(moe_synth.host_x(wl), moe_synth.host_logits(wl), moe_synth.host_w13(wl),
+                       moe_synth.host_w2(wl), wl.k, wl.R, moe_synth.host_w13s(wl) if wl.n_shared else None,
+                       moe_synth.host_w2s(wl) if wl.n_shared else None, capacity=cap)
+    assert np.array_equal(np_i32(outs["topk_idx"]), res["topk_idx"])
+    for n in ("expert_counts", "expert_offsets", "rank_counts", "rank_offsets", "row_src", "assign_row"):
+        assert np.array_equal(np_i32(outs[n]), res[n]), n
+    close(f64(bits(outs["out"])), res["out"], f"out {wl.name}")
