@@ -2,10 +2,14 @@
 copy of the oracle's source (on the CPU), rebuilds it, and checks that the pin
 written for that function fails on the mutant while it passes on the oracle.
 
-Mutants: reversed tie-break, wrong sign in the gate exponent, unstable
-(reversed) row order, imbalance denominator with the wrong count, swapped gate
-and up halves, wrong silu sign, transposed down-projection index, gate dropped
-in combine, capacity keeping the last instead of the first assignments.
+Mutants: reversed tie-break, wrong sign in the gate exponent, softmax over all
+E logits instead of the k selected, unstable (reversed) row order, imbalance
+denominator with the wrong count, experts dealt to ranks round-robin instead of
+in contiguous blocks, rank offsets not scaled by experts per rank, counts that
+still include dropped assignments, token index taken as a % k in the row copy,
+swapped gate and up halves, wrong silu sign, transposed down-projection index,
+gate dropped in combine, shared-expert output dropped in combine, capacity
+keeping the last instead of the first assignments.
 """
 import importlib.util
 import math
@@ -108,6 +112,45 @@ def pin_capacity_first(o):
     return bool(np.array_equal(d["assign_row"] >= 0, keep))
 
 
+def pin_rank_offsets(o):
+    """rank r's rows start after every row of the experts below r*E/R (numpy count)."""
+    E, R = 12, 4
+    idx = np.random.default_rng(11).integers(0, E, size=(90, 3)).astype(np.int32)
+    d = o.dispatch(idx, E, R)
+    n = np.bincount(idx.reshape(-1), minlength=E)
+    want = [int(n[:r * E // R].sum()) for r in range(R + 1)]
+    return list(d["rank_offsets"]) == want and list(d["rank_counts"]) == list(np.diff(want))
+
+
+def pin_permute_token(o):
+    """x_perm row p is the row of token a // k, a = row_src[p] (numpy indexing)."""
+    k = 3
+    idx = np.random.default_rng(12).integers(0, 5, size=(17, k)).astype(np.int32)
+    d = o.dispatch(idx, 5, 1)
+    x = np.random.default_rng(13).integers(0, 1 << 16, size=(17, 24)).astype(np.uint16)
+    xp = o.permute_rows(x, d["row_src"], k)
+    return bool(np.array_equal(xp, x[d["row_src"] // k]))
+
+
+def pin_combine_shared(o):
+    """zero expert outputs leave exactly the shared expert's output (weight one)."""
+    idx = np.random.default_rng(14).integers(0, 4, size=(10, 2)).astype(np.int32)
+    d = o.dispatch(idx, 4, 1)
+    gate = np.random.default_rng(15).uniform(0.1, 0.9, size=(10, 2)).astype(np.float32)
+    ys = np.random.default_rng(16).normal(size=(10, 8))
+    out = o.combine(np.zeros((20, 8)), d["assign_row"], gate, ys)
+    return bool(np.array_equal(out, ys))
+
+
+def pin_capacity_counts(o):
+    """with capacity c, expert e keeps min(n_e, c) rows and the offsets scan those."""
+    idx = np.random.default_rng(17).integers(0, 5, size=(80, 2)).astype(np.int32)
+    d = o.dispatch(idx, 5, 1, capacity=12)
+    kept = np.minimum(np.bincount(idx.reshape(-1), minlength=5), 12)
+    return (list(d["expert_counts"]) == list(kept)
+            and list(d["expert_offsets"]) == [0] + list(np.cumsum(kept)))
+
+
 MUTANTS = [
     ("reversed tie-break", "return ka > kb || (ka == kb && a < b);", "return ka > kb || (ka == kb && a > b);",
      pin_topk),
@@ -129,6 +172,19 @@ MUTANTS = [
      "for (int32_t c = 0; c < d; ++c) o[c] += y_perm[p * d + c];", pin_identity_experts),
     ("capacity keeps the last", "if (capacity > 0 && seen[e] >= capacity) {",
      "if (capacity > 0 && seen[e] < capacity) {", pin_capacity_first),
+    ("softmax over all experts", "for (int32_t j = 0; j < k; ++j) s += std::exp(order_key(l[order[j]]) - l0);",
+     "for (int32_t j = 0; j < E; ++j) s += std::exp(order_key(l[order[j]]) - l0);", pin_gate_logistic),
+    ("ranks own interleaved experts",
+     "for (int32_t e = r * per_rank; e < (r + 1) * per_rank; ++e) c += counts[e];",
+     "for (int32_t e = r; e < E; e += R) c += counts[e];", pin_worked_example),
+    ("rank offsets unscaled", "rank_offsets[r] = offsets[r * per_rank];", "rank_offsets[r] = offsets[r];",
+     pin_rank_offsets),
+    ("dropped assignments counted", "if (keep[a]) counts[topk_idx[a]] += 1;", "counts[topk_idx[a]] += 1;",
+     pin_capacity_counts),
+    ("token index by modulo", "const int64_t t = row_src[p] / k;", "const int64_t t = row_src[p] % k;",
+     pin_permute_token),
+    ("shared output dropped", "for (int32_t c = 0; c < d; ++c) o[c] += y_shared[t * d + c];",
+     "for (int32_t c = 0; c < d; ++c) o[c] += 0.0 * y_shared[t * d + c];", pin_combine_shared),
 ]
 
 
