@@ -4,9 +4,11 @@
  * Page "Expert Parallelism" (learning-materials IX.05) §1: each token is routed
  * to k of the E experts; §4: the router's output names, per token, the experts
  * it goes to. One warp per token: lane l holds the logits of experts l, l+32, ...
- * (coalesced 128-byte loads), k rounds of a warp-shuffle arg-max select the
- * experts in descending logit order with ties to the lower index, and the gates
- * are the softmax over the k selected logits.
+ * (coalesced 128-byte loads) as order-preserving 32-bit keys; each of k rounds
+ * takes the warp's largest key with one redux.sync max and the lowest expert
+ * holding it with one redux.sync min, so the experts come out in descending
+ * logit order with ties to the lower index. The gates are the softmax over the
+ * k selected logits.
  *
  * Bytes per token: E*4 read + k*8 written; bandwidth-bound at large T.
  */
@@ -18,10 +20,21 @@ namespace moe {
 
 namespace {
 
-/* (v, e) ranks before (bv, be): larger logit, or equal logit and lower index.
- * IEEE compare, so -0.0 and +0.0 tie. */
-__device__ __forceinline__ bool ranks_before(float v, int e, float bv, int be) {
-  return v > bv || (v == bv && e < be);
+/* Unsigned key of a (non-NaN) logit: key(a) > key(b) iff a > b, and key(a) ==
+ * key(b) iff a == b under IEEE compare (-0.0 is folded onto +0.0 first). Sign-
+ * magnitude floats become monotone unsigned integers by flipping every bit of a
+ * negative value and only the sign bit of a positive one. The smallest key a
+ * logit can take is key(-inf) = 0x007FFFFF, so 0 marks a slot that cannot be
+ * selected (already taken, or past the last expert). */
+__device__ __forceinline__ uint32_t logit_key(float l) {
+  uint32_t u = __float_as_uint(l);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+/* The logit of a key (inverse of logit_key; -0.0 comes back as +0.0). */
+__device__ __forceinline__ float key_logit(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
 template <int NV>
@@ -33,51 +46,42 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
   bool saw_nan = false;
   for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
     const float* row = logits + t * E;
-    float v[NV];
-    uint32_t taken = 0;
+    uint32_t key[NV];
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       const int e = lane + 32 * i;
+      key[i] = 0u; /* not an expert: never selectable */
       if (e < E) {
         float l = __ldg(row + e);
         if (isnan(l)) {
           saw_nan = true;
           l = -INFINITY;
         }
-        v[i] = l;
-      } else {
-        v[i] = -INFINITY;
-        taken |= 1u << i; /* not an expert: never selectable */
+        key[i] = logit_key(l);
       }
     }
-    float my_v = -INFINITY;
-    int my_e = 0;
+    uint32_t my_key = 0u;
+    uint32_t my_e = 0u;
     for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
-      int be = 0x7FFFFFFF;
+      uint32_t m = key[0];
 #pragma unroll
-      for (int i = 0; i < NV; ++i) {
-        const int e = lane + 32 * i;
-        if (!((taken >> i) & 1u) && ranks_before(v[i], e, bv, be)) {
-          bv = v[i];
-          be = e;
-        }
-      }
+      for (int i = 1; i < NV; ++i) m = max(m, key[i]);
+      const uint32_t best = __reduce_max_sync(0xFFFFFFFFu, m);
+      /* this lane's lowest expert holding the best key (slots ascend in expert) */
+      uint32_t cand = 0xFFFFFFFFu;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
-        const int oe = __shfl_xor_sync(0xFFFFFFFFu, be, off);
-        if (ranks_before(ov, oe, bv, be)) {
-          bv = ov;
-          be = oe;
-        }
-      }
-      if (lane == (be & 31)) taken |= 1u << (be >> 5);
+      for (int i = NV - 1; i >= 0; --i)
+        if (key[i] == best) cand = (uint32_t)(lane + 32 * i);
+      const uint32_t be = __reduce_min_sync(0xFFFFFFFFu, cand);
+#pragma unroll
+      for (int i = 0; i < NV; ++i)
+        if ((uint32_t)(lane + 32 * i) == be) key[i] = 0u;
       if (lane == j) {
-        my_v = bv;
+        my_key = best;
         my_e = be;
       }
     }
+    const float my_v = key_logit(my_key); /* meaningful on lanes < k only */
     /* gates: softmax over the selected logits, relative to the largest */
     const float l0 = __shfl_sync(0xFFFFFFFFu, my_v, 0);
     float ex = 0.0f;
@@ -86,7 +90,7 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
     if (lane < k) {
-      topk_idx[t * k + lane] = my_e;
+      topk_idx[t * k + lane] = (int32_t)my_e;
       topk_gate[t * k + lane] = ex / sum;
     }
   }

@@ -111,6 +111,27 @@ def test_route_ties_signed_zeros_and_infinities(E, k):
     assert np.max(np.abs(gate.astype(np.float64) - rgate)) <= GATE_TOL
 
 
+@pytest.mark.parametrize("E,k", [(8, 2), (256, 8), (200, 5)])
+def test_route_positive_infinity_orders_first(E, k):
+    """+inf ranks above every finite logit, ties to the lower index among +inf; the gate
+    of a +inf expert is NaN (inf - inf) on both sides, so gates are compared where finite."""
+    rng = np.random.default_rng(E + k)
+    T = 300
+    lg = rng.normal(size=(T, E)).astype(np.float32)
+    lg[::3, E // 2] = np.inf
+    lg[1::3, [E - 1, 0]] = np.inf
+    lg[5, :] = np.inf
+    shape = moe.Shape(T=T, d=128, E=E, k=k, f=128, R=1)
+    idx, gate, status = _gpu_route(shape, lg)
+    ridx, rgate, nan = oracle.route(lg, k)
+    assert status == 0 and nan == 0
+    assert np.array_equal(idx, ridx)
+    g = gate.astype(np.float64)
+    assert np.array_equal(np.isnan(g), np.isnan(rgate))
+    fin = ~np.isnan(rgate)
+    assert np.max(np.abs(g[fin] - rgate[fin])) <= GATE_TOL
+
+
 def test_route_nan_is_ordered_last_and_flagged():
     lg = np.random.default_rng(0).normal(size=(64, 16)).astype(np.float32)
     lg[7, 3] = np.nan
