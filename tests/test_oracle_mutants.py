@@ -2,14 +2,15 @@
 copy of the oracle's source (on the CPU), rebuilds it, and checks that the pin
 written for that function fails on the mutant while it passes on the oracle.
 
-Mutants: reversed tie-break, wrong sign in the gate exponent, softmax over all
-E logits instead of the k selected, unstable (reversed) row order, imbalance
-denominator with the wrong count, experts dealt to ranks round-robin instead of
-in contiguous blocks, rank offsets not scaled by experts per rank, counts that
-still include dropped assignments, token index taken as a % k in the row copy,
-swapped gate and up halves, wrong silu sign, transposed down-projection index,
-gate dropped in combine, shared-expert output dropped in combine, capacity
-keeping the last instead of the first assignments.
+Mutants: reversed tie-break, NaN ordered first instead of as -inf, wrong sign
+in the gate exponent, softmax over all E logits instead of the k selected,
+unstable (reversed) row order, imbalance denominator with the wrong count,
+experts dealt to ranks round-robin instead of in contiguous blocks, rank
+offsets not scaled by experts per rank, counts that still include dropped
+assignments, token index taken as a % k in the row copy, swapped gate and up
+halves, wrong silu sign, transposed down-projection index, gate dropped in
+combine, shared-expert output dropped in combine, capacity keeping the last
+instead of the first assignments.
 """
 import importlib.util
 import math
@@ -50,6 +51,13 @@ def pin_topk(o):
     lg = rng.integers(-2, 3, size=(64, 5)).astype(np.float32)
     idx, _, _ = o.route(lg, 3)
     return all(list(idx[t]) == _brute_topk([float(v) for v in lg[t]], 3) for t in range(64))
+
+
+def pin_nan_last(o):
+    """NaN orders as -inf: after every number, tied with -inf by index; each NaN counted."""
+    lg = np.array([[np.nan, 1.0, 0.5, -3.0], [2.0, np.nan, np.nan, -np.inf]], np.float32)
+    idx, _, nan = o.route(lg, 4)
+    return list(idx[0]) == [1, 2, 3, 0] and list(idx[1]) == [0, 1, 2, 3] and nan == 3
 
 
 def pin_gate_logistic(o):
@@ -154,6 +162,8 @@ def pin_capacity_counts(o):
 MUTANTS = [
     ("reversed tie-break", "return ka > kb || (ka == kb && a < b);", "return ka > kb || (ka == kb && a > b);",
      pin_topk),
+    ("NaN orders first", "return std::isnan(l) ? -std::numeric_limits<double>::infinity() : (double)l;",
+     "return std::isnan(l) ? std::numeric_limits<double>::infinity() : (double)l;", pin_nan_last),
     ("gate exponent sign", "topk_gate[t * k + j] = (float)(std::exp(order_key(l[order[j]]) - l0) / s);",
      "topk_gate[t * k + j] = (float)(std::exp(l0 - order_key(l[order[j]])) / s);", pin_gate_logistic),
     ("unstable row order", "const int32_t p = offsets[e] + cursor[e]++;",

@@ -62,6 +62,38 @@ def test_topk_signed_zero_ties_go_to_lower_index():
         assert gate[0, 0] == np.float32(0.5) and gate[0, 1] == np.float32(0.5)
 
 
+def test_topk_matches_python_sort_on_arbitrary_floats():
+    """Any float32 logits, special values mixed in (signed zeros, infinities, NaN,
+    subnormals, the largest finite values): the selection equals Python's own sort by
+    (logit descending with NaN as -inf, index ascending), and the NaN count is exact."""
+    from hypothesis import given, settings, strategies as st
+
+    special = st.sampled_from([0.0, -0.0, float("inf"), float("-inf"), float("nan"), 1e-45, -1e-45,
+                               3.4028234663852886e38, -3.4028234663852886e38, 1.0, -1.0])
+    value = st.one_of(st.floats(width=32), special)
+
+    @st.composite
+    def case(draw):
+        E = draw(st.integers(1, 40))
+        k = draw(st.integers(1, min(E, 8)))
+        T = draw(st.integers(0, 5))
+        return k, np.array([[draw(value) for _ in range(E)] for _ in range(T)], np.float32).reshape(T, E)
+
+    @settings(max_examples=120, deadline=None)
+    @given(case())
+    def check(c):
+        k, lg = c
+        T, E = lg.shape
+        idx, _, nan = oracle.route(lg, k)
+        assert nan == int(np.isnan(lg).sum())
+        for t in range(T):
+            key = [float("-inf") if np.isnan(v) else float(v) for v in lg[t]]
+            want = sorted(range(E), key=lambda e: (-key[e], e))[:k]
+            assert list(idx[t]) == want, (lg[t], list(idx[t]), want)
+
+    check()
+
+
 def test_topk_nan_orders_as_minus_inf_and_is_counted():
     lg = np.array([[np.nan, 1.0, 0.5, -3.0]], np.float32)
     idx, _, nan = oracle.route(lg, 3)
