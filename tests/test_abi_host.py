@@ -70,6 +70,71 @@ def test_invalid_shapes_are_rejected_before_launch(shape, code):
     assert lib.moe_combine(s, *([FAKE] * 5), FAKE, 1 << 30, None) == code
 
 
+SHAPE_CHECKS = [
+    ("T<0", dict(T=-1), moe.MOE_ERR_INVALID_ARG),
+    ("d<1", dict(d=0), moe.MOE_ERR_INVALID_ARG),
+    ("f<1", dict(f=0), moe.MOE_ERR_INVALID_ARG),
+    ("E<1", dict(E=0), moe.MOE_ERR_INVALID_ARG),
+    ("R<1", dict(R=0), moe.MOE_ERR_INVALID_ARG),
+    ("capacity<0", dict(capacity=-1), moe.MOE_ERR_INVALID_ARG),
+    ("T*k>2^27", dict(T=(1 << 26) + 1), moe.MOE_ERR_UNSUPPORTED),
+    ("d>65536", dict(d=65536 + 128), moe.MOE_ERR_UNSUPPORTED),
+    ("f>65536", dict(f=65536 + 128), moe.MOE_ERR_UNSUPPORTED),
+]
+
+
+@pytest.mark.parametrize("kw,code", [c[1:] for c in SHAPE_CHECKS], ids=[c[0] for c in SHAPE_CHECKS])
+def test_every_shape_check_holds_at_every_entry_point(kw, code):
+    """Each shape rule rejects the shape at every entry point, and the workspace size is 0."""
+    lib = moe.load()
+    base = dict(T=8, d=512, E=8, k=2, f=1024, R=2)
+    base.update(kw)
+    s = ctypes.byref(moe.Shape(**base).c())
+    assert lib.moe_workspace_bytes(s) == 0
+    assert lib.moe_route(s, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == code
+    assert lib.moe_dispatch(s, *([FAKE] * 10), FAKE, 1 << 30, None) == code
+    assert lib.moe_dispatch_static(s, *([FAKE] * 10), None, None) == code
+    assert lib.moe_expert_ffn(s, *([FAKE] * 9), FAKE, 1 << 30, None) == code
+    assert lib.moe_expert_gate_up(s, *([FAKE] * 5), FAKE, 1 << 30, None) == code
+    assert lib.moe_expert_gate_up_gather(s, *([FAKE] * 5), FAKE, 1 << 30, None) == code
+    assert lib.moe_expert_down(s, *([FAKE] * 5), FAKE, 1 << 30, None) == code
+    assert lib.moe_combine(s, *([FAKE] * 5), FAKE, 1 << 30, None) == code
+    b = moe.moe_layer_buffers_t(*([FAKE] * len(moe.moe_layer_buffers_t._fields_)))
+    assert lib.moe_layer(s, ctypes.byref(b), FAKE, 1 << 30, None) == code
+
+
+def test_misaligned_operands_are_rejected_before_launch():
+    """Every bf16 operand must start on a 16-byte boundary (16-byte vector and TMA access)."""
+    lib = moe.load()
+    s = ctypes.byref(TINY.c())
+    bad, ws, inv = FAKE + 8, (FAKE, 1 << 30), moe.MOE_ERR_INVALID_ARG
+    # moe_dispatch: x_perm (x is covered above)
+    assert lib.moe_dispatch(s, FAKE, *([FAKE] * 7), bad, FAKE, *ws, None) == inv
+    # moe_expert_gate_up(x_perm, expert_offsets, w13, x, w13s)
+    assert lib.moe_expert_gate_up(s, bad, FAKE, FAKE, FAKE, None, *ws, None) == inv
+    assert lib.moe_expert_gate_up(s, FAKE, FAKE, bad, FAKE, None, *ws, None) == inv
+    # moe_expert_gate_up_gather(x, row_src, expert_offsets, w13, w13s)
+    assert lib.moe_expert_gate_up_gather(s, bad, FAKE, FAKE, FAKE, None, *ws, None) == inv
+    assert lib.moe_expert_gate_up_gather(s, FAKE, FAKE, FAKE, bad, None, *ws, None) == inv
+    # moe_expert_down(expert_offsets, w2, w2s, y_perm, y_shared)
+    assert lib.moe_expert_down(s, FAKE, bad, None, FAKE, None, *ws, None) == inv
+    assert lib.moe_expert_down(s, FAKE, FAKE, None, bad, None, *ws, None) == inv
+    # moe_expert_ffn(x_perm, expert_offsets, w13, w2, x, w13s, w2s, y_perm, y_shared)
+    for i in (0, 2, 3, 7):
+        p = [FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE, None]
+        p[i] = bad
+        assert lib.moe_expert_ffn(s, *p, *ws, None) == inv, i
+    # moe_combine(y_perm, assign_row, topk_gate, y_shared, out)
+    assert lib.moe_combine(s, bad, FAKE, FAKE, None, FAKE, *ws, None) == inv
+    assert lib.moe_combine(s, FAKE, FAKE, FAKE, bad, FAKE, *ws, None) == inv
+    assert lib.moe_combine(s, FAKE, FAKE, FAKE, None, bad, *ws, None) == inv
+    # moe_layer: each bf16 buffer in turn
+    for name in ("x", "w13", "w2", "w13s", "w2s", "x_perm", "y_perm", "y_shared", "out"):
+        b = moe.moe_layer_buffers_t(*([FAKE] * len(moe.moe_layer_buffers_t._fields_)))
+        setattr(b, name, bad)
+        assert lib.moe_layer(s, ctypes.byref(b), *ws, None) == inv, name
+
+
 def test_null_pointers_and_small_workspace_are_rejected():
     lib = moe.load()
     s = ctypes.byref(TINY.c())
