@@ -403,6 +403,7 @@ def run_gpu(args, wl, rank, world, local_rank):
                    "capacity_factor": args.capacity_factor, "capacity": cap,
                    "dropped_fraction": 1.0 - sum(counts) / float(wl.T * wl.k) if wl.T else 0.0,
                    "experts_active": work["_n_act"], "imbalance_rank_expert": imbalance,
+                   "expert_counts": counts,
                    "layer_roofline_frac": t_roof / (max_ms / args.steps / 1e3),
                    "per_step_ms": {n: round(v, 4) for n, v in kern_ms.items()},
                    "per_step_roofline": {n: {"bound": r["bound"], "frac": round(r["frac"], 4)} for n, r in roof.items()},
