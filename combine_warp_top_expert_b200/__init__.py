@@ -144,6 +144,17 @@ def _stream(stream) -> Optional[int]:
     return stream.cuda_stream
 
 
+def _ws(ws):
+    """(pointer, bytes) of a workspace: a contiguous uint8 CUDA tensor such as
+    new_workspace returns. A host tensor would hand a host address to the kernels,
+    so it is refused here."""
+    import torch
+    if ws is None:
+        raise ValueError("ws must be a CUDA uint8 tensor (see new_workspace)")
+    _dev(ws, torch.uint8, None, "ws")
+    return ws.data_ptr(), ws.numel()
+
+
 def _dev(t, dtype, shape, name):
     import torch
     if t is None:
@@ -172,12 +183,12 @@ def new_workspace(shape: Shape, device="cuda"):
 
 
 def clear_status(ws, stream=None):
-    _check("moe_clear_status", load().moe_clear_status(_ptr(ws), ws.numel(), _stream(stream)))
+    _check("moe_clear_status", load().moe_clear_status(*_ws(ws), _stream(stream)))
 
 
 def get_status(ws, stream=None) -> int:
     bits = ctypes.c_uint32(0)
-    _check("moe_get_status", load().moe_get_status(_ptr(ws), ws.numel(), ctypes.byref(bits), _stream(stream)))
+    _check("moe_get_status", load().moe_get_status(*_ws(ws), ctypes.byref(bits), _stream(stream)))
     return bits.value
 
 
@@ -205,7 +216,7 @@ def moe_route(shape: Shape, logits, topk_idx, topk_gate, ws, stream=None):
     _dev(topk_idx, torch.int32, (shape.T, shape.k), "topk_idx")
     _dev(topk_gate, torch.float32, (shape.T, shape.k), "topk_gate")
     _check("moe_route", load().moe_route(ctypes.byref(shape.c()), _ptr(logits), _ptr(topk_idx), _ptr(topk_gate),
-                                         _ptr(ws), ws.numel(), _stream(stream)))
+                                         *_ws(ws), _stream(stream)))
 
 
 def moe_dispatch(shape: Shape, x, topk_idx, expert_counts, expert_offsets, rank_counts, rank_offsets, row_src,
@@ -225,7 +236,7 @@ def moe_dispatch(shape: Shape, x, topk_idx, expert_counts, expert_offsets, rank_
     _check("moe_dispatch", load().moe_dispatch(
         ctypes.byref(shape.c()), _ptr(x), _ptr(topk_idx), _ptr(expert_counts), _ptr(expert_offsets),
         _ptr(rank_counts), _ptr(rank_offsets), _ptr(row_src), _ptr(assign_row), _ptr(x_perm), _ptr(imbalance),
-        _ptr(ws), ws.numel(), _stream(stream)))
+        *_ws(ws), _stream(stream)))
 
 
 def moe_expert_ffn(shape: Shape, x_perm, expert_offsets, w13, w2, x, w13s, w2s, y_perm, y_shared, ws, stream=None):
@@ -243,7 +254,7 @@ def moe_expert_ffn(shape: Shape, x_perm, expert_offsets, w13, w2, x, w13s, w2s, 
         _dev(y_shared, bf, (shape.T, shape.d), "y_shared")
     _check("moe_expert_ffn", load().moe_expert_ffn(
         ctypes.byref(shape.c()), _ptr(x_perm), _ptr(expert_offsets), _ptr(w13), _ptr(w2), _ptr(x), _ptr(w13s),
-        _ptr(w2s), _ptr(y_perm), _ptr(y_shared), _ptr(ws), ws.numel(), _stream(stream)))
+        _ptr(w2s), _ptr(y_perm), _ptr(y_shared), *_ws(ws), _stream(stream)))
 
 
 def moe_expert_gate_up(shape: Shape, x_perm, expert_offsets, w13, x, w13s, ws, stream=None):
@@ -257,8 +268,8 @@ def moe_expert_gate_up(shape: Shape, x_perm, expert_offsets, w13, x, w13s, ws, s
         _dev(x, bf, (shape.T, shape.d), "x")
         _dev(w13s, bf, (2 * shape.f, shape.d), "w13s")
     _check("moe_expert_gate_up", load().moe_expert_gate_up(
-        ctypes.byref(shape.c()), _ptr(x_perm), _ptr(expert_offsets), _ptr(w13), _ptr(x), _ptr(w13s), _ptr(ws),
-        ws.numel(), _stream(stream)))
+        ctypes.byref(shape.c()), _ptr(x_perm), _ptr(expert_offsets), _ptr(w13), _ptr(x), _ptr(w13s),
+        *_ws(ws), _stream(stream)))
 
 
 def moe_expert_gate_up_gather(shape: Shape, x, row_src, expert_offsets, w13, w13s, ws, stream=None):
@@ -272,8 +283,8 @@ def moe_expert_gate_up_gather(shape: Shape, x, row_src, expert_offsets, w13, w13
     if shape.n_shared:
         _dev(w13s, bf, (2 * shape.f, shape.d), "w13s")
     _check("moe_expert_gate_up_gather", load().moe_expert_gate_up_gather(
-        ctypes.byref(shape.c()), _ptr(x), _ptr(row_src), _ptr(expert_offsets), _ptr(w13), _ptr(w13s), _ptr(ws),
-        ws.numel(), _stream(stream)))
+        ctypes.byref(shape.c()), _ptr(x), _ptr(row_src), _ptr(expert_offsets), _ptr(w13), _ptr(w13s),
+        *_ws(ws), _stream(stream)))
 
 
 def moe_expert_down(shape: Shape, expert_offsets, w2, w2s, y_perm, y_shared, ws, stream=None):
@@ -287,8 +298,8 @@ def moe_expert_down(shape: Shape, expert_offsets, w2, w2s, y_perm, y_shared, ws,
         _dev(w2s, bf, (shape.d, shape.f), "w2s")
         _dev(y_shared, bf, (shape.T, shape.d), "y_shared")
     _check("moe_expert_down", load().moe_expert_down(
-        ctypes.byref(shape.c()), _ptr(expert_offsets), _ptr(w2), _ptr(w2s), _ptr(y_perm), _ptr(y_shared), _ptr(ws),
-        ws.numel(), _stream(stream)))
+        ctypes.byref(shape.c()), _ptr(expert_offsets), _ptr(w2), _ptr(w2s), _ptr(y_perm), _ptr(y_shared),
+        *_ws(ws), _stream(stream)))
 
 
 def moe_combine(shape: Shape, y_perm, assign_row, topk_gate, y_shared, out, ws, stream=None):
@@ -301,7 +312,7 @@ def moe_combine(shape: Shape, y_perm, assign_row, topk_gate, y_shared, out, ws, 
     _dev(out, bf, (shape.T, shape.d), "out")
     _check("moe_combine", load().moe_combine(
         ctypes.byref(shape.c()), _ptr(y_perm), _ptr(assign_row), _ptr(topk_gate), _ptr(y_shared), _ptr(out),
-        _ptr(ws), ws.numel(), _stream(stream)))
+        *_ws(ws), _stream(stream)))
 
 
 _LAYER_OUTPUTS = ("topk_idx", "topk_gate", "expert_counts", "expert_offsets", "rank_counts", "rank_offsets",
@@ -343,9 +354,12 @@ def moe_layer(shape: Shape, logits, x, w13, w2, w13s, w2s, outs: dict, ws, strea
     if shape.n_shared:
         _dev(w13s, bf, (2 * shape.f, shape.d), "w13s")
         _dev(w2s, bf, (shape.d, shape.f), "w2s")
+    for n in _LAYER_OUTPUTS:
+        if outs[n] is not None and not outs[n].is_cuda:
+            raise ValueError(f"outs[{n!r}] must be a CUDA tensor")
     b = moe_layer_buffers_t(_ptr(logits), _ptr(x), _ptr(w13), _ptr(w2), _ptr(w13s), _ptr(w2s),
                             *(_ptr(outs[n]) for n in _LAYER_OUTPUTS))
-    _check("moe_layer", load().moe_layer(ctypes.byref(shape.c()), ctypes.byref(b), _ptr(ws), ws.numel(),
+    _check("moe_layer", load().moe_layer(ctypes.byref(shape.c()), ctypes.byref(b), *_ws(ws),
                                          _stream(stream)))
     return outs
 

@@ -193,3 +193,21 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(moe, "LIB_PATH", str(tmp_path / "absent" / "libmoe_b200.so"))
     with pytest.raises(RuntimeError, match="not built"):
         moe.load(build_if_missing=False)
+
+
+def test_binding_refuses_host_buffers_before_the_abi():
+    """A host tensor where a device buffer belongs raises ValueError in Python, so no
+    host address ever reaches a kernel; a missing workspace is refused the same way."""
+    import torch
+    cpu_ws = torch.zeros(moe.workspace_bytes(TINY), dtype=torch.uint8)
+    for call in (lambda: moe.get_status(cpu_ws), lambda: moe.clear_status(cpu_ws),
+                 lambda: moe.moe_route(TINY, None, None, None, cpu_ws),
+                 lambda: moe.moe_combine(TINY, None, None, None, None, None, cpu_ws)):
+        with pytest.raises(ValueError, match="ws must be a CUDA tensor"):
+            call()
+    with pytest.raises(ValueError, match="ws must be a CUDA uint8 tensor"):
+        moe.moe_expert_down(TINY, None, None, None, None, None, None)
+    with pytest.raises(ValueError, match=r"outs\['topk_idx'\] must be a CUDA tensor"):
+        moe.moe_layer(TINY, None, None, None, None, None, None, moe.alloc_layer_outputs(TINY, device="cpu"), cpu_ws)
+    with pytest.raises(ValueError, match="logits must be a CUDA tensor"):
+        moe.moe_route(TINY, torch.zeros((TINY.T, TINY.E)), None, None, cpu_ws)
