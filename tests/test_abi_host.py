@@ -211,3 +211,21 @@ def test_binding_refuses_host_buffers_before_the_abi():
         moe.moe_layer(TINY, None, None, None, None, None, None, moe.alloc_layer_outputs(TINY, device="cpu"), cpu_ws)
     with pytest.raises(ValueError, match="logits must be a CUDA tensor"):
         moe.moe_route(TINY, torch.zeros((TINY.T, TINY.E)), None, None, cpu_ws)
+
+
+def test_capacity_for_is_the_exact_ceiling():
+    """capacity = ceil(C * T * k / E) in exact arithmetic: checked against integer ceiling
+    division for two-decimal factors C = n / 100, and on a factor whose binary value sits
+    just above a decimal (0.1 * 3 = 0.30000000000000004) where float arithmetic rounds up."""
+    from hypothesis import given, settings, strategies as st
+
+    assert moe.capacity_for(1.0, 4096, 2, 8) == 1024
+    assert moe.capacity_for(1.25, 4096, 2, 8) == 1280
+    assert moe.capacity_for(0.1 * 3, 10, 1, 3) == 1          # float: 1.0000000000000002 -> 2
+
+    @settings(max_examples=200, deadline=None)
+    @given(st.integers(1, 400), st.integers(0, 20000), st.integers(1, 8), st.integers(1, 256))
+    def check(n, T, k, E):
+        assert moe.capacity_for(n / 100, T, k, E) == -(-(n * T * k) // (100 * E))
+
+    check()
