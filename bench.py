@@ -7,9 +7,12 @@ are already resident in HBM (weights, x, logits), timed with CUDA events on the
 launching stream. L2 is flushed (a 512 MiB write) between steps, outside the
 step's events. Prints one JSON line (rank 0).
 
-N > 1 runs under torchrun: each rank runs an independent replica of the layer on
-its own batch (the path has no cross-GPU exchange on one node here; "replicas
-only"), value = all ranks' tokens / the max over ranks of the timed region.
+N > 1 runs one process per GPU: launched under torchrun (WORLD_SIZE set, which
+must equal --gpus), or, when started directly with --gpus N, bench.py re-launches
+itself under torch.distributed.run with N ranks on this node. Each rank runs an
+independent replica of the layer on its own batch (the path has no cross-GPU
+exchange on one node here; "replicas only"), value = all ranks' tokens / the max
+over ranks of the timed region.
 
 --impl reference times the CPU oracle (the plain fp64 definition of the layer)
 on the host cores, on a bounded sample of tokens of the same workload.
@@ -510,6 +513,35 @@ def run_regime_sweep(args):
         print(json.dumps(dict(regime_fit=fit)), flush=True)
 
 
+def free_port() -> int:
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as so:
+        so.bind(("127.0.0.1", 0))
+        return so.getsockname()[1]
+
+
+def relaunch_command(gpus: int, argv, port: int):
+    """The command that runs this benchmark as `gpus` ranks on this node (one process per GPU)."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+            "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+
+
+def rank_check(args, rank, world):
+    """--rank-check: join the process group (gloo, no GPU), agree on the slowest rank's
+    value, print one line per rank and leave; checks the multi-rank launch on any host."""
+    import datetime
+
+    import torch.distributed as dist
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    try:
+        mx = max_over_ranks(100.0 * (rank + 1), world)
+        print(json.dumps({"rank_check": {"rank": rank, "world": world, "gpus": args.gpus, "max_ms": mx,
+                                         "seed": replica_seed(0, rank)}}), flush=True)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -534,9 +566,20 @@ def main():
                          "on the default seed)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the workload's batch size T (smaller cases for profiling)")
+    ap.add_argument("--rank-check", action="store_true",
+                    help="start the ranks, join a gloo process group, print one line per rank and exit (no GPU)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.gpus < 1:
+        sys.exit(f"--gpus must be >= 1, got {args.gpus}")
+    world_env = os.environ.get("WORLD_SIZE")
+    if world_env is None and args.gpus > 1:
+        # one process per GPU: re-launch under torch.distributed.run with --gpus ranks
+        r = subprocess.run(relaunch_command(args.gpus, sys.argv[1:], free_port()))
+        sys.exit(r.returncode)
+    if world_env is not None and int(world_env) != args.gpus:
+        sys.exit(f"--gpus {args.gpus} does not match WORLD_SIZE={world_env}")
 
     if args.regime_sweep:
         run_regime_sweep(args)
@@ -551,6 +594,9 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
+    if args.rank_check:
+        rank_check(args, rank, world)
+        return
     if args.impl == "reference":
         run_reference(args, wl, rank, world)
         return

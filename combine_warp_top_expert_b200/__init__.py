@@ -24,7 +24,7 @@ ABI_FUNCTIONS = (
     "moe_workspace_bytes", "moe_clear_status", "moe_get_status", "moe_route", "moe_dispatch", "moe_expert_ffn",
     "moe_combine", "moe_layer", "moe_status_string", "moe_last_cuda_error", "moe_set_wait_timeout_ns",
     "moe_expert_gate_up", "moe_expert_down", "moe_dispatch_static", "moe_set_gemm_policy",
-    "moe_set_test_stall", "moe_expert_gate_up_gather",
+    "moe_set_test_stall", "moe_expert_gate_up_gather", "moe_capacity_for", "moe_dispatch_static_scratch",
 )
 GEMM_AUTO, GEMM_SINGLE, GEMM_PAIR, GEMM_SPLIT = 0, 1, 2, 3
 
@@ -72,6 +72,10 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     L.moe_dispatch.argtypes = [shp] + [vp] * 10 + [vp, sz, vp]
     L.moe_dispatch_static.restype = st
     L.moe_dispatch_static.argtypes = [shp] + [vp] * 11 + [vp]
+    L.moe_dispatch_static_scratch.restype = st
+    L.moe_dispatch_static_scratch.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_size_t)]
+    L.moe_capacity_for.restype = ctypes.c_int32
+    L.moe_capacity_for.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
     L.moe_expert_ffn.restype = st
     L.moe_expert_ffn.argtypes = [shp] + [vp] * 9 + [vp, sz, vp]
     L.moe_expert_gate_up.restype = st
@@ -127,10 +131,14 @@ class Shape:
 
 
 def capacity_for(C: float, T: int, k: int, E: int) -> int:
-    """Per-expert capacity of a capacity factor C: ceil(C * T * k / E) assignments."""
+    """Per-expert capacity of a capacity factor C, computed by moe_capacity_for in the
+    library (C is passed as an exact fraction with a denominator of at most 2^20)."""
     from fractions import Fraction
-    q = Fraction(C).limit_denominator(1 << 20) * T * k / E
-    return int(-(-q.numerator // q.denominator))
+    q = Fraction(C).limit_denominator(1 << 20)
+    c = load().moe_capacity_for(q.numerator, q.denominator, T, k, E)
+    if c < 0:
+        raise ValueError(f"no capacity for C={C}, T={T}, k={k}, E={E}")
+    return c
 
 
 def _ptr(t) -> Optional[int]:
@@ -155,18 +163,18 @@ def _ws(ws):
     return ws.data_ptr(), ws.numel()
 
 
-def _dev(t, dtype, shape, name):
-    import torch
+def _dev(t, dtype, shape, name, device: bool = True):
+    """dtype, contiguity and shape of a buffer, then (device=True) that it lives on a CUDA device."""
     if t is None:
         return
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
     if t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if device and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
 
 
 def workspace_bytes(shape: Shape) -> int:
@@ -319,6 +327,17 @@ _LAYER_OUTPUTS = ("topk_idx", "topk_gate", "expert_counts", "expert_offsets", "r
                   "row_src", "assign_row", "x_perm", "imbalance", "y_perm", "y_shared", "out")
 
 
+def _layer_output_specs(shape: Shape) -> dict:
+    """dtype and shape of every output buffer of moe_layer."""
+    import torch
+    i32, f32, bf = torch.int32, torch.float32, torch.bfloat16
+    T, k, E, R, d, A = shape.T, shape.k, shape.E, shape.R, shape.d, shape.A
+    return dict(topk_idx=(i32, (T, k)), topk_gate=(f32, (T, k)), expert_counts=(i32, (E,)),
+                expert_offsets=(i32, (E + 1,)), rank_counts=(i32, (R,)), rank_offsets=(i32, (R + 1,)),
+                row_src=(i32, (A,)), assign_row=(i32, (A,)), x_perm=(bf, (A, d)), imbalance=(f32, (2,)),
+                y_perm=(bf, (A, d)), y_shared=(bf, (T, d)), out=(bf, (T, d)))
+
+
 def alloc_layer_outputs(shape: Shape, device="cuda", x_perm: bool = True) -> dict:
     """Device buffers for every output of moe_layer (x_perm=False: the layer gathers
     rows of x inside the grouped GEMM and x_perm is not materialised)."""
@@ -354,11 +373,17 @@ def moe_layer(shape: Shape, logits, x, w13, w2, w13s, w2s, outs: dict, ws, strea
     if shape.n_shared:
         _dev(w13s, bf, (2 * shape.f, shape.d), "w13s")
         _dev(w2s, bf, (shape.d, shape.f), "w2s")
-    for n in _LAYER_OUTPUTS:
-        if outs[n] is not None and not outs[n].is_cuda:
-            raise ValueError(f"outs[{n!r}] must be a CUDA tensor")
+    specs = _layer_output_specs(shape)
+    for n, (dtype, shp) in specs.items():  # every buffer's layout first, then where it lives
+        if outs.get(n) is None:
+            if n == "x_perm" or (n == "y_shared" and not shape.n_shared):
+                continue  # x_perm None: rows gathered in GEMM1; no shared expert
+            raise ValueError(f"outs[{n!r}] is required")
+        _dev(outs[n], dtype, shp, f"outs[{n!r}]", device=False)
+    for n, (dtype, shp) in specs.items():
+        _dev(outs.get(n), dtype, shp, f"outs[{n!r}]")
     b = moe_layer_buffers_t(_ptr(logits), _ptr(x), _ptr(w13), _ptr(w2), _ptr(w13s), _ptr(w2s),
-                            *(_ptr(outs[n]) for n in _LAYER_OUTPUTS))
+                            *(_ptr(outs.get(n)) for n in _LAYER_OUTPUTS))
     _check("moe_layer", load().moe_layer(ctypes.byref(shape.c()), ctypes.byref(b), *_ws(ws),
                                          _stream(stream)))
     return outs

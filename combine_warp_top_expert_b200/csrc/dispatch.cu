@@ -232,8 +232,10 @@ __global__ void __launch_bounds__(256) dispatch_permute_kernel(
     const uint16_t* __restrict__ x, const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ chunk_base,
     const int32_t* __restrict__ local_rank, const int32_t* __restrict__ expert_offsets, int64_t T, int d, int E,
     int k, int32_t cap, int64_t tok_per_chunk, int slices, int vps, int32_t* __restrict__ row_src,
-    int32_t* __restrict__ assign_row, uint16_t* __restrict__ x_perm) {
+    int32_t* __restrict__ assign_row, uint16_t* __restrict__ x_perm, uint32_t* status) {
   const int lane = threadIdx.x & 31;
+  const int64_t A = T * k;
+  bool bad = false;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int nv = d >> 3; /* 16-byte vectors per row */
   const int64_t items = T * slices;
@@ -258,7 +260,14 @@ __global__ void __launch_bounds__(256) dispatch_permute_kernel(
       const int lr = __ldg(local_rank + a);
       if (e >= 0 && e < E && lr >= 0) {
         const int rank = __ldg(chunk_base + (t / tok_per_chunk) * E + e) + lr; /* among e's assignments */
-        if (rank < cap) pos = __ldg(expert_offsets + e) + rank;                /* else dropped */
+        if (rank < cap) {                                                      /* else dropped */
+          const int64_t q = (int64_t)__ldg(expert_offsets + e) + rank;
+          /* a row outside [0, A) can only come from inconsistent scratch: skip it, report it */
+          if (rank >= 0 && q >= 0 && q < A)
+            pos = (int)q;
+          else
+            bad = true;
+        }
       }
       if (sl == 0) {
         if (pos >= 0) row_src[pos] = (int32_t)a;
@@ -291,6 +300,7 @@ __global__ void __launch_bounds__(256) dispatch_permute_kernel(
       }
     }
   }
+  if (bad) raise_status(status, MOE_DEV_BOUNDS);
 }
 
 }  // namespace
@@ -342,7 +352,7 @@ cudaError_t launch_dispatch(const moe_shape_t& s, const WsLayout& L, uint8_t* ws
   }
   dispatch_permute_kernel<4><<<(unsigned)rs.blocks, 256, 0, stream>>>(
       x, topk_idx, chunk, lrank, expert_offsets, s.T, s.d, s.E, s.k, cap, L.tok_per_chunk, rs.slices, rs.vps,
-      row_src, assign_row, x_perm);
+      row_src, assign_row, x_perm, status);
   return cudaGetLastError();
 }
 

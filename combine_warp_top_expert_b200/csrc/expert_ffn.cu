@@ -921,16 +921,29 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uin
   return r == CUDA_SUCCESS;
 }
 
+/* The opt-in to more than 48 KB of dynamic shared memory is a property of the
+ * kernel on one device: set it once per device (and kernel instantiation) before
+ * the first launch there. A failed attempt is retried on the next launch. */
+constexpr int kMaxDevices = 64;
+
+template <typename Kernel>
+cudaError_t smem_opt_in(std::atomic<int> (&done)[kMaxDevices], Kernel kernel, size_t bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done[dev].store(1, std::memory_order_release);
+  return e;
+}
+
 template <int MODE, int BN, bool GATHER = false>
 cudaError_t launch_single(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0, const CUtensorMap& b1,
                           const CUtensorMap& o0, const CUtensorMap& o1, const FfnParams& p, cudaStream_t stream) {
   using C = SingleCfg<MODE, BN>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(ffn_gemm_single_kernel<MODE, BN, GATHER>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM_BYTES);
-  });
+  static std::atomic<int> attr_done[kMaxDevices];
+  const cudaError_t attr_err = smem_opt_in(attr_done, ffn_gemm_single_kernel<MODE, BN, GATHER>, C::SMEM_BYTES);
   if (attr_err != cudaSuccess) return attr_err;
   ffn_gemm_single_kernel<MODE, BN, GATHER>
       <<<num_sms(), kThreads, C::SMEM_BYTES, stream>>>(a0, a1, b0, b1, o0, o1, p);
@@ -967,12 +980,8 @@ cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
                         const CUtensorMap& o0, const CUtensorMap& o1, const FfnParams& p, cudaStream_t stream,
                         bool* launched) {
   *launched = false;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(ffn_gemm_pair_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)PairCfg::SMEM_BYTES);
-  });
+  static std::atomic<int> attr_done[kMaxDevices];
+  const cudaError_t attr_err = smem_opt_in(attr_done, ffn_gemm_pair_kernel<MODE>, PairCfg::SMEM_BYTES);
   if (attr_err != cudaSuccess) return attr_err;
   const int clusters = pair_clusters<MODE>();
   if (debug_log()) std::fprintf(stderr, "[moe] pair GEMM%d: %d resident clusters of 2 CTAs\n", MODE + 1, clusters);

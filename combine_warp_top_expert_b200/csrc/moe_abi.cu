@@ -315,6 +315,15 @@ const char* moe_status_string(moe_status_t status) {
 
 const char* moe_last_cuda_error(void) { return g_last_cuda_error; }
 
+int32_t moe_capacity_for(int64_t c_num, int64_t c_den, int32_t T, int32_t k, int32_t E) {
+  if (c_num < 1 || c_den < 1 || T < 0 || k < 1 || E < 1) return -1;
+  /* ceil(c_num * T * k / (c_den * E)) with no rounding: 128-bit products */
+  const unsigned __int128 num = (unsigned __int128)(uint64_t)c_num * (uint64_t)T * (uint64_t)k;
+  const unsigned __int128 den = (unsigned __int128)(uint64_t)c_den * (uint64_t)E;
+  const unsigned __int128 q = (num + den - 1) / den;
+  return q > (unsigned __int128)INT32_MAX ? -1 : (int32_t)q;
+}
+
 int moe_set_gemm_policy(int policy) {
   if (policy != kGemmAuto && policy != kGemmSingle && policy != kGemmPair && policy != kGemmSplit) return -1;
   return g_gemm_policy.exchange(policy, std::memory_order_relaxed);

@@ -120,39 +120,59 @@ moe_status_t moe_route(const moe_shape_t* shape, const float* logits, int32_t* t
  *                  [1] = max_e expert_counts[e] / mean; {1, 1} when nothing is placed.
  * Capacity (page §5 "Mitigations", capacity factor): with shape->capacity = c > 0
  * an expert keeps only its first c assignments in assignment order; the others
- * are dropped: assign_row = -1, no row, nothing added by moe_combine ("skip the
- * expert, pass through the residual"). Counts, offsets, ranks and imbalance then
- * describe the kept rows; T*k - expert_offsets[E] assignments were dropped.
- * c = ceil(C * T * k / E) gives the page's capacity factor C. */
+ * are dropped: assign_row = -1, no row, nothing added by moe_combine (a dropped
+ * assignment bypasses its expert, so the token keeps only its residual path
+ * outside this layer). Counts, offsets, ranks and imbalance then describe the
+ * kept rows; T*k - expert_offsets[E] assignments were dropped.
+ * moe_capacity_for gives c for the page's capacity factor C. */
 moe_status_t moe_dispatch(const moe_shape_t* shape, const moe_bf16_t* x, const int32_t* topk_idx,
                           int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
                           int32_t* rank_offsets, int32_t* row_src, int32_t* assign_row, moe_bf16_t* x_perm,
                           float* imbalance, void* ws, size_t ws_bytes, void* stream);
+
+/* Per-expert capacity of the capacity factor C = c_num / c_den (page "Expert
+ * Parallelism" §5 "Mitigations": an expert accepts at most C times the tokens an
+ * even split would give it). With k choices per token the even split is T*k/E
+ * assignments, so the capacity is ceil(c_num * T * k / (c_den * E)), computed in
+ * exact integer arithmetic (no rounding of C). Pass the result as
+ * moe_shape_t.capacity. Returns -1 for c_num < 1, c_den < 1, T < 0, k < 1,
+ * E < 1, or a capacity above INT32_MAX. */
+int32_t moe_capacity_for(int64_t c_num, int64_t c_den, int32_t T, int32_t k, int32_t E);
 
 /* moe_dispatch for callers that cannot allocate device memory. The pages have
  * no counterpart to this entry point: it exists for callers such as engine
  * plugins or serving runtimes whose device memory is planned and owned by their
  * own arena, and FFI callers with no CUDA allocator, for whom a cudaMalloc on the
  * hot path is not allowed or would synchronise the device.
- * Same kernels, arguments (minus the workspace) and outputs as moe_dispatch. The
- * scratch the kernels need (status word, per-chunk counts, in-chunk ranks) is a
- * fixed 1 MiB array inside the library, held on every GPU that loads the library
- * until the process exits. Shapes whose scratch exceeds it are rejected with
- * MOE_ERR_UNSUPPORTED before anything runs: the need is 256 + (bytes of
- * ceil(T / floor(2048 / k)) * E int32 rounded up to 256) + (bytes of T*k int32
- * rounded up to 256), e.g. T = 16384, k = 8, E = 256 needs 590,080 bytes.
- * This entry point allocates nothing (no cudaMalloc/cudaFree). Its first call on
- * a device looks up the array's device address (cudaGetSymbolAddress) with that
- * device current; make that first call before any stream capture. Every call
- * shares the one array and clears its status word at the start, so calls whose
- * executions overlap on the GPU (other streams, other host threads) race and
- * must be serialised by the caller.
+ * Same kernels, arguments (minus the workspace) and outputs as moe_dispatch,
+ * including the index-only form (x_perm = NULL, and x may then be NULL). The
+ * scratch the kernels need (status word, last-chunk ticket, per-chunk counts,
+ * in-chunk ranks) is a fixed 1 MiB array inside the library, held on every GPU
+ * that loads the library until the process exits. Shapes whose scratch exceeds
+ * it are rejected with MOE_ERR_UNSUPPORTED before anything runs: the need is
+ * 256 + (bytes of ceil(T / floor(2048 / k)) * E int32 rounded up to 256) +
+ * (bytes of T*k int32 rounded up to 256), e.g. T = 16384, k = 8, E = 256 needs
+ * 590,080 bytes.
+ * This entry point allocates nothing (no cudaMalloc/cudaFree). The first call in
+ * a device's CUDA context looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current, and a call after the context
+ * was re-created (cudaDeviceReset) looks it up again; make the first call on
+ * each device before any stream capture. Every call zeroes the array's header
+ * (status word and ticket) on `stream` before its kernels run, so a call never
+ * depends on what an earlier call left. Every call shares the one array, so
+ * calls whose executions overlap on the GPU (other streams, other host threads)
+ * race and must be serialised by the caller.
  *   status  device pointer to one uint32 (may be NULL): receives this call's
  *           MOE_DEV_* bits (asynchronously, on `stream`). */
 moe_status_t moe_dispatch_static(const moe_shape_t* shape, const moe_bf16_t* x, const int32_t* topk_idx,
                                  int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
                                  int32_t* rank_offsets, int32_t* row_src, int32_t* assign_row, moe_bf16_t* x_perm,
                                  float* imbalance, uint32_t* status, void* stream);
+
+/* Diagnostics of moe_dispatch_static: the device address and size of its fixed
+ * scratch array in the current device's context (the pages have no counterpart).
+ * Allocates nothing; the address is valid until the context is destroyed. */
+moe_status_t moe_dispatch_static_scratch(void** scratch, size_t* bytes);
 
 /* Expert FFN: one grouped GEMM over all experts (tcgen05 tensor cores).
  * Page "Expert Parallelism" §4 COMPUTE (every expert multiplies its own tokens;

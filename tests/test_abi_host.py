@@ -229,3 +229,46 @@ def test_capacity_for_is_the_exact_ceiling():
         assert moe.capacity_for(n / 100, T, k, E) == -(-(n * T * k) // (100 * E))
 
     check()
+
+
+def test_capacity_for_in_the_library_rejects_invalid_factors_and_overflow():
+    """moe_capacity_for (the C ABI) takes C as num/den and keeps every product in 128 bits."""
+    lib = moe.load()
+    assert lib.moe_capacity_for(5, 4, 4096, 2, 8) == 1280
+    assert lib.moe_capacity_for(1, 3, 10, 1, 1) == 4                     # ceil(10/3)
+    assert lib.moe_capacity_for(1, 1, 0, 2, 8) == 0                      # empty batch
+    for args in ((0, 1, 16, 2, 8), (1, 0, 16, 2, 8), (1, 1, -1, 2, 8), (1, 1, 16, 0, 8), (1, 1, 16, 2, 0),
+                 (-3, 1, 16, 2, 8)):
+        assert lib.moe_capacity_for(*args) == -1, args
+    big = (1 << 62)
+    assert lib.moe_capacity_for(big, 1, 1 << 30, 8, 1) == -1             # above INT32_MAX
+    assert lib.moe_capacity_for(big, big, (1 << 31) - 1, 1, 1) == (1 << 31) - 1
+    with pytest.raises(ValueError):
+        moe.capacity_for(0.0, 16, 2, 8)
+
+
+def test_layer_binding_checks_every_output_buffer():
+    """moe_layer's binding checks dtype, contiguity and shape of every output (the C ABI cannot
+    see tensor sizes), so a short `out` or a missing required buffer never reaches a kernel."""
+    import torch
+    outs = moe.alloc_layer_outputs(TINY, device="cpu")
+    ws = torch.zeros(16, dtype=torch.uint8)
+    cases = [("out", torch.empty((TINY.T - 1, TINY.d), dtype=torch.bfloat16), r"outs\['out'\] has shape"),
+             ("y_perm", torch.empty((TINY.A, TINY.d), dtype=torch.float32), r"outs\['y_perm'\] must be torch.bfloat16"),
+             ("row_src", torch.empty((TINY.A * 2,), dtype=torch.int32)[::2], r"outs\['row_src'\] must be contiguous"),
+             ("x_perm", torch.empty((TINY.A + 8, TINY.d), dtype=torch.bfloat16), r"outs\['x_perm'\] has shape"),
+             ("imbalance", torch.empty((1,), dtype=torch.float32), r"outs\['imbalance'\] has shape")]
+    for name, bad, msg in cases:
+        o = dict(outs)
+        o[name] = bad
+        with pytest.raises(ValueError, match=msg):
+            moe.moe_layer(TINY, None, None, None, None, None, None, o, ws)
+    o = dict(outs)
+    o["out"] = None
+    with pytest.raises(ValueError, match=r"outs\['out'\] is required"):
+        moe.moe_layer(TINY, None, None, None, None, None, None, o, ws)
+    sh = moe.Shape(T=16, d=128, E=8, k=2, f=128, R=2, n_shared=1)
+    o = moe.alloc_layer_outputs(sh, device="cpu")
+    o["y_shared"] = None
+    with pytest.raises(ValueError, match=r"outs\['y_shared'\] is required"):
+        moe.moe_layer(sh, None, None, None, None, None, None, o, ws)

@@ -66,3 +66,30 @@ def test_max_affine_fit_recovers_known_regimes():
     fit = bench.fit_max_affine(G, N, t)
     assert fit["b"] == pytest.approx(0.0135) and fit["beta"] == pytest.approx(6.3e-5)
     assert fit["n_star"] == pytest.approx(0.0135 / 6.3e-5) and fit["rel_rms"] < 1e-9
+
+
+def test_gpus_flag_launches_that_many_ranks():
+    """`bench.py --gpus 2` started directly (no WORLD_SIZE) re-launches itself as two ranks
+    under torch.distributed.run; --rank-check makes each rank join a gloo group, agree on the
+    slowest rank's time and report, without touching a GPU."""
+    import json
+    import subprocess
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--rank-check"],
+                       capture_output=True, text=True, timeout=240, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(ln)["rank_check"] for ln in r.stdout.splitlines() if ln.startswith('{"rank_check"')]
+    assert sorted(x["rank"] for x in lines) == [0, 1]
+    for x in lines:
+        assert x["world"] == 2 and x["gpus"] == 2
+        assert x["max_ms"] == 200.0                # the slower rank's value, on every rank
+        assert x["seed"] == x["rank"]
+
+
+def test_gpus_flag_must_match_world_size():
+    import subprocess
+    env = dict(os.environ, WORLD_SIZE="2", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "3", "--rank-check"],
+                       capture_output=True, text=True, timeout=120, env=env)
+    assert r.returncode != 0
+    assert "does not match WORLD_SIZE=2" in r.stderr

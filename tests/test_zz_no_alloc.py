@@ -10,8 +10,11 @@ This file is collected last on purpose. Through the C ABI it checks that two
 calls in a row (different shapes, so the second call runs on scratch the first
 one left behind) give exactly what moe_dispatch gives on the same inputs (bit
 for bit, the bar for integer and byte outputs), that the status output is
-per call, and that a shape needing more scratch than the array holds is refused
-before anything runs. The test only allocates the caller's own buffers.
+per call, that a call is not thrown off by what an earlier call left in the
+array's header (a non-zero last-chunk ticket), that the largest workload (64
+histogram chunks) and the index-only form (x_perm NULL) match too, and that a
+shape needing more scratch than the array holds is refused before anything
+runs. The test only allocates the caller's own buffers.
 """
 import ctypes
 
@@ -44,8 +47,9 @@ def _buffers(shape):
 def _static_call(shape, x, idx, b, status):
     lib = moe.load()
     import torch
-    rc = lib.moe_dispatch_static(ctypes.byref(shape.c()), x.data_ptr(), idx.data_ptr(),
-                                 *(b[n].data_ptr() for n in OUTS), status.data_ptr(),
+    ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+    rc = lib.moe_dispatch_static(ctypes.byref(shape.c()), ptr(x), idx.data_ptr(),
+                                 *(ptr(b[n]) for n in OUTS), status.data_ptr(),
                                  torch.cuda.current_stream().cuda_stream)
     assert rc == moe.MOE_OK, lib.moe_status_string(rc)
 
@@ -54,6 +58,36 @@ def _reference_call(shape, x, idx, b):
     ws = moe.new_workspace(shape)
     moe.moe_dispatch(shape, x, idx, *(b[n] for n in OUTS), ws)
     return moe.get_status(ws)
+
+
+def _scratch():
+    """Device address and size of the library's fixed scratch array (current device)."""
+    addr, size = ctypes.c_void_p(0), ctypes.c_size_t(0)
+    assert moe.load().moe_dispatch_static_scratch(ctypes.byref(addr), ctypes.byref(size)) == moe.MOE_OK
+    return addr.value, size.value
+
+
+def _scratch_header():
+    """The array's 256-byte header (status word at 0, last-chunk ticket at 64) as uint32."""
+    import torch
+    from cuda.bindings import runtime as rt
+    torch.cuda.synchronize()
+    addr, _ = _scratch()
+    host = np.zeros(64, np.uint32)
+    err, = rt.cudaMemcpy(host.ctypes.data, addr, 256, rt.cudaMemcpyKind.cudaMemcpyDeviceToHost)
+    assert err == rt.cudaError_t.cudaSuccess
+    return host
+
+
+def _poison_scratch_header(ticket: int, status: int):
+    import torch
+    from cuda.bindings import runtime as rt
+    torch.cuda.synchronize()
+    addr, _ = _scratch()
+    host = np.zeros(64, np.uint32)
+    host[0], host[16] = status, ticket
+    err, = rt.cudaMemcpy(addr, host.ctypes.data, 256, rt.cudaMemcpyKind.cudaMemcpyHostToDevice)
+    assert err == rt.cudaError_t.cudaSuccess
 
 
 def _case(wl, idx_np=None):
@@ -112,3 +146,77 @@ def test_static_dispatch_reports_per_call_status_and_refuses_oversized_shapes():
     fake = 1 << 20
     rc = lib.moe_dispatch_static(ctypes.byref(big.c()), *([fake] * 10), None, None)
     assert rc == moe.MOE_ERR_UNSUPPORTED
+
+
+def _chunks(shape):
+    per = max(1, 2048 // shape.k)
+    return -(-shape.T // per)
+
+
+def test_static_dispatch_ignores_a_stale_ticket_and_status_left_in_the_header():
+    """A call that was interrupted or raced could leave the last-chunk ticket and the
+    status word non-zero; the next call zeroes the header first and is still exact."""
+    import torch
+    wl = moe_synth.workload("qwen3_mixed").with_(T=1280)      # 1280 * 8 / 2048 = 5 chunks
+    shape, x, idx = _case(wl)
+    assert _chunks(shape) == 5
+    _poison_scratch_header(ticket=3, status=moe.MOE_DEV_TIMEOUT)
+    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    got, want = _buffers(shape), _buffers(shape)
+    _static_call(shape, x, idx, got, status)
+    ref_status = _reference_call(shape, x, idx, want)
+    torch.cuda.synchronize()
+    _same(got, want)
+    assert int(status.item()) == ref_status == 0
+    hdr = _scratch_header()
+    assert hdr[16] == 0 and hdr[0] == 0                        # ticket back at zero, no status bits
+
+
+def test_static_dispatch_three_then_two_chunks_leaves_the_ticket_at_zero():
+    import torch
+    status = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    for T in (768, 512):                                      # k = 8: 3 chunks, then 2
+        wl = moe_synth.workload("qwen3_mixed").with_(T=T)
+        shape, x, idx = _case(wl)
+        assert _chunks(shape) == T // 256
+        got, want = _buffers(shape), _buffers(shape)
+        _static_call(shape, x, idx, got, status)
+        _reference_call(shape, x, idx, want)
+        torch.cuda.synchronize()
+        _same(got, want)
+        assert _scratch_header()[16] == 0
+
+
+def test_static_dispatch_skewed_prefill_shape_64_chunks():
+    """The largest workload (T 16384, top-8, E 256: 64 chunks, 590,080 bytes of scratch)."""
+    import torch
+    wl = moe_synth.workload("dsv3_skewed_prefill")
+    shape, x, idx = _case(wl)
+    assert _chunks(shape) == 64
+    status = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    got, want = _buffers(shape), _buffers(shape)
+    _static_call(shape, x, idx, got, status)
+    ref_status = _reference_call(shape, x, idx, want)
+    torch.cuda.synchronize()
+    _same(got, want)
+    assert int(status.item()) == ref_status == 0
+    del got, want, x
+    torch.cuda.empty_cache()
+
+
+def test_static_dispatch_index_only():
+    """x_perm = NULL (and x = NULL): indices, counts, offsets and imbalance only."""
+    import torch
+    wl = moe_synth.workload("qwen3_mixed")
+    shape, x, idx = _case(wl)
+    status = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    got, want = _buffers(shape), _buffers(shape)
+    got["x_perm"] = None
+    _static_call(shape, None, idx, got, status)
+    _reference_call(shape, x, idx, want)
+    torch.cuda.synchronize()
+    for n in OUTS:
+        if n != "x_perm":
+            u, v = got[n], want[n]
+            assert torch.equal(u, v), n
+    assert int(status.item()) == 0
