@@ -289,6 +289,7 @@ def run_gpu(args, wl, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     moe.set_gemm_policy({"auto": moe.GEMM_AUTO, "single": moe.GEMM_SINGLE, "pair": moe.GEMM_PAIR,
                          "split": moe.GEMM_SPLIT}[args.gemm_policy])
+    moe.set_pdl(not args.no_pdl)
     wl_r = wl.with_(seed=replica_seed(wl.seed, rank))
     cap = moe.capacity_for(args.capacity_factor, wl.T, wl.k, wl.E) if args.capacity_factor else 0
     shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, n_shared=wl.n_shared, capacity=cap)
@@ -299,7 +300,13 @@ def run_gpu(args, wl, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
 
-    def step(evs):
+    def layer_step():
+        """One step as a user calls it: the whole layer, one moe_layer call."""
+        layer(dv["logits"], dv["x"], stream)
+
+    def split_step(evs):
+        """The same work as five separate entry points, with an event between them (the
+        per-step split; each interval also holds its call's launch latency)."""
         evs[0].record(stream)
         moe.moe_route(shape, dv["logits"], o["topk_idx"], o["topk_gate"], ws, stream)
         evs[1].record(stream)
@@ -321,36 +328,48 @@ def run_gpu(args, wl, rank, world, local_rank):
         evs[5].record(stream)
 
     names = ("route", "dispatch", "gate_up", "down", "combine")
-    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(6)]  # noqa: E731
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     for _ in range(args.warmup):
         flush.zero_()
-        step(mk())
+        layer_step()
     torch.cuda.synchronize(dev)
     status = moe.get_status(ws)
     counts = o["expert_counts"].cpu().numpy().tolist()
     imbalance = o["imbalance"].cpu().numpy().tolist()
 
+    # timed region: K steps of one moe_layer call each; L2 flushed before every step,
+    # outside that step's events
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    events = [mk() for _ in range(args.steps)]
+    events = [(ev(), ev()) for _ in range(args.steps)]
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
     smi_index = vis.split(",")[local_rank].strip() if vis else str(local_rank)
     with ClockSampler(smi_index) as clocks:
-        region0 = torch.cuda.Event(enable_timing=True)
-        region1 = torch.cuda.Event(enable_timing=True)
-        region0.record(stream)
         for i in range(args.steps):
             flush.zero_()
-            step(events[i])
-        region1.record(stream)
+            events[i][0].record(stream)
+            layer_step()
+            events[i][1].record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    per_step = [ev[0].elapsed_time(ev[5]) for ev in events]
-    per_kernel = {n: [ev[j].elapsed_time(ev[j + 1]) for ev in events] for j, n in enumerate(names)}
+    per_step = [a.elapsed_time(b) for a, b in events]
     max_ms = max_over_ranks(sum(per_step), world, dev)
     value = aggregate_throughput(wl.T, args.steps, world, max_ms / 1e3)
+    status |= moe.get_status(ws)
+
+    # per-step split: the same K steps through the five entry points, events between calls
+    for _ in range(2):
+        flush.zero_()
+        split_step([ev() for _ in range(6)])
+    split_events = [[ev() for _ in range(6)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        split_step(split_events[i])
+    torch.cuda.synchronize(dev)
+    per_kernel = {n: [e[j].elapsed_time(e[j + 1]) for e in split_events] for j, n in enumerate(names)}
+    split_ms = statistics.mean(e[0].elapsed_time(e[5]) for e in split_events)
 
     # e2e through the public API with host buffers (pinned): every step copies its inputs
     # host->device and its result device->host inside the timed region; successive steps
@@ -402,6 +421,7 @@ def run_gpu(args, wl, rank, world, local_rank):
                    "n_shared": wl.n_shared, "seed": wl.seed, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "flushed between steps (512 MiB write, outside the step's events)",
                    "gemm_tiles": args.gemm_policy,
+                   "launch_overlap": "off" if args.no_pdl else "programmatic dependent launch",
                    "x_perm": "not materialised (rows gathered in the gate/up GEMM)" if args.gather else "materialised",
                    "capacity_factor": args.capacity_factor, "capacity": cap,
                    "dropped_fraction": 1.0 - sum(counts) / float(wl.T * wl.k) if wl.T else 0.0,
@@ -409,6 +429,8 @@ def run_gpu(args, wl, rank, world, local_rank):
                    "expert_counts": counts,
                    "layer_roofline_frac": t_roof / (max_ms / args.steps / 1e3),
                    "per_step_ms": {n: round(v, 4) for n, v in kern_ms.items()},
+                   "per_step_split": "a second pass of K steps through the five entry points, CUDA events "
+                                     f"between calls ({split_ms:.4f} ms per step in that pass)",
                    "per_step_roofline": {n: {"bound": r["bound"], "frac": round(r["frac"], 4)} for n, r in roof.items()},
                    "peaks": peaks, "device_status": status},
         "roofline": {"kernel": f"moe_expert_{dom}", "bound": d["bound"], "achieved": d["achieved"],
@@ -424,8 +446,7 @@ def run_gpu(args, wl, rank, world, local_rank):
                 "timing": "wall clock over the K steps issued back to back (copies of each step overlap the "
                           "neighbouring steps' compute), one synchronize at the end",
                 "isolated_call_ms": e2e_single_ms},
-        # route 1 + dispatch 2 (count+scan, permute) + gate/up 1 + down 1 + combine 1 per step
-        "gpu_launches": args.steps * 6,
+        "gpu_launches": args.steps * launches_per_layer(shape, args.gemm_policy),
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
@@ -513,6 +534,14 @@ def run_regime_sweep(args):
         print(json.dumps(dict(regime_fit=fit)), flush=True)
 
 
+def launches_per_layer(shape, gemm_policy: str) -> int:
+    """Kernels one moe_layer call launches: route 1, dispatch 2 (histogram + scan, permute),
+    gate/up 1, down 1, combine 1; the split tile schedule adds a second launch to each GEMM."""
+    if shape.T == 0:
+        return 1  # dispatch's empty-batch kernel
+    return 6 + (2 if gemm_policy == "split" else 0)
+
+
 def free_port() -> int:
     import socket
     with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as so:
@@ -566,6 +595,8 @@ def main():
                          "on the default seed)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the workload's batch size T (smaller cases for profiling)")
+    ap.add_argument("--no-pdl", action="store_true",
+                    help="launch every kernel in plain stream order (no programmatic dependent launch)")
     ap.add_argument("--rank-check", action="store_true",
                     help="start the ranks, join a gloo process group, print one line per rank and exit (no GPU)")
     args = ap.parse_args()

@@ -25,6 +25,7 @@ ABI_FUNCTIONS = (
     "moe_combine", "moe_layer", "moe_status_string", "moe_last_cuda_error", "moe_set_wait_timeout_ns",
     "moe_expert_gate_up", "moe_expert_down", "moe_dispatch_static", "moe_set_gemm_policy",
     "moe_set_test_stall", "moe_expert_gate_up_gather", "moe_capacity_for", "moe_dispatch_static_scratch",
+    "moe_set_pdl",
 )
 GEMM_AUTO, GEMM_SINGLE, GEMM_PAIR, GEMM_SPLIT = 0, 1, 2, 3
 
@@ -94,6 +95,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     L.moe_last_cuda_error.argtypes = []
     L.moe_set_gemm_policy.restype = ctypes.c_int
     L.moe_set_gemm_policy.argtypes = [ctypes.c_int]
+    L.moe_set_pdl.restype = ctypes.c_int
+    L.moe_set_pdl.argtypes = [ctypes.c_int]
     L.moe_set_test_stall.restype = ctypes.c_int
     L.moe_set_test_stall.argtypes = [ctypes.c_int]
     L.moe_set_wait_timeout_ns.restype = ctypes.c_uint64
@@ -207,6 +210,11 @@ def set_wait_timeout_ns(ns: int) -> int:
 def set_test_stall(enable: bool) -> int:
     """Test hook of the bounded-wait path (see moe_set_test_stall in include/moe.h)."""
     return load().moe_set_test_stall(1 if enable else 0)
+
+
+def set_pdl(enable: bool) -> int:
+    """Programmatic dependent launch of the library's kernels on (default) or off (see moe_set_pdl)."""
+    return load().moe_set_pdl(1 if enable else 0)
 
 
 def set_gemm_policy(policy: int) -> int:

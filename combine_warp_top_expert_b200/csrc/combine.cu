@@ -24,25 +24,38 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(const uint16_t* __restr
                                                       const float* __restrict__ topk_gate,
                                                       const uint16_t* __restrict__ y_shared,
                                                       uint16_t* __restrict__ out, int64_t T, int d, int k,
-                                                      int64_t A, int slices, int vps, uint32_t* status) {
+                                                      int64_t A, int slices, int vps, uint32_t* status,
+                                                      int early_index_reads) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int nv = d >> 3;
   const int64_t items = T * slices;
   bool bad = false;
-  for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < items; w += warps) {
+  const int64_t w0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  int row = -1;
+  float g = 0.0f;
+  auto load_index = [&](int64_t w) {
     const int64_t t = w / slices;
-    const int sl = (int)(w - t * slices);
-    const int v_end = min(nv, (sl + 1) * vps);
-    int row = -1;
-    float g = 0.0f;
+    row = -1;
+    g = 0.0f;
     if (lane < k) {
       row = __ldg(assign_row + t * k + lane);
       g = __ldg(topk_gate + t * k + lane);
-      if (row >= A) {
-        bad = true;
-        row = -1;
-      }
+    }
+  };
+  /* inside the whole-layer call the indices and gates come from kernels before the
+   * down GEMM that this kernel follows: the first item's are read before pdl_wait */
+  if (early_index_reads && w0 < items) load_index(w0);
+  pdl_wait(); /* y_perm and y_shared come from the down GEMM */
+  pdl_trigger();
+  for (int64_t w = w0; w < items; w += warps) {
+    const int64_t t = w / slices;
+    const int sl = (int)(w - t * slices);
+    const int v_end = min(nv, (sl + 1) * vps);
+    if (!(early_index_reads && w == w0)) load_index(w);
+    if (lane < k && row >= A) {
+      bad = true;
+      row = -1;
     }
     int64_t src[KMAX];
     float gs[KMAX];
@@ -106,20 +119,14 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(const uint16_t* __restr
 
 cudaError_t launch_combine(const moe_shape_t& s, const uint16_t* y_perm, const int32_t* assign_row,
                            const float* topk_gate, const uint16_t* y_shared, uint16_t* out, uint32_t* status,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, bool early_index_reads) {
   if (s.T == 0) return cudaSuccess;
   const RowSlices rs = row_slices(s.T, s.d);
   const int64_t A = (int64_t)s.T * s.k;
-  if (s.k <= 2)
-    combine_kernel<4, 2><<<(unsigned)rs.blocks, 256, 0, stream>>>(y_perm, assign_row, topk_gate, y_shared, out, s.T,
-                                                                   s.d, s.k, A, rs.slices, rs.vps, status);
-  else if (s.k <= 4)
-    combine_kernel<2, 4><<<(unsigned)rs.blocks, 256, 0, stream>>>(y_perm, assign_row, topk_gate, y_shared, out, s.T,
-                                                                   s.d, s.k, A, rs.slices, rs.vps, status);
-  else
-    combine_kernel<1, 8><<<(unsigned)rs.blocks, 256, 0, stream>>>(y_perm, assign_row, topk_gate, y_shared, out, s.T,
-                                                                   s.d, s.k, A, rs.slices, rs.vps, status);
-  return cudaGetLastError();
+  auto kernel = s.k <= 2 ? combine_kernel<4, 2> : (s.k <= 4 ? combine_kernel<2, 4> : combine_kernel<1, 8>);
+  return launch_kernel(kernel, dim3((unsigned)rs.blocks), dim3(256), 0, stream, 1, y_perm, assign_row, topk_gate,
+                       y_shared, out, (int64_t)s.T, s.d, s.k, A, rs.slices, rs.vps, status,
+                       early_index_reads ? 1 : 0);
 }
 
 }  // namespace moe

@@ -144,6 +144,9 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_count_kernel(
   const int n = (int)(rem < chunk_assign ? rem : chunk_assign);
   const int per_warp = (n + kHistWarps - 1) / kHistWarps;
   const int w_begin = warp * per_warp, w_end = min(n, (warp + 1) * per_warp);
+  for (int i = threadIdx.x; i < kHistWarps * E; i += blockDim.x) hist[i] = 0;
+  pdl_wait(); /* topk_idx may come from the kernel just before this one */
+  pdl_trigger();
   /* all of this warp's expert ids in flight at once, before the histogram needs them */
   constexpr int kIters = kChunkAssign / (kHistWarps * 32);
   static_assert(kIters * kHistWarps * 32 == kChunkAssign, "a chunk is whole 32-wide steps of every warp");
@@ -153,7 +156,6 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_count_kernel(
     const int i = w_begin + it * 32 + lane;
     ev[it] = i < w_end ? __ldg(topk_idx + a0 + i) : -1;
   }
-  for (int i = threadIdx.x; i < kHistWarps * E; i += blockDim.x) hist[i] = 0;
   __syncthreads();
 
   bool bad = false;
@@ -223,6 +225,8 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_count_kernel(
 __global__ void __launch_bounds__(kScanThreads) dispatch_empty_kernel(int E, int R, int32_t* expert_counts,
                                                                       int32_t* expert_offsets, int32_t* rank_counts,
                                                                       int32_t* rank_offsets, float* imbalance) {
+  pdl_wait();
+  pdl_trigger();
   scan_chunks(nullptr, 0, E, R, 0, 0x7FFFFFFF, expert_counts, expert_offsets, rank_counts, rank_offsets, imbalance,
               nullptr);
 }
@@ -239,20 +243,31 @@ __global__ void __launch_bounds__(256) dispatch_permute_kernel(
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int nv = d >> 3; /* 16-byte vectors per row */
   const int64_t items = T * slices;
-  for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < items; w += warps) {
+  const int64_t w0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  /* the first row vectors need no index: their loads go out before the index chain.
+   * The first item's go out even before pdl_wait: x predates the count kernel that
+   * this kernel follows, and that kernel has passed its own wait when this one starts. */
+  uint4 buf[U];
+  auto load_first = [&](int64_t w) {
+    const int64_t t = w / slices;
+    const int sl = (int)(w - t * slices);
+    const uint16_t* src = x + t * d;
+    const int v_begin = sl * vps + lane, v_end = min(nv, (sl + 1) * vps);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int v = v_begin + 32 * u;
+      if (v < v_end) buf[u] = ld_nc_v4(src + (int64_t)v * 8);
+    }
+  };
+  if (x_perm != nullptr && w0 < items) load_first(w0);
+  pdl_wait(); /* chunk counts, ranks and offsets come from the count kernel */
+  pdl_trigger();
+  for (int64_t w = w0; w < items; w += warps) {
     const int64_t t = w / slices;
     const int sl = (int)(w - t * slices);
     const uint16_t* src = x_perm ? x + t * d : nullptr;
     const int v_begin = sl * vps + lane, v_end = min(nv, (sl + 1) * vps);
-    /* the first row vectors need no index: their loads go out before the index chain */
-    uint4 buf[U];
-    if (x_perm != nullptr) {
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int v = v_begin + 32 * u;
-        if (v < v_end) buf[u] = ld_nc_v4(src + (int64_t)v * 8);
-      }
-    }
+    if (x_perm != nullptr && w != w0) load_first(w);
     int pos = -1;
     if (lane < k) {
       const int64_t a = t * k + lane;
@@ -334,15 +349,15 @@ cudaError_t launch_dispatch(const moe_shape_t& s, const WsLayout& L, uint8_t* ws
   int32_t* lrank = reinterpret_cast<int32_t*>(ws + L.local_rank);
   const int64_t chunk_assign = L.tok_per_chunk * s.k;
   if (L.n_chunks == 0) {
-    dispatch_empty_kernel<<<1, kScanThreads, 0, stream>>>(s.E, s.R, expert_counts, expert_offsets, rank_counts,
-                                                          rank_offsets, imbalance);
-    return cudaGetLastError();
+    return launch_kernel(dispatch_empty_kernel, dim3(1), dim3(kScanThreads), 0, stream, 1, s.E, s.R, expert_counts,
+                         expert_offsets, rank_counts, rank_offsets, imbalance);
   }
   const size_t smem = (size_t)kHistWarps * s.E * sizeof(int32_t);
   const int32_t cap = s.capacity > 0 ? s.capacity : 0x7FFFFFFF;
-  dispatch_count_kernel<<<(unsigned)L.n_chunks, kHistThreads, smem, stream>>>(
-      topk_idx, L.A, s.E, s.R, cap, chunk_assign, L.n_chunks, chunk, lrank, status, ticket, expert_counts,
-      expert_offsets, rank_counts, rank_offsets, imbalance, row_src);
+  cudaError_t e = launch_kernel(dispatch_count_kernel, dim3((unsigned)L.n_chunks), dim3(kHistThreads), smem, stream,
+                                1, topk_idx, L.A, s.E, s.R, cap, chunk_assign, L.n_chunks, chunk, lrank, status,
+                                ticket, expert_counts, expert_offsets, rank_counts, rank_offsets, imbalance, row_src);
+  if (e != cudaSuccess) return e;
   RowSlices rs = row_slices(s.T, s.d);
   if (x_perm == nullptr) { /* indices only: one warp per token */
     rs.slices = 1;
@@ -350,10 +365,9 @@ cudaError_t launch_dispatch(const moe_shape_t& s, const WsLayout& L, uint8_t* ws
     const int64_t blocks = ((int64_t)s.T + 7) / 8, cap = (int64_t)num_sms() * 8;
     rs.blocks = (int)(blocks > cap ? cap : blocks);
   }
-  dispatch_permute_kernel<4><<<(unsigned)rs.blocks, 256, 0, stream>>>(
-      x, topk_idx, chunk, lrank, expert_offsets, s.T, s.d, s.E, s.k, cap, L.tok_per_chunk, rs.slices, rs.vps,
-      row_src, assign_row, x_perm, status);
-  return cudaGetLastError();
+  return launch_kernel(dispatch_permute_kernel<4>, dim3((unsigned)rs.blocks), dim3(256), 0, stream, 1, x, topk_idx,
+                       (const int32_t*)chunk, (const int32_t*)lrank, (const int32_t*)expert_offsets, (int64_t)s.T,
+                       s.d, s.E, s.k, cap, L.tok_per_chunk, rs.slices, rs.vps, row_src, assign_row, x_perm, status);
 }
 
 }  // namespace moe

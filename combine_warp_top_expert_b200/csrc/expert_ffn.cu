@@ -397,6 +397,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&ctl->tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
+  pdl_wait(); /* expert_offsets and the A rows come from earlier kernels */
+  pdl_trigger();
   if (warp == 2) {
     const bool ok = build_schedule<128>(p, ctl->off, ctl->mpref, ctl->hpref, lane);
     if (lane == 0) ctl->ok = ok ? 1 : 0;
@@ -717,6 +719,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc_pair(&ctl->tmem_slot, C::TMEM_COLS);
     tmem_relinquish_pair();
   }
+  pdl_wait(); /* expert_offsets and the A rows come from earlier kernels */
+  pdl_trigger();
   if (warp == 2) {
     const bool ok = build_schedule<256>(p, ctl->off, ctl->mpref, ctl->hpref, lane);
     if (lane == 0) ctl->ok = ok ? 1 : 0;
@@ -945,9 +949,8 @@ cudaError_t launch_single(const CUtensorMap& a0, const CUtensorMap& a1, const CU
   static std::atomic<int> attr_done[kMaxDevices];
   const cudaError_t attr_err = smem_opt_in(attr_done, ffn_gemm_single_kernel<MODE, BN, GATHER>, C::SMEM_BYTES);
   if (attr_err != cudaSuccess) return attr_err;
-  ffn_gemm_single_kernel<MODE, BN, GATHER>
-      <<<num_sms(), kThreads, C::SMEM_BYTES, stream>>>(a0, a1, b0, b1, o0, o1, p);
-  return cudaGetLastError();
+  return launch_kernel(ffn_gemm_single_kernel<MODE, BN, GATHER>, dim3((unsigned)num_sms()), dim3(kThreads),
+                       C::SMEM_BYTES, stream, 1, a0, a1, b0, b1, o0, o1, p);
 }
 
 /* Number of CTA pairs that can be resident at once (per device, cached). */
@@ -986,19 +989,8 @@ cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   const int clusters = pair_clusters<MODE>();
   if (debug_log()) std::fprintf(stderr, "[moe] pair GEMM%d: %d resident clusters of 2 CTAs\n", MODE + 1, clusters);
   if (clusters <= 0) return cudaSuccess; /* caller falls back to single-CTA tiles */
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3(2 * (unsigned)clusters, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = PairCfg::SMEM_BYTES;
-  cfg.stream = stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, ffn_gemm_pair_kernel<MODE>, a0, a1, b0, b1, o0, o1, p);
+  const cudaError_t e = launch_kernel(ffn_gemm_pair_kernel<MODE>, dim3(2 * (unsigned)clusters), dim3(kThreads),
+                                     PairCfg::SMEM_BYTES, stream, 2, a0, a1, b0, b1, o0, o1, p);
   if (e == cudaSuccess) *launched = true;
   return e;
 }

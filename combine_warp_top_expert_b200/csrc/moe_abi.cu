@@ -31,6 +31,7 @@ thread_local char g_last_cuda_error[256] = "";
 std::atomic<uint64_t> g_wait_timeout_ns{kDefaultWaitNs};
 std::atomic<int> g_gemm_policy{kGemmAuto};
 std::atomic<int> g_test_stall{0};
+std::atomic<int> g_pdl{1};
 
 }  // namespace
 
@@ -109,6 +110,8 @@ uint64_t wait_timeout_ns() { return g_wait_timeout_ns.load(std::memory_order_rel
 int gemm_policy() { return g_gemm_policy.load(std::memory_order_relaxed); }
 
 bool test_stall() { return g_test_stall.load(std::memory_order_relaxed) != 0; }
+
+bool pdl_enabled() { return g_pdl.load(std::memory_order_relaxed) != 0; }
 
 bool debug_log() {
   static const bool on = [] {
@@ -298,7 +301,8 @@ moe_status_t moe_layer(const moe_shape_t* shape, const moe_layer_buffers_t* b, v
   e = launch_down(*shape, L, w, b->expert_offsets, b->w2, b->w2s, b->y_perm, shape->n_shared ? b->y_shared : nullptr,
                   s);
   if (e != cudaSuccess) return cuda_fail(e);
-  e = launch_combine(*shape, b->y_perm, b->assign_row, b->topk_gate, ysh_in, b->out, status, s);
+  /* combine's predecessor is the down GEMM: assign_row and topk_gate come from earlier kernels */
+  e = launch_combine(*shape, b->y_perm, b->assign_row, b->topk_gate, ysh_in, b->out, status, s, true);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }
 
@@ -328,6 +332,8 @@ int moe_set_gemm_policy(int policy) {
   if (policy != kGemmAuto && policy != kGemmSingle && policy != kGemmPair && policy != kGemmSplit) return -1;
   return g_gemm_policy.exchange(policy, std::memory_order_relaxed);
 }
+
+int moe_set_pdl(int enable) { return g_pdl.exchange(enable ? 1 : 0, std::memory_order_relaxed); }
 
 int moe_set_test_stall(int enable) { return g_test_stall.exchange(enable ? 1 : 0, std::memory_order_relaxed); }
 

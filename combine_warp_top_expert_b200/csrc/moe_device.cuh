@@ -22,6 +22,25 @@ __device__ __forceinline__ void raise_status(uint32_t* status, uint32_t bits) {
   if (status) atomicOr(status, bits);
 }
 
+/* ---- programmatic dependent launch ----------------------------------------
+ * Every kernel of the library may be launched with programmatic stream
+ * serialization, so that its launch and prologue overlap the tail of the kernel
+ * before it in the stream. The protocol each kernel keeps:
+ *   - before pdl_wait: no global writes, and global reads only of data that the
+ *     kernel before the previous one (or an earlier stream operation) produced;
+ *   - pdl_wait, then pdl_trigger, executed by every thread;
+ *   - everything else after.
+ * Because a kernel triggers its dependent only after its own wait, a kernel that
+ * starts early finds every kernel but its immediate predecessor complete. */
+
+/* Wait until the grid this launch depends on has completed and its writes are
+ * visible (returns at once for a launch without a programmatic dependency). */
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+/* Allow the next kernel in the stream to launch (it waits in pdl_wait before it
+ * uses anything this kernel writes). */
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

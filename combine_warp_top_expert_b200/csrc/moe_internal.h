@@ -8,6 +8,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "moe.h" /* include/ is on the include path */
 
 namespace moe {
@@ -68,6 +70,39 @@ bool test_stall();
 /* MOE_DEBUG set in the environment: launch configuration notes on stderr. */
 bool debug_log();
 
+/* Launches carry programmatic stream serialization (see moe_set_pdl). */
+bool pdl_enabled();
+
+/* Launch `kernel` on `stream`, with programmatic stream serialization when
+ * pdl_enabled() (the kernel keeps the pdl_wait / pdl_trigger protocol of
+ * moe_device.cuh), and an optional cluster of `cluster_x` CTAs. */
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                          unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 cudaError_t launch_route(const float* logits, int32_t* topk_idx, float* topk_gate, int64_t T, int E, int k,
                          uint32_t* status, cudaStream_t stream);
 
@@ -87,8 +122,11 @@ cudaError_t launch_down(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, co
                         const uint16_t* w2, const uint16_t* w2s, uint16_t* y_perm, uint16_t* y_shared,
                         cudaStream_t stream);
 
+/* early_index_reads: the combine kernel may read assign_row and topk_gate before
+ * its pdl_wait (only when they come from kernels before its predecessor, as inside
+ * moe_layer; a standalone call waits first). */
 cudaError_t launch_combine(const moe_shape_t& s, const uint16_t* y_perm, const int32_t* assign_row,
                            const float* topk_gate, const uint16_t* y_shared, uint16_t* out, uint32_t* status,
-                           cudaStream_t stream);
+                           cudaStream_t stream, bool early_index_reads = false);
 
 }  // namespace moe

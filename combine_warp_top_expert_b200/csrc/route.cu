@@ -41,6 +41,8 @@ template <int NV>
 __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int32_t* __restrict__ topk_idx,
                                                     float* __restrict__ topk_gate, int64_t T, int E, int k,
                                                     uint32_t* status) {
+  pdl_wait(); /* the logits may come from the kernel just before this one */
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   bool saw_nan = false;
@@ -109,9 +111,10 @@ cudaError_t launch_route(const float* logits, int32_t* topk_idx, float* topk_gat
   if (blocks > cap) blocks = cap;
   const int nv = (E + 31) / 32;
   switch (nv) {
-#define MOE_ROUTE_CASE(N) \
-  case N:                 \
-    route_kernel<N><<<(int)blocks, threads, 0, stream>>>(logits, topk_idx, topk_gate, T, E, k, status); break;
+#define MOE_ROUTE_CASE(N)                                                                                      \
+  case N:                                                                                                      \
+    return launch_kernel(route_kernel<N>, dim3((unsigned)blocks), dim3(threads), 0, stream, 1, logits, topk_idx, \
+                         topk_gate, T, E, k, status);
     MOE_ROUTE_CASE(1)
     MOE_ROUTE_CASE(2)
     MOE_ROUTE_CASE(3)
@@ -124,7 +127,6 @@ cudaError_t launch_route(const float* logits, int32_t* topk_idx, float* topk_gat
     default:
       return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 }  // namespace moe

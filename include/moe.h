@@ -294,6 +294,16 @@ uint64_t moe_set_wait_timeout_ns(uint64_t ns);
  * or -1 for an unknown policy (unchanged). */
 int moe_set_gemm_policy(int policy);
 
+/* Launch-overlap knob: while enabled (the default, non-zero), every kernel the
+ * library launches carries programmatic stream serialization (programmatic
+ * dependent launch): it may be scheduled while the kernel before it in the
+ * stream is still running, does only work that needs none of that kernel's
+ * results, and waits for it (griddepcontrol.wait) before reading its inputs or
+ * writing anything. Results are identical either way; 0 launches every kernel
+ * in plain stream order. Process-wide, for launches made after the call.
+ * Returns the previous value. */
+int moe_set_pdl(int enable);
+
 /* Test hook for the bounded-wait path: while enabled (non-zero), every CTA of
  * the grouped-GEMM launches made after the call arms its first pipeline stage
  * but never loads it, so the MMA's wait on that stage runs out after the

@@ -297,3 +297,47 @@ def test_layer_random_shapes_match_oracle(wl, cf):
     for n in ("expert_counts", "expert_offsets", "rank_counts", "rank_offsets", "row_src", "assign_row"):
         assert np.array_equal(np_i32(outs[n]), res[n]), n
     close(f64(bits(outs["out"])), res["out"], f"out {wl.name}")
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen3_mixed", "dsv3_decode"])
+def test_layer_is_bit_identical_with_and_without_launch_overlap(name):
+    """Programmatic dependent launch changes when kernels start, not what they compute:
+    every output of moe_layer, and of the five entry points called one by one, is bit for
+    bit the same with the overlap on and off, over two calls in a row."""
+    import torch
+    wl = moe_synth.workload(name)
+    dv = moe_synth.device_inputs(wl)
+    shape = _shape(wl)
+    names = ("topk_idx", "topk_gate", "expert_offsets", "row_src", "assign_row", "x_perm", "y_perm", "out",
+             "imbalance")
+    results = {}
+    old = moe.set_pdl(True)
+    try:
+        for pdl in (True, False):
+            moe.set_pdl(pdl)
+            layer = moe.MoELayer(shape, dv["w13"], dv["w2"], dv.get("w13s"), dv.get("w2s"))
+            for _ in range(2):
+                outs = layer(dv["logits"], dv["x"])
+            assert moe.get_status(layer.ws) == 0
+            results[pdl] = {n: outs[n].clone() for n in names}
+            o, ws = layer.outs, layer.ws
+            moe.moe_route(shape, dv["logits"], o["topk_idx"], o["topk_gate"], ws)
+            moe.moe_dispatch(shape, dv["x"], o["topk_idx"], o["expert_counts"], o["expert_offsets"],
+                             o["rank_counts"], o["rank_offsets"], o["row_src"], o["assign_row"], o["x_perm"],
+                             o["imbalance"], ws)
+            moe.moe_expert_ffn(shape, o["x_perm"], o["expert_offsets"], dv["w13"], dv["w2"], dv["x"], dv.get("w13s"),
+                               dv.get("w2s"), o["y_perm"], o.get("y_shared"), ws)
+            moe.moe_combine(shape, o["y_perm"], o["assign_row"], o["topk_gate"], o.get("y_shared"), o["out"], ws)
+            assert moe.get_status(ws) == 0
+            for n in names:
+                a, b = results[pdl][n], o[n]
+                if a.dtype == torch.bfloat16:
+                    a, b = a.view(torch.int16), b.view(torch.int16)
+                assert torch.equal(a, b), (pdl, n)
+    finally:
+        moe.set_pdl(old)
+    for n in names:
+        a, b = results[True][n], results[False][n]
+        if a.dtype == torch.bfloat16:
+            a, b = a.view(torch.int16), b.view(torch.int16)
+        assert torch.equal(a, b), n
