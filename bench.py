@@ -287,8 +287,7 @@ def run_gpu(args, wl, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    moe.set_gemm_policy({"auto": moe.GEMM_AUTO, "single": moe.GEMM_SINGLE, "pair": moe.GEMM_PAIR,
-                         "split": moe.GEMM_SPLIT}[args.gemm_policy])
+    moe.set_gemm_policy({"auto": moe.GEMM_AUTO, "single": moe.GEMM_SINGLE, "pair": moe.GEMM_PAIR}[args.gemm_policy])
     moe.set_pdl(not args.no_pdl)
     wl_r = wl.with_(seed=replica_seed(wl.seed, rank))
     cap = moe.capacity_for(args.capacity_factor, wl.T, wl.k, wl.E) if args.capacity_factor else 0
@@ -454,6 +453,75 @@ def run_gpu(args, wl, rank, world, local_rank):
 
 
 # ---------------------------------------------------------------------------
+# expert parallelism across GPUs (--ep)
+# ---------------------------------------------------------------------------
+
+def run_gpu_ep(args, wl, rank, world, local_rank):
+    """The expert-parallel layer: `world` ranks (one per GPU), each with its own batch of the
+    workload's T tokens and the weights of E / world experts; rows and results cross NVLink
+    inside the dispatch and combine kernels (peer buffers in PyTorch symmetric memory).
+    At world = 1 the one rank owns every expert and exchanges with itself. Timed per step
+    with CUDA events (L2 flushed between steps), max over ranks."""
+    import torch
+    import torch.distributed as dist
+
+    import combine_warp_top_expert_b200 as moe
+    import moe_synth
+    from combine_warp_top_expert_b200 import ep
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    moe.set_pdl(not args.no_pdl)
+    if wl.E % world:
+        raise SystemExit(f"--ep needs E % ranks == 0 (E={wl.E}, ranks={world})")
+    Er = wl.E // world
+    wl_r = wl.with_(seed=replica_seed(wl.seed, rank))
+    cap = moe.capacity_for(args.capacity_factor, wl.T * world, wl.k, wl.E) if args.capacity_factor else 0
+    shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=world, n_shared=wl.n_shared, capacity=cap)
+    dv = moe_synth.device_inputs(wl_r, device=dev, weights=False)
+    wts = moe_synth.device_expert_weights(wl, rank * Er, (rank + 1) * Er, device=dev)  # this rank's experts only
+    w13, w2, w13s, w2s = wts["w13"], wts["w2"], wts.get("w13s"), wts.get("w2s")
+    rows_cap = world * wl.T * wl.k
+    peers = (ep.EPPeers.symmetric(dist.group.WORLD, wl.E, wl.d, rows_cap, dev) if world > 1
+             else ep.EPPeers.emulated(1, wl.E, wl.d, rows_cap, dev))
+    layer = ep.EPMoELayer(shape, rank, w13, w2, peers, w13s, w2s, device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        layer(dv["logits"], dv["x"])
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        evs[i][0].record()
+        layer(dv["logits"], dv["x"])
+        evs[i][1].record()
+    torch.cuda.synchronize(dev)
+    status = layer.status()
+    local_ms = sum(a.elapsed_time(b) for a, b in evs)
+    max_ms = max_over_ranks(local_ms, world, dev)
+    value = aggregate_throughput(wl.T, args.steps, world, max_ms / 1e3)
+    recv = int(layer.recv_offsets[-1].item())
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded generator; weights random-init)",
+            "config": {"workload": wl.name, "T_per_rank": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "f": wl.f,
+                       "n_shared": wl.n_shared, "parallelism": f"expert parallel x{world} (E/R = {Er} experts per GPU)",
+                       "capacity": cap, "rows_received_rank0": recv, "device_status": status,
+                       "l2": "flushed between steps (512 MiB write, outside the step's events)"},
+            # route 1; counts 2 (histogram, exchange); dispatch 4 (wait, plan, rows, signal); expert FFN 2
+            # (+2 shared) between a wait and a signal; combine 3 (wait, gather-sum, signal); final wait 1
+            "gpu_launches": args.steps * (15 + 2 * wl.n_shared),
+        }), flush=True)
+    del layer, peers
+    torch.cuda.synchronize(dev)
+
+
+# ---------------------------------------------------------------------------
 # regime sweep: per-expert cost against activated experts and tokens per expert
 # ---------------------------------------------------------------------------
 
@@ -536,10 +604,10 @@ def run_regime_sweep(args):
 
 def launches_per_layer(shape, gemm_policy: str) -> int:
     """Kernels one moe_layer call launches: route 1, dispatch 2 (histogram + scan, permute),
-    gate/up 1, down 1, combine 1; the split tile schedule adds a second launch to each GEMM."""
+    gate/up 1, down 1, combine 1."""
     if shape.T == 0:
         return 1  # dispatch's empty-batch kernel
-    return 6 + (2 if gemm_policy == "split" else 0)
+    return 6
 
 
 def free_port() -> int:
@@ -564,9 +632,11 @@ def rank_check(args, rank, world):
     dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
     try:
         mx = max_over_ranks(100.0 * (rank + 1), world)
-        print(json.dumps({"rank_check": {"rank": rank, "world": world, "gpus": args.gpus, "max_ms": mx,
-                                         "seed": replica_seed(0, rank)}}), flush=True)
-        dist.barrier()
+        mine = {"rank": rank, "world": world, "gpus": args.gpus, "max_ms": mx, "seed": replica_seed(0, rank)}
+        every = [None] * world
+        dist.all_gather_object(every, mine)
+        if rank == 0:  # one line for all ranks (the ranks share one output stream)
+            print(json.dumps({"rank_check": every}), flush=True)
     finally:
         dist.destroy_process_group()
 
@@ -579,9 +649,9 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--gemm-policy", default="auto", choices=["auto", "single", "pair", "split"],
-                    help="grouped-GEMM tiles: chosen from the shape (auto), single-CTA 128-row, CTA-pair 256x256, "
-                         "or split (pairs for whole 256-row blocks, single CTAs for short last blocks)")
+    ap.add_argument("--gemm-policy", default="auto", choices=["auto", "single", "pair"],
+                    help="grouped-GEMM tiles: chosen from the shape (auto), single-CTA 128-row, or CTA-pair 256x256 "
+                         "(a group's last block of <= 128 rows as a half-height pair tile)")
     ap.add_argument("--capacity-factor", type=float, default=None,
                     help="per-expert capacity ceil(C*T*k/E); excess assignments are dropped (default: none)")
     ap.add_argument("--regime-sweep", action="store_true",
@@ -597,6 +667,9 @@ def main():
                     help="override the workload's batch size T (smaller cases for profiling)")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch every kernel in plain stream order (no programmatic dependent launch)")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism across the --gpus ranks (E/R experts per GPU, rows exchanged over "
+                         "NVLink inside dispatch and combine) instead of independent replicas")
     ap.add_argument("--rank-check", action="store_true",
                     help="start the ranks, join a gloo process group, print one line per rank and exit (no GPU)")
     args = ap.parse_args()
@@ -640,7 +713,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_gpu(args, wl, rank, world, local_rank)
+        if args.ep:
+            run_gpu_ep(args, wl, rank, world, local_rank)
+        else:
+            run_gpu(args, wl, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

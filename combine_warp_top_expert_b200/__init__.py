@@ -25,9 +25,11 @@ ABI_FUNCTIONS = (
     "moe_combine", "moe_layer", "moe_status_string", "moe_last_cuda_error", "moe_set_wait_timeout_ns",
     "moe_expert_gate_up", "moe_expert_down", "moe_dispatch_static", "moe_set_gemm_policy",
     "moe_set_test_stall", "moe_expert_gate_up_gather", "moe_capacity_for", "moe_dispatch_static_scratch",
-    "moe_set_pdl",
+    "moe_set_pdl", "moe_ep_exchange_counts", "moe_ep_dispatch", "moe_ep_signal", "moe_ep_wait", "moe_ep_combine",
+    "moe_ep_plan_host", "moe_expert_down_combine", "moe_set_fused_combine",
 )
-GEMM_AUTO, GEMM_SINGLE, GEMM_PAIR, GEMM_SPLIT = 0, 1, 2, 3
+EP_SLOT_COUNTS, EP_SLOT_ROWS, EP_SLOT_OUTPUTS, EP_SLOT_DONE = 0, 1, 2, 3
+GEMM_AUTO, GEMM_SINGLE, GEMM_PAIR = 0, 1, 2
 
 
 class MoEError(RuntimeError):
@@ -44,6 +46,11 @@ class moe_layer_buffers_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "logits", "x", "w13", "w2", "w13s", "w2s", "topk_idx", "topk_gate", "expert_counts", "expert_offsets",
         "rank_counts", "rank_offsets", "row_src", "assign_row", "x_perm", "imbalance", "y_perm", "y_shared", "out")]
+
+
+class moe_ep_peers_t(ctypes.Structure):
+    _fields_ = [("counts", ctypes.c_void_p), ("recv_rows", ctypes.c_void_p), ("y_rows", ctypes.c_void_p),
+                ("flags", ctypes.c_void_p), ("rows_cap", ctypes.c_int64)]
 
 
 _lib = None
@@ -95,6 +102,24 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     L.moe_last_cuda_error.argtypes = []
     L.moe_set_gemm_policy.restype = ctypes.c_int
     L.moe_set_gemm_policy.argtypes = [ctypes.c_int]
+    epp = ctypes.POINTER(moe_ep_peers_t)
+    i32, u64 = ctypes.c_int32, ctypes.c_uint64
+    L.moe_ep_exchange_counts.restype = st
+    L.moe_ep_exchange_counts.argtypes = [shp, i32, u64, vp, vp, epp, vp, sz, vp]
+    L.moe_ep_dispatch.restype = st
+    L.moe_ep_dispatch.argtypes = [shp, i32, u64, vp, vp, vp, vp, epp, vp, sz, vp]
+    L.moe_ep_signal.restype = st
+    L.moe_ep_signal.argtypes = [i32, i32, i32, u64, epp, vp]
+    L.moe_ep_wait.restype = st
+    L.moe_ep_wait.argtypes = [i32, i32, i32, u64, epp, vp, sz, vp]
+    L.moe_ep_combine.restype = st
+    L.moe_ep_combine.argtypes = [shp, i32, u64, vp, vp, vp, vp, vp, epp, vp, sz, vp]
+    L.moe_ep_plan_host.restype = i32
+    L.moe_ep_plan_host.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp]
+    L.moe_expert_down_combine.restype = st
+    L.moe_expert_down_combine.argtypes = [shp] + [vp] * 9 + [vp, sz, vp]
+    L.moe_set_fused_combine.restype = ctypes.c_int
+    L.moe_set_fused_combine.argtypes = [ctypes.c_int]
     L.moe_set_pdl.restype = ctypes.c_int
     L.moe_set_pdl.argtypes = [ctypes.c_int]
     L.moe_set_test_stall.restype = ctypes.c_int
@@ -217,9 +242,14 @@ def set_pdl(enable: bool) -> int:
     return load().moe_set_pdl(1 if enable else 0)
 
 
+def set_fused_combine(enable: bool) -> int:
+    """moe_layer folds the combine into the down GEMM's epilogue (see moe_set_fused_combine)."""
+    return load().moe_set_fused_combine(1 if enable else 0)
+
+
 def set_gemm_policy(policy: int) -> int:
-    """GEMM_AUTO (chosen from the shape), GEMM_SINGLE (128-row tiles), GEMM_PAIR (CTA-pair 256x256 tiles)
-    or GEMM_SPLIT (CTA pairs for whole 256-row blocks, single CTAs for last blocks of <= 128 rows)."""
+    """GEMM_AUTO (chosen from the shape), GEMM_SINGLE (128-row single-CTA tiles) or GEMM_PAIR
+    (256 x 256 CTA-pair tiles, a group's last block of <= 128 rows as a half-height pair tile)."""
     old = load().moe_set_gemm_policy(policy)
     if old < 0:
         raise ValueError(f"unknown GEMM policy {policy}")
@@ -316,6 +346,26 @@ def moe_expert_down(shape: Shape, expert_offsets, w2, w2s, y_perm, y_shared, ws,
     _check("moe_expert_down", load().moe_expert_down(
         ctypes.byref(shape.c()), _ptr(expert_offsets), _ptr(w2), _ptr(w2s), _ptr(y_perm), _ptr(y_shared),
         *_ws(ws), _stream(stream)))
+
+
+def moe_expert_down_combine(shape: Shape, expert_offsets, w2, w2s, row_src, assign_row, topk_gate, y_perm, y_shared,
+                            out, ws, stream=None):
+    """GEMM2 with the combine folded into its epilogue: y_perm (y_shared) and out."""
+    import torch
+    bf = torch.bfloat16
+    _dev(expert_offsets, torch.int32, (shape.E + 1,), "expert_offsets")
+    _dev(w2, bf, (shape.E, shape.d, shape.f), "w2")
+    _dev(row_src, torch.int32, (shape.A,), "row_src")
+    _dev(assign_row, torch.int32, (shape.A,), "assign_row")
+    _dev(topk_gate, torch.float32, (shape.T, shape.k), "topk_gate")
+    _dev(y_perm, bf, (shape.A, shape.d), "y_perm")
+    _dev(out, bf, (shape.T, shape.d), "out")
+    if shape.n_shared:
+        _dev(w2s, bf, (shape.d, shape.f), "w2s")
+        _dev(y_shared, bf, (shape.T, shape.d), "y_shared")
+    _check("moe_expert_down_combine", load().moe_expert_down_combine(
+        ctypes.byref(shape.c()), _ptr(expert_offsets), _ptr(w2), _ptr(w2s), _ptr(row_src), _ptr(assign_row),
+        _ptr(topk_gate), _ptr(y_perm), _ptr(y_shared), _ptr(out), *_ws(ws), _stream(stream)))
 
 
 def moe_combine(shape: Shape, y_perm, assign_row, topk_gate, y_shared, out, ws, stream=None):
@@ -459,3 +509,65 @@ class MoELayer:
         """Block until the last forward_host's copy-out has landed in host memory."""
         if getattr(self, "_last_out", None) is not None:
             self._last_out.synchronize()
+
+
+# ---------------------------------------------------------------------------
+# expert parallelism across GPUs (include/moe.h, "Expert parallelism across GPUs")
+# ---------------------------------------------------------------------------
+
+def ep_plan_host(R: int, E: int, rank: int, capacity: int, counts_all) -> dict:
+    """The exchange plan of `rank` from all ranks' expert counts (int32 [R, E], host), as
+    moe_ep_plan_host computes it: row_base [E], keep [E], recv_offsets [E/R + 1]."""
+    import numpy as np
+    c = np.ascontiguousarray(counts_all, dtype=np.int32)
+    if c.shape != (R, E):
+        raise ValueError(f"counts_all has shape {c.shape}, expected {(R, E)}")
+    row_base, keep = np.empty(E, np.int32), np.empty(E, np.int32)
+    recv_offsets = np.empty(E // R + 1 if R > 0 and E % R == 0 else 1, np.int32)
+    rc = load().moe_ep_plan_host(R, E, rank, capacity, c.ctypes.data, row_base.ctypes.data, keep.ctypes.data,
+                                 recv_offsets.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"invalid plan arguments R={R} E={E} rank={rank} capacity={capacity}")
+    return dict(row_base=row_base, keep=keep, recv_offsets=recv_offsets)
+
+
+def moe_ep_exchange_counts(shape: Shape, rank: int, epoch: int, topk_idx, expert_counts, peers, ws, stream=None):
+    import torch
+    _dev(topk_idx, torch.int32, (shape.T, shape.k), "topk_idx")
+    _dev(expert_counts, torch.int32, (shape.E,), "expert_counts")
+    _check("moe_ep_exchange_counts", load().moe_ep_exchange_counts(
+        ctypes.byref(shape.c()), rank, epoch, _ptr(topk_idx), _ptr(expert_counts), ctypes.byref(peers.c()),
+        *_ws(ws), _stream(stream)))
+
+
+def moe_ep_dispatch(shape: Shape, rank: int, epoch: int, x, topk_idx, send_row, recv_offsets, peers, ws, stream=None):
+    import torch
+    _dev(x, torch.bfloat16, (shape.T, shape.d), "x")
+    _dev(topk_idx, torch.int32, (shape.T, shape.k), "topk_idx")
+    _dev(send_row, torch.int32, (shape.A,), "send_row")
+    _dev(recv_offsets, torch.int32, (shape.E // shape.R + 1,), "recv_offsets")
+    _check("moe_ep_dispatch", load().moe_ep_dispatch(
+        ctypes.byref(shape.c()), rank, epoch, _ptr(x), _ptr(topk_idx), _ptr(send_row), _ptr(recv_offsets),
+        ctypes.byref(peers.c()), *_ws(ws), _stream(stream)))
+
+
+def moe_ep_signal(R: int, rank: int, slot: int, epoch: int, peers, stream=None):
+    _check("moe_ep_signal", load().moe_ep_signal(R, rank, slot, epoch, ctypes.byref(peers.c()), _stream(stream)))
+
+
+def moe_ep_wait(R: int, rank: int, slot: int, epoch: int, peers, ws, stream=None):
+    _check("moe_ep_wait", load().moe_ep_wait(R, rank, slot, epoch, ctypes.byref(peers.c()), *_ws(ws),
+                                             _stream(stream)))
+
+
+def moe_ep_combine(shape: Shape, rank: int, epoch: int, send_row, topk_idx, topk_gate, y_shared, out, peers, ws,
+                   stream=None):
+    import torch
+    _dev(send_row, torch.int32, (shape.A,), "send_row")
+    _dev(topk_idx, torch.int32, (shape.T, shape.k), "topk_idx")
+    _dev(topk_gate, torch.float32, (shape.T, shape.k), "topk_gate")
+    _dev(y_shared, torch.bfloat16, (shape.T, shape.d), "y_shared")
+    _dev(out, torch.bfloat16, (shape.T, shape.d), "out")
+    _check("moe_ep_combine", load().moe_ep_combine(
+        ctypes.byref(shape.c()), rank, epoch, _ptr(send_row), _ptr(topk_idx), _ptr(topk_gate), _ptr(y_shared),
+        _ptr(out), ctypes.byref(peers.c()), *_ws(ws), _stream(stream)))

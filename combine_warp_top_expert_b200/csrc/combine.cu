@@ -7,7 +7,9 @@
  * indices and gates are loaded by lanes 0..k-1 and broadcast by shuffle; each
  * lane then streams 16-byte vectors of the k expert rows (+ the shared-expert
  * row), accumulates in fp32 in j order and stores one bf16 vector. Slices keep
- * every SM busy when T is small.
+ * every SM busy when T is small. The expert-parallel form reads each expert row
+ * from the GPU that computed it (peer loads over NVLink): the return trip of the
+ * page's COMBINE step fused into the weighted sum.
  *
  * Bytes per token: k*d*2 + (shared) d*2 read, d*2 written, k*8 of indices.
  */
@@ -17,22 +19,33 @@ namespace moe {
 
 namespace {
 
-/* U vectors per lane per step, rows of up to KMAX experts in flight together. */
-template <int U, int KMAX>
+/* Where the expert-parallel combine reads rows (EP form): the output buffers of the
+ * R ranks (peer-mapped device pointers); a token's row j sits in the buffer of the
+ * rank owning expert topk_idx[t, j] (experts_per_rank per rank), at assign_row. */
+struct EpSource {
+  uint16_t* const* y_rows = nullptr;
+  const int32_t* topk_idx = nullptr;
+  int experts_per_rank = 1;
+};
+
+/* U vectors per lane per step, rows of up to KMAX experts in flight together.
+ * Local form: rows come from y_perm (A rows). EP form: from the owners' buffers
+ * (ep; A is then the rows each of them holds). */
+template <int U, int KMAX, bool EP>
 __global__ void __launch_bounds__(256, 2) combine_kernel(const uint16_t* __restrict__ y_perm,
                                                       const int32_t* __restrict__ assign_row,
                                                       const float* __restrict__ topk_gate,
                                                       const uint16_t* __restrict__ y_shared,
                                                       uint16_t* __restrict__ out, int64_t T, int d, int k,
                                                       int64_t A, int slices, int vps, uint32_t* status,
-                                                      int early_index_reads) {
+                                                      int early_index_reads, const EpSource ep) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int nv = d >> 3;
   const int64_t items = T * slices;
   bool bad = false;
   const int64_t w0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  int row = -1;
+  int row = -1, owner = 0;
   float g = 0.0f;
   auto load_index = [&](int64_t w) {
     const int64_t t = w / slices;
@@ -41,6 +54,7 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(const uint16_t* __restr
     if (lane < k) {
       row = __ldg(assign_row + t * k + lane);
       g = __ldg(topk_gate + t * k + lane);
+      if (EP) owner = __ldg(ep.topk_idx + t * k + lane) / ep.experts_per_rank;
     }
   };
   /* inside the whole-layer call the indices and gates come from kernels before the
@@ -57,13 +71,15 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(const uint16_t* __restr
       bad = true;
       row = -1;
     }
-    int64_t src[KMAX];
+    const uint16_t* src[KMAX];
     float gs[KMAX];
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
       const int r = __shfl_sync(0xFFFFFFFFu, row, j);
+      const int o = __shfl_sync(0xFFFFFFFFu, owner, j);
       gs[j] = __shfl_sync(0xFFFFFFFFu, g, j);
-      src[j] = (j < k && r >= 0) ? (int64_t)r * d : -1;
+      const uint16_t* base = EP ? ep.y_rows[o] : y_perm;
+      src[j] = (j < k && r >= 0) ? base + (int64_t)r * d : nullptr;
     }
     const uint16_t* ysh = y_shared ? y_shared + t * d : nullptr;
     uint16_t* o = out + t * d;
@@ -75,7 +91,7 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(const uint16_t* __restr
 #pragma unroll
         for (int u = 0; u < U; ++u) {
           const int v = v0 + 32 * u;
-          wv[j][u] = (src[j] >= 0 && v < v_end) ? ld_nc_v4(y_perm + src[j] + (int64_t)v * 8) : make_uint4(0, 0, 0, 0);
+          wv[j][u] = (src[j] != nullptr && v < v_end) ? ld_nc_v4(src[j] + (int64_t)v * 8) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -89,7 +105,7 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(const uint16_t* __restr
         for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
 #pragma unroll
         for (int j = 0; j < KMAX; ++j) {
-          if (src[j] < 0) continue;
+          if (src[j] == nullptr) continue;
           const uint32_t ww[4] = {wv[j][u].x, wv[j][u].y, wv[j][u].z, wv[j][u].w};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -123,10 +139,26 @@ cudaError_t launch_combine(const moe_shape_t& s, const uint16_t* y_perm, const i
   if (s.T == 0) return cudaSuccess;
   const RowSlices rs = row_slices(s.T, s.d);
   const int64_t A = (int64_t)s.T * s.k;
-  auto kernel = s.k <= 2 ? combine_kernel<4, 2> : (s.k <= 4 ? combine_kernel<2, 4> : combine_kernel<1, 8>);
+  auto kernel = s.k <= 2 ? combine_kernel<4, 2, false>
+                         : (s.k <= 4 ? combine_kernel<2, 4, false> : combine_kernel<1, 8, false>);
   return launch_kernel(kernel, dim3((unsigned)rs.blocks), dim3(256), 0, stream, 1, y_perm, assign_row, topk_gate,
                        y_shared, out, (int64_t)s.T, s.d, s.k, A, rs.slices, rs.vps, status,
-                       early_index_reads ? 1 : 0);
+                       early_index_reads ? 1 : 0, EpSource{});
+}
+
+cudaError_t launch_ep_combine(const moe_shape_t& s, uint16_t* const* y_rows, int experts_per_rank, int64_t rows_cap,
+                              const int32_t* send_row, const int32_t* topk_idx, const float* topk_gate,
+                              const uint16_t* y_shared, uint16_t* out, uint32_t* status, cudaStream_t stream) {
+  if (s.T == 0) return cudaSuccess;
+  const RowSlices rs = row_slices(s.T, s.d);
+  EpSource ep;
+  ep.y_rows = y_rows;
+  ep.topk_idx = topk_idx;
+  ep.experts_per_rank = experts_per_rank;
+  auto kernel = s.k <= 2 ? combine_kernel<4, 2, true>
+                         : (s.k <= 4 ? combine_kernel<2, 4, true> : combine_kernel<1, 8, true>);
+  return launch_kernel(kernel, dim3((unsigned)rs.blocks), dim3(256), 0, stream, 1, (const uint16_t*)nullptr, send_row,
+                       topk_gate, y_shared, out, (int64_t)s.T, s.d, s.k, rows_cap, rs.slices, rs.vps, status, 0, ep);
 }
 
 }  // namespace moe

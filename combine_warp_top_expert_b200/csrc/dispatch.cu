@@ -127,7 +127,8 @@ __device__ void scan_chunks(int32_t* chunk, int64_t C, int E, int R, int64_t A, 
       imbalance[1] = (float)((double)((int64_t)s_max[1] * E) / (double)total);
     }
   }
-  for (int64_t p = total + tid; p < A; p += blockDim.x) row_src[p] = -1;
+  if (row_src)
+    for (int64_t p = total + tid; p < A; p += blockDim.x) row_src[p] = -1;
 }
 
 __global__ void __launch_bounds__(kHistThreads) dispatch_count_kernel(
@@ -231,14 +232,18 @@ __global__ void __launch_bounds__(kScanThreads) dispatch_empty_kernel(int E, int
               nullptr);
 }
 
-template <int U>
+/* EP form: rows go to the receive buffer of the rank that owns their expert, at the
+ * rows the exchange plan gives (ep.cu); x_perm, row_src and `cap` are not used. */
+template <int U, bool EP>
 __global__ void __launch_bounds__(256) dispatch_permute_kernel(
     const uint16_t* __restrict__ x, const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ chunk_base,
     const int32_t* __restrict__ local_rank, const int32_t* __restrict__ expert_offsets, int64_t T, int d, int E,
     int k, int32_t cap, int64_t tok_per_chunk, int slices, int vps, int32_t* __restrict__ row_src,
-    int32_t* __restrict__ assign_row, uint16_t* __restrict__ x_perm, uint32_t* status) {
+    int32_t* __restrict__ assign_row, uint16_t* __restrict__ x_perm, uint32_t* status, const EpTarget ep,
+    uint32_t* __restrict__ fc_cnt, uint16_t* __restrict__ fc_out, int n_shared) {
   const int lane = threadIdx.x & 31;
   const int64_t A = T * k;
+  const bool move = EP || x_perm != nullptr; /* false: index-only dispatch */
   bool bad = false;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int nv = d >> 3; /* 16-byte vectors per row */
@@ -259,23 +264,33 @@ __global__ void __launch_bounds__(256) dispatch_permute_kernel(
       if (v < v_end) buf[u] = ld_nc_v4(src + (int64_t)v * 8);
     }
   };
-  if (x_perm != nullptr && w0 < items) load_first(w0);
-  pdl_wait(); /* chunk counts, ranks and offsets come from the count kernel */
+  if (move && w0 < items) load_first(w0);
+  pdl_wait(); /* chunk counts, ranks and offsets (EP: the plan) come from the kernel before */
   pdl_trigger();
   for (int64_t w = w0; w < items; w += warps) {
     const int64_t t = w / slices;
     const int sl = (int)(w - t * slices);
-    const uint16_t* src = x_perm ? x + t * d : nullptr;
+    const uint16_t* src = move ? x + t * d : nullptr;
     const int v_begin = sl * vps + lane, v_end = min(nv, (sl + 1) * vps);
-    if (x_perm != nullptr && w != w0) load_first(w);
-    int pos = -1;
+    if (move && w != w0) load_first(w);
+    int pos = -1, owner = 0;
     if (lane < k) {
       const int64_t a = t * k + lane;
       const int e = __ldg(topk_idx + a);
       const int lr = __ldg(local_rank + a);
       if (e >= 0 && e < E && lr >= 0) {
         const int rank = __ldg(chunk_base + (t / tok_per_chunk) * E + e) + lr; /* among e's assignments */
-        if (rank < cap) {                                                      /* else dropped */
+        if (EP) {
+          if (rank < __ldg(ep.keep + e)) { /* else dropped by the capacity */
+            const int64_t q = (int64_t)__ldg(ep.row_base + e) + rank;
+            if (rank >= 0 && q >= 0 && q < ep.rows_cap) {
+              pos = (int)q;
+              owner = e / ep.experts_per_rank;
+            } else {
+              bad = true;
+            }
+          }
+        } else if (rank < cap) { /* else dropped */
           const int64_t q = (int64_t)__ldg(expert_offsets + e) + rank;
           /* a row outside [0, A) can only come from inconsistent scratch: skip it, report it */
           if (rank >= 0 && q >= 0 && q < A)
@@ -285,16 +300,28 @@ __global__ void __launch_bounds__(256) dispatch_permute_kernel(
         }
       }
       if (sl == 0) {
-        if (pos >= 0) row_src[pos] = (int32_t)a;
+        if (!EP && pos >= 0) row_src[pos] = (int32_t)a;
         assign_row[a] = pos;
       }
     }
-    if (x_perm == nullptr) continue; /* index-only dispatch */
-    int64_t dst[kMaxK];
+    if (fc_cnt != nullptr) {
+      /* the combine folded into GEMM2 follows: zero the token's counters of this slice's
+       * 64-column blocks, and, if none of its rows will arrive (all dropped, no shared
+       * expert), its output */
+      const int nb = d >> 6;
+      for (int cb = (sl * vps >> 3) + lane; cb < (v_end >> 3); cb += 32) fc_cnt[t * nb + cb] = 0u;
+      const unsigned kept = __ballot_sync(0xFFFFFFFFu, lane < k && pos >= 0);
+      if (kept == 0u && n_shared == 0)
+        for (int v = v_begin; v < v_end; v += 32) st_v4(fc_out + t * d + (int64_t)v * 8, make_uint4(0, 0, 0, 0));
+    }
+    if (!move) continue; /* index-only dispatch */
+    uint16_t* dst[kMaxK];
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) {
       const int p = __shfl_sync(0xFFFFFFFFu, pos, j);
-      dst[j] = (j < k && p >= 0) ? (int64_t)p * d : -1;
+      const int o = __shfl_sync(0xFFFFFFFFu, owner, j);
+      uint16_t* base = EP ? ep.dst_rows[o] : x_perm;
+      dst[j] = (j < k && p >= 0) ? base + (int64_t)p * d : nullptr;
     }
     for (int v0 = v_begin; v0 < v_end; v0 += 32 * U) {
       if (v0 != v_begin) {
@@ -306,16 +333,18 @@ __global__ void __launch_bounds__(256) dispatch_permute_kernel(
       }
 #pragma unroll
       for (int j = 0; j < kMaxK; ++j) {
-        if (dst[j] < 0) continue;
+        if (dst[j] == nullptr) continue;
 #pragma unroll
         for (int u = 0; u < U; ++u) {
           const int v = v0 + 32 * u;
-          if (v < v_end) st_v4(x_perm + dst[j] + (int64_t)v * 8, buf[u]);
+          if (v < v_end) st_v4(dst[j] + (int64_t)v * 8, buf[u]);
         }
       }
     }
   }
   if (bad) raise_status(status, MOE_DEV_BOUNDS);
+  /* EP: the rows went to other GPUs; make them visible there before the rank's signal */
+  if (EP) __threadfence_system();
 }
 
 }  // namespace
@@ -342,7 +371,7 @@ RowSlices row_slices(int64_t T, int d) {
 cudaError_t launch_dispatch(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const uint16_t* x,
                             const int32_t* topk_idx, int32_t* expert_counts, int32_t* expert_offsets,
                             int32_t* rank_counts, int32_t* rank_offsets, int32_t* row_src, int32_t* assign_row,
-                            uint16_t* x_perm, float* imbalance, cudaStream_t stream) {
+                            uint16_t* x_perm, float* imbalance, cudaStream_t stream, uint16_t* fc_out) {
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
   uint32_t* ticket = reinterpret_cast<uint32_t*>(ws + L.status + kTicketOffset);
   int32_t* chunk = reinterpret_cast<int32_t*>(ws + L.chunk);
@@ -365,9 +394,42 @@ cudaError_t launch_dispatch(const moe_shape_t& s, const WsLayout& L, uint8_t* ws
     const int64_t blocks = ((int64_t)s.T + 7) / 8, cap = (int64_t)num_sms() * 8;
     rs.blocks = (int)(blocks > cap ? cap : blocks);
   }
-  return launch_kernel(dispatch_permute_kernel<4>, dim3((unsigned)rs.blocks), dim3(256), 0, stream, 1, x, topk_idx,
-                       (const int32_t*)chunk, (const int32_t*)lrank, (const int32_t*)expert_offsets, (int64_t)s.T,
-                       s.d, s.E, s.k, cap, L.tok_per_chunk, rs.slices, rs.vps, row_src, assign_row, x_perm, status);
+  return launch_kernel(dispatch_permute_kernel<4, false>, dim3((unsigned)rs.blocks), dim3(256), 0, stream, 1, x,
+                       topk_idx, (const int32_t*)chunk, (const int32_t*)lrank, (const int32_t*)expert_offsets,
+                       (int64_t)s.T, s.d, s.E, s.k, cap, L.tok_per_chunk, rs.slices, rs.vps, row_src, assign_row,
+                       x_perm, status, EpTarget{},
+                       fc_out ? reinterpret_cast<uint32_t*>(ws + L.fc_cnt) : (uint32_t*)nullptr, fc_out,
+                       s.n_shared);
+}
+
+cudaError_t launch_dispatch_count(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const int32_t* topk_idx,
+                                  int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
+                                  int32_t* rank_offsets, float* imbalance, bool apply_capacity, cudaStream_t stream) {
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+  uint32_t* ticket = reinterpret_cast<uint32_t*>(ws + L.status + kTicketOffset);
+  int32_t* chunk = reinterpret_cast<int32_t*>(ws + L.chunk);
+  int32_t* lrank = reinterpret_cast<int32_t*>(ws + L.local_rank);
+  if (L.n_chunks == 0)
+    return launch_kernel(dispatch_empty_kernel, dim3(1), dim3(kScanThreads), 0, stream, 1, s.E, s.R, expert_counts,
+                         expert_offsets, rank_counts, rank_offsets, imbalance);
+  const size_t smem = (size_t)kHistWarps * s.E * sizeof(int32_t);
+  const int32_t cap = apply_capacity && s.capacity > 0 ? s.capacity : 0x7FFFFFFF;
+  return launch_kernel(dispatch_count_kernel, dim3((unsigned)L.n_chunks), dim3(kHistThreads), smem, stream, 1,
+                       topk_idx, L.A, s.E, s.R, cap, L.tok_per_chunk * s.k, L.n_chunks, chunk, lrank, status, ticket,
+                       expert_counts, expert_offsets, rank_counts, rank_offsets, imbalance, (int32_t*)nullptr);
+}
+
+cudaError_t launch_ep_scatter(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const uint16_t* x,
+                              const int32_t* topk_idx, const EpTarget& ep, int32_t* send_row, cudaStream_t stream) {
+  if (s.T == 0) return cudaSuccess;
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+  int32_t* chunk = reinterpret_cast<int32_t*>(ws + L.chunk);
+  int32_t* lrank = reinterpret_cast<int32_t*>(ws + L.local_rank);
+  const RowSlices rs = row_slices(s.T, s.d);
+  return launch_kernel(dispatch_permute_kernel<4, true>, dim3((unsigned)rs.blocks), dim3(256), 0, stream, 1, x,
+                       topk_idx, (const int32_t*)chunk, (const int32_t*)lrank, (const int32_t*)nullptr, (int64_t)s.T,
+                       s.d, s.E, s.k, (int32_t)0, L.tok_per_chunk, rs.slices, rs.vps, (int32_t*)nullptr, send_row,
+                       (uint16_t*)nullptr, status, ep, (uint32_t*)nullptr, (uint16_t*)nullptr, 0);
 }
 
 }  // namespace moe

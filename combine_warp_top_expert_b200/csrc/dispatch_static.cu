@@ -108,8 +108,8 @@ extern "C" moe_status_t moe_dispatch_static(const moe_shape_t* shape, const moe_
       (!x || (reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(x_perm) & 15)))
     return MOE_ERR_INVALID_ARG;
   const WsLayout L = ws_layout(*shape);
-  /* the dispatch kernels use the layout's prefix [0, L.h): header, chunk counts, local ranks */
-  if (L.h > kStaticScratchBytes) return MOE_ERR_UNSUPPORTED;
+  /* the dispatch kernels use the layout's prefix [0, L.dispatch_end): header, chunk counts, local ranks */
+  if (L.dispatch_end > kStaticScratchBytes) return MOE_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   cudaError_t e = scratch_address(&scratch);
   if (e == cudaSuccess) e = cudaMemsetAsync(scratch, 0, kHeaderBytes, (cudaStream_t)stream);

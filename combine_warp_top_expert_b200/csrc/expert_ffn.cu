@@ -16,33 +16,39 @@
  * n_shared = 1, a shared expert over all T rows of x.
  *
  * Schedule (device side, no host read-back of the counts): every CTA loads
- * expert_offsets, computes the m-tile prefix over the groups in shared memory,
- * and walks the linear tile index L = blockIdx.x, blockIdx.x + gridDim.x, ...
- * Inside a group the 128-row m-tiles are the inner index, so consecutive tiles
- * (running on neighbouring SMs at the same time) share one weight tile in L2.
+ * expert_offsets and computes the m-tile prefix over the groups in shared memory.
+ * The tiles are numbered group by group; inside a group the m-tiles are the inner
+ * index, so consecutive tiles share one weight tile. CTAs (CTA pairs) claim tile
+ * numbers from an atomic counter in the workspace header, so the tiles in flight
+ * at any moment are consecutive (they share weight tiles in L2 however the CTAs
+ * drift) and a CTA that finishes a tile early simply takes the next one; the last
+ * CTA to finish puts the counter back to zero for the next launch.
  *
- * Two tile shapes, same roles (warp 0 issues TMA loads from one thread, warp 1
- * owns TMEM and issues tcgen05.mma from one thread, warps 2-5 drain the
- * accumulator with tcgen05.ld and run the epilogue), two TMEM accumulators of
- * 256 fp32 columns so the epilogue of tile i overlaps the main loop of tile i+1:
+ * Two tile shapes, same roles (warp 0 claims tiles and issues TMA loads from one
+ * thread, warp 1 owns TMEM and issues tcgen05.mma from one thread, warps 2-5 drain
+ * the accumulator with tcgen05.ld and run the epilogue; the claimed tile numbers go
+ * from warp 0 to the others through a small shared-memory queue), two TMEM
+ * accumulators of 256 fp32 columns so the epilogue of tile i overlaps the main loop
+ * of tile i+1:
  *   single one CTA computes a 128 x 256 (GEMM1) or 128 x BN (GEMM2) tile with
- *          cta_group::1 MMAs (4-stage ring of 48 KB); the default for GEMM1 and
- *          for every workload whose experts average fewer than 1024 rows;
+ *          cta_group::1 MMAs (4-stage ring of 48 KB);
  *   pair   a cluster of 2 CTAs on neighbouring SMs computes a 256 x 256 tile
  *          with cta_group::2 MMAs: each CTA stages its own 128 rows of A and 128
  *          of the 256 rows of B (6-stage ring of 32 KB), so each SM moves 32 KB
- *          of operands per 64-deep K step instead of 48 KB; faster per flop but
- *          pads every group to 256 rows, so the default only for GEMM2 when
- *          d % 256 == 0 and the experts average at least 1024 rows.
- * moe_set_gemm_policy forces either shape, or a split that runs each group's
- * whole 256-row blocks as pairs and a last block of <= 128 rows in a second,
- * single-CTA launch (FfnParams::part selects the rows a launch covers).
+ *          of operands per 64-deep K step instead of 48 KB. A group's last block
+ *          of at most 128 rows runs as a half-height pair tile (M = 128, 64 rows
+ *          per CTA, half the MMA time), so pairs pad a group to a multiple of 128
+ *          rows, like single tiles.
+ * moe_set_gemm_policy chooses the shape: by default single tiles for GEMM1 and
+ * pair tiles for GEMM2 when d % 256 == 0 and the experts average at least 1024
+ * rows.
  * GEMM1 can also gather its A rows straight from x through row_src instead of
  * reading x_perm (the GATHER instantiation: a warp of cp.async copies instead of
  * one TMA tile per stage).
- * GEMM1's B tile stacks 128 gate rows over the matching 128 up rows, so one
- * N=256 MMA yields both halves of the SwiGLU for 128 output columns and the
- * epilogue combines them before anything leaves the SM.
+ * GEMM1's B tile holds gate rows and the matching up rows, so one N=256 MMA yields
+ * both halves of the SwiGLU for 128 output columns and the epilogue combines them
+ * before anything leaves the SM (single: 128 gate over 128 up rows; pair: each CTA
+ * 64 gate over the matching 64 up rows).
  * The hidden rows h live in the workspace, each group's rows padded to a
  * multiple of 256, so GEMM1 stores whole tiles and GEMM2 loads whole tiles with
  * either tile shape; GEMM2 masks its stores to the group's real rows.
@@ -85,42 +91,34 @@ struct FfnParams {
   uint32_t* status;
   uint64_t timeout_ns;
   int stall_first_stage; /* test hook: arm the first stage of each CTA's first tile but never load it */
-  int part;              /* rows of each group this launch covers: kPartAll, kPartPair or kPartTail */
+  uint32_t* tile_ctr;    /* [0]: next tile to claim, [1]: CTAs finished (workspace header; zero between launches) */
   const int32_t* row_src;   /* GEMM1 gathering A from x: row_src of dispatch (null: A is x_perm) */
   const uint16_t* gather_x; /* x [T, d] rows to gather from */
   int k;                    /* experts per token (token of assignment a = a / k) */
+  /* GEMM2 with the combine folded into its epilogue (fc_out null: y only) */
+  const int32_t* fc_row_src;    /* [A] assignment held by each row of y_perm */
+  const int32_t* fc_assign_row; /* [T*k] row of each assignment (-1: dropped) */
+  const float* fc_gate;         /* [T, k] */
+  uint16_t* fc_out;             /* [T, d] */
+  uint32_t* fc_cnt;             /* [T][d / 64] rows of a token stored so far (zero at the start) */
 };
 
 struct Tile {
   int g;           /* group: expert index, or E for the shared expert */
   int m, n;        /* m-tile inside the group, n-tile */
   int valid;       /* real rows in this m-tile (<= TM) */
+  int half;        /* CTA-pair tile of at most 128 rows: computed as M = 128 (64 rows per CTA) */
   int a_row;       /* first A row (TMA coordinate) */
   int b_row;       /* first B row (TMA coordinate); GEMM1: the gate rows */
   int64_t out_row; /* first output row */
 };
 
-/* Which rows of a group one launch covers. kPartAll: every row, in TM-row tiles.
- * The split schedule runs a group in two launches so that its last partial block
- * is not padded to 256 rows: kPartPair takes the 256-row CTA-pair tiles, including
- * a last one with more than 128 real rows; kPartTail takes a last block of 1..128
- * rows as one 128-row single-CTA tile. */
-constexpr int kPartAll = 0, kPartPair = 1, kPartTail = 2;
-
-/* m-tiles (TM rows, counted from the group's first row) of a group of `rows`
- * rows that a launch covers: [first, first + count). */
-template <int TM>
-__device__ __forceinline__ int part_tiles(int rows, int part, int* first) {
-  const int rem = rows & 255;
-  const bool short_tail = rem > 0 && rem <= 128;
-  *first = 0;
-  if (part == kPartPair) return short_tail ? rows >> 8 : (rows + 255) >> 8;
-  if (part == kPartTail) {
-    *first = (rows - rem) / TM;
-    return short_tail ? 1 : 0;
-  }
-  return (rows + TM - 1) / TM;
-}
+/* Tiles are claimed at run time: each CTA (each CTA pair) takes the next tile index
+ * from a counter in the workspace, so a CTA that finishes early (a half-height tile,
+ * or weights already in L2) takes more tiles, and the tiles running at any moment are
+ * consecutive in the order below, sharing weight tiles in L2. The claimer passes each
+ * index to the CTA's other roles through a small shared-memory queue. */
+constexpr int kTQ = 8; /* tile-queue slots */
 
 /* Shared-memory schedule, built by one warp: s_off = expert_offsets,
  * s_mpref[g] = m-tiles (TM rows) of groups < g, s_hpref[g] = 256-row blocks of h
@@ -144,8 +142,7 @@ __device__ __forceinline__ bool build_schedule(const FfnParams& p, int32_t* s_of
     } else if (g < G) {
       rows = (int)p.T;
     }
-    int first_m;
-    int im = part_tiles<TM>(rows, p.part, &first_m), ih = (rows + kHPad - 1) / kHPad;
+    int im = (rows + TM - 1) / TM, ih = (rows + kHPad - 1) / kHPad;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int ym = __shfl_up_sync(0xFFFFFFFFu, im, o);
@@ -190,11 +187,10 @@ __device__ __forceinline__ Tile decode_tile(int64_t L, const FfnParams& p, const
   const int local = (int)(L - (int64_t)s_mpref[lo] * p.n_tiles_n);
   const bool shared = lo >= p.E;
   const int rows = shared ? (int)p.T : s_off[lo + 1] - s_off[lo];
-  int first_m;
-  part_tiles<TM>(rows, p.part, &first_m);
   t.n = local / mt;
-  t.m = first_m + (local - t.n * mt);
+  t.m = local - t.n * mt;
   t.valid = min(TM, rows - t.m * TM);
+  t.half = (TM == 256 && t.valid <= 128) ? 1 : 0;
   const int hrow = s_hpref[lo] * kHPad + t.m * TM;
   if (MODE == 0) {
     t.a_row = shared ? t.m * TM : s_off[lo] + t.m * TM;
@@ -239,45 +235,178 @@ __device__ __forceinline__ void staging_reusable(int lane) {
   __syncwarp();
 }
 
-/* Epilogue of this warp's 32 accumulator rows. `taddr` addresses the warp's TMEM
- * lane quarter at the accumulator's first column; `row0` is the warp's first row
- * inside the tile (this thread's row is row0 + lane).
- * GEMM1: h = silu(gate) * up -> bf16, 128 columns, always stored (h is padded),
- *        as two TMA-stored 32 x 64 blocks.
- * GEMM2: bf16 of BN columns; a warp whose 32 rows are all real stores TMA blocks,
- *        a warp holding the expert's ragged end stores its real rows directly. */
+/* GEMM1 epilogue block: 32 rows (this warp's TMEM lanes) x 64 columns of
+ * h = silu(gate) * up, with gate at accumulator columns [gcol, gcol + 64) and up at
+ * [ucol, ucol + 64); staged in shared memory and TMA-stored at column x, row y. */
+__device__ __forceinline__ void epi_swiglu_block(uint32_t taddr, int gcol, int ucol, uint8_t* stage,
+                                                 const CUtensorMap* map, int32_t x, int32_t y, int lane) {
+  const uint32_t sbase = smem_u32(stage);
+  staging_reusable(lane);
+#pragma unroll 1
+  for (int hh = 0; hh < 2; ++hh) {
+    const int c = hh * 32;
+    uint32_t g0[16], g1[16], u0[16], u1[16];
+    tmem_ld16(taddr + gcol + c, g0);
+    tmem_ld16(taddr + gcol + c + 16, g1);
+    tmem_ld16(taddr + ucol + c, u0);
+    tmem_ld16(taddr + ucol + c + 16, u1);
+    tmem_ld_wait();
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      w[i] = pack_bf16x2(silu_f(__uint_as_float(g0[2 * i])) * __uint_as_float(u0[2 * i]),
+                         silu_f(__uint_as_float(g0[2 * i + 1])) * __uint_as_float(u0[2 * i + 1]));
+      w[8 + i] = pack_bf16x2(silu_f(__uint_as_float(g1[2 * i])) * __uint_as_float(u1[2 * i]),
+                             silu_f(__uint_as_float(g1[2 * i + 1])) * __uint_as_float(u1[2 * i + 1]));
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      stage_row_chunk(sbase, lane, hh * 4 + q, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  }
+  store_staged_block(map, stage, x, y, lane);
+}
+
+/* GEMM2 epilogue block: 32 rows x 64 columns of bf16 from accumulator columns
+ * [col, col + 64). A warp whose 32 rows are all real (whole) stages them and
+ * TMA-stores at column x, row y; a warp holding a group's ragged end stores its real
+ * rows (live lanes) directly, row by row at dst (this lane's row, column x). */
+__device__ __forceinline__ void epi_store_block(uint32_t taddr, int col, bool whole, bool live, uint16_t* dst,
+                                                uint8_t* stage, const CUtensorMap* map, int32_t x, int32_t y,
+                                                int lane) {
+  uint32_t v[4][16];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) tmem_ld16(taddr + col + q * 16, v[q]);
+  tmem_ld_wait();
+  if (whole) {
+    const uint32_t sbase = smem_u32(stage);
+    staging_reusable(lane);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const uint32_t* r = &v[q][hf * 8];
+        stage_row_chunk(sbase, lane, q * 2 + hf, pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
+                        pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
+                        pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
+                        pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
+      }
+    store_staged_block(map, stage, x, y, lane);
+  } else if (live) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const uint32_t* r = &v[q][hf * 8];
+        st_v4(dst + q * 16 + hf * 8,
+              make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
+                         pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
+                         pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
+                         pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7]))));
+      }
+  }
+}
+
+/* Combine of token `tok`, columns [cb * 64, cb * 64 + 64): the gate-weighted sum of
+ * its k rows of y_perm in j order, plus its y_shared row, fp32, one bf16 rounding
+ * (the arithmetic of the separate combine kernel). The rows were stored by any CTA
+ * of this launch: read through L2. */
+__device__ __forceinline__ void fused_combine_block(const FfnParams& p, int64_t tok, int cb) {
+#pragma unroll 1
+  for (int h = 0; h < 2; ++h) {
+    const int c0 = cb * 64 + h * 32;
+    float acc[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
+#pragma unroll 1
+    for (int j = 0; j < p.k; ++j) {
+      const int pr = __ldg(p.fc_assign_row + tok * p.k + j);
+      if (pr < 0) continue;
+      const float g = __ldg(p.fc_gate + tok * p.k + j);
+      const uint4* src = reinterpret_cast<const uint4*>(p.out0 + (int64_t)pr * p.ld_out + c0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 v = __ldcg(src + q);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[q * 8 + 2 * i] = fmaf(g, bf16lo(w[i]), acc[q * 8 + 2 * i]);
+          acc[q * 8 + 2 * i + 1] = fmaf(g, bf16hi(w[i]), acc[q * 8 + 2 * i + 1]);
+        }
+      }
+    }
+    if (p.n_shared) {
+      const uint4* sh = reinterpret_cast<const uint4*>(p.out1 + tok * p.ld_out + c0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 v = __ldcg(sh + q);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[q * 8 + 2 * i] += bf16lo(w[i]);
+          acc[q * 8 + 2 * i + 1] += bf16hi(w[i]);
+        }
+      }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(p.fc_out + tok * p.ld_out + c0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      st_v4(dst + q, make_uint4(pack_bf16x2(acc[q * 8], acc[q * 8 + 1]), pack_bf16x2(acc[q * 8 + 2], acc[q * 8 + 3]),
+                                pack_bf16x2(acc[q * 8 + 4], acc[q * 8 + 5]),
+                                pack_bf16x2(acc[q * 8 + 6], acc[q * 8 + 7])));
+  }
+}
+
+/* GEMM2 with the combine folded in: after this warp has stored its 32 rows of
+ * columns [xcol, xcol + 64 * nblk), each row counts itself in on its token's
+ * counter of every 64-column block; the row whose count completes the token (its
+ * kept assignments, plus its shared row) sums that block of the token's rows.
+ * Deterministic: the sum is taken in j order from memory, whichever row is last. */
+__device__ __forceinline__ void fused_combine_warp(const FfnParams& p, const Tile& t, int row0, int xcol, int nblk,
+                                                   int lane) {
+  if (lane == 0) {
+    bulk_wait_all(); /* this warp's TMA stores are complete ... */
+    fence_proxy_async_global(); /* ... and ordered before what the generic proxy does next */
+  }
+  __syncwarp();
+  const int r = row0 + lane;
+  if (r >= t.valid) return;
+  const bool shared = t.g >= p.E;
+  const int64_t prow = t.out_row + r;
+  int64_t tok;
+  if (shared) {
+    tok = prow;
+  } else {
+    const int a = __ldg(p.fc_row_src + prow);
+    if (a < 0) return;
+    tok = a / p.k;
+  }
+  uint32_t need = (uint32_t)p.n_shared;
+  for (int j = 0; j < p.k; ++j) need += __ldg(p.fc_assign_row + tok * p.k + j) >= 0 ? 1u : 0u;
+  __threadfence(); /* this row's stores before its count */
+  const int nb = p.d / 64;
+#pragma unroll 1
+  for (int b = 0; b < nblk; ++b) {
+    const int cb = xcol / 64 + b;
+    if (atomicAdd(p.fc_cnt + tok * nb + cb, 1u) == need - 1u) {
+      __threadfence(); /* every other row of the token is visible */
+      fused_combine_block(p, tok, cb);
+    }
+  }
+}
+
+/* Epilogue of this warp's 32 accumulator rows of a single-CTA tile. `taddr`
+ * addresses the warp's TMEM lane quarter at the accumulator's first column; `row0`
+ * is the warp's first row inside the tile (this thread's row is row0 + lane).
+ * GEMM1: the accumulator holds gate in columns [0, 128) and up in [128, 256); h =
+ *        silu(gate) * up, 128 columns, always stored (h is padded), as two blocks.
+ * GEMM2: BN columns, BN / 64 blocks, masked to the group's real rows. */
 template <int MODE, int BN>
 __device__ __forceinline__ void epilogue_warp(const FfnParams& p, const Tile& t, uint32_t taddr, int row0, int lane,
                                               uint8_t* stage, const CUtensorMap* out0, const CUtensorMap* out1) {
-  const uint32_t sbase = smem_u32(stage);
   const int32_t grow = (int32_t)(t.out_row + row0); /* output row of lane 0 */
   if (MODE == 0) {
 #pragma unroll 1
-    for (int j = 0; j < 2; ++j) {
-      staging_reusable(lane);
-#pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {
-        const int c = j * 64 + hh * 32;
-        uint32_t g0[16], g1[16], u0[16], u1[16];
-        tmem_ld16(taddr + c, g0);
-        tmem_ld16(taddr + c + 16, g1);
-        tmem_ld16(taddr + 128 + c, u0);
-        tmem_ld16(taddr + 128 + c + 16, u1);
-        tmem_ld_wait();
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          w[i] = pack_bf16x2(silu_f(__uint_as_float(g0[2 * i])) * __uint_as_float(u0[2 * i]),
-                             silu_f(__uint_as_float(g0[2 * i + 1])) * __uint_as_float(u0[2 * i + 1]));
-          w[8 + i] = pack_bf16x2(silu_f(__uint_as_float(g1[2 * i])) * __uint_as_float(u1[2 * i]),
-                                 silu_f(__uint_as_float(g1[2 * i + 1])) * __uint_as_float(u1[2 * i + 1]));
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          stage_row_chunk(sbase, lane, hh * 4 + q, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-      }
-      store_staged_block(out0, stage, t.n * 128 + j * 64, grow, lane);
-    }
+    for (int j = 0; j < 2; ++j) epi_swiglu_block(taddr, j * 64, 128 + j * 64, stage, out0, t.n * 128 + j * 64, grow, lane);
   } else {
     const bool shared = t.g >= p.E;
     const CUtensorMap* map = shared ? out1 : out0;
@@ -285,38 +414,52 @@ __device__ __forceinline__ void epilogue_warp(const FfnParams& p, const Tile& t,
     const bool live = row0 + lane < t.valid;
     uint16_t* dst = (shared ? p.out1 : p.out0) + (t.out_row + row0 + lane) * p.ld_out + (int64_t)t.n * BN;
 #pragma unroll 1
-    for (int j = 0; j < BN / 64; ++j) {
-      uint32_t v[4][16];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld16(taddr + j * 64 + q * 16, v[q]);
-      tmem_ld_wait();
-      if (whole) {
-        staging_reusable(lane);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            const uint32_t* r = &v[q][hf * 8];
-            stage_row_chunk(sbase, lane, q * 2 + hf, pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
-                            pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
-                            pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
-                            pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
-          }
-        store_staged_block(map, stage, t.n * BN + j * 64, grow, lane);
-      } else if (live) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            const uint32_t* r = &v[q][hf * 8];
-            st_v4(dst + j * 64 + q * 16 + hf * 8,
-                  make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
-                             pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
-                             pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
-                             pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7]))));
-          }
-      }
+    for (int j = 0; j < BN / 64; ++j)
+      epi_store_block(taddr, j * 64, whole, live, dst + j * 64, stage, map, t.n * BN + j * 64, grow, lane);
+    if (p.fc_out) fused_combine_warp(p, t, row0, t.n * BN, BN / 64, lane);
+  }
+}
+
+/* Epilogue of warp q (lane quarter q) of CTA `rank` of a CTA-pair tile.
+ * Full tile (M = 256): the CTA holds rows [rank * 128, +128) of the tile, warp q
+ *   rows q * 32 + [0, 32), every column of the tile.
+ * Half tile (M = 128, at most 128 real rows): the CTA holds rows [rank * 64, +64);
+ *   TMEM lanes 0-63 hold them for the tile's first half of columns and lanes 64-127
+ *   the same rows for the second half, so warp q has rows (q % 2) * 32 + [0, 32) and
+ *   column half q / 2.
+ * GEMM1: each CTA staged 64 gate rows and the matching 64 up rows of the weights, so
+ *   the accumulator columns run [gate 64 | up 64] per 64 columns of h: a full tile
+ *   has h columns [0, 64) from gate [0, 64) / up [64, 128) and [64, 128) from gate
+ *   [128, 192) / up [192, 256); a half tile's warp has its 64 h columns from gate
+ *   [0, 64) / up [64, 128) of its lanes.
+ * GEMM2: 256 output columns (full) or 128 per column half (half). */
+template <int MODE>
+__device__ __forceinline__ void epilogue_pair_warp(const FfnParams& p, const Tile& t, uint32_t taddr, int q,
+                                                   uint32_t rank, int lane, uint8_t* stage, const CUtensorMap* out0,
+                                                   const CUtensorMap* out1) {
+  const int row0 = t.half ? (int)rank * 64 + (q & 1) * 32 : (int)rank * 128 + q * 32; /* inside the tile */
+  const int col0 = t.half ? (q >> 1) * (MODE == 0 ? 64 : 128) : 0;                   /* inside the tile */
+  const int32_t grow = (int32_t)(t.out_row + row0);
+  if (MODE == 0) {
+    if (t.half) {
+      epi_swiglu_block(taddr, 0, 64, stage, out0, t.n * 128 + col0, grow, lane);
+    } else {
+#pragma unroll 1
+      for (int j = 0; j < 2; ++j)
+        epi_swiglu_block(taddr, j * 128, j * 128 + 64, stage, out0, t.n * 128 + j * 64, grow, lane);
     }
+  } else {
+    const bool shared = t.g >= p.E;
+    const CUtensorMap* map = shared ? out1 : out0;
+    const bool whole = row0 + 32 <= t.valid; /* warp-uniform */
+    const bool live = row0 + lane < t.valid;
+    const int xcol = t.n * 256 + col0;
+    uint16_t* dst = (shared ? p.out1 : p.out0) + (t.out_row + row0 + lane) * p.ld_out + (int64_t)xcol;
+    const int nblk = t.half ? 2 : 4;
+#pragma unroll 1
+    for (int j = 0; j < nblk; ++j)
+      epi_store_block(taddr, j * 64, whole, live, dst + j * 64, stage, map, xcol + j * 64, grow, lane);
+    if (p.fc_out) fused_combine_warp(p, t, row0, xcol, nblk, lane);
   }
 }
 
@@ -327,6 +470,9 @@ struct Ctrl {
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
+  uint64_t tq_full[kTQ];  /* tile index written (claimer arrives) */
+  uint64_t tq_empty[kTQ]; /* tile index read by every consumer role */
+  int32_t tq[kTQ];        /* claimed tile index, -1 = no more tiles */
   uint32_t tmem_slot;
   int abort_flag;
   int ok;
@@ -350,6 +496,36 @@ struct SingleCfg {
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
+
+/* Claim the next tile index (-1 once every tile is taken). One thread per CTA (per
+ * CTA pair) claims; the counter sits in the workspace header. */
+__device__ __forceinline__ int claim_tile(const FfnParams& p, int64_t total) {
+  const uint32_t L = atomicAdd(p.tile_ctr, 1u);
+  return (int64_t)L < total ? (int)L : -1;
+}
+
+/* Called once per CTA by one thread after every role has stopped claiming: the
+ * last CTA of the launch to get here puts the counters back to zero, ready for the
+ * next launch on this workspace (which touches them only after this one completed). */
+__device__ __forceinline__ void release_tile_counter(const FfnParams& p) {
+  __threadfence();
+  if (atomicAdd(p.tile_ctr + 1, 1u) == gridDim.x - 1) {
+    atomicExch(p.tile_ctr, 0u);
+    atomicExch(p.tile_ctr + 1, 0u);
+  }
+}
+
+/* A consumer role's turn on queue slot i: wait for the claimed index, read it. The
+ * caller releases the slot (tq_empty) once it has the value. Returns false on
+ * timeout or abort. CLUSTER: the index was written by the peer CTA of a pair. */
+template <bool CLUSTER = false>
+__device__ __forceinline__ bool read_tile_index(Ctrl* ctl, int i, uint64_t timeout_ns, volatile int* s_abort,
+                                                int* v) {
+  const int slot = i % kTQ;
+  if (!mbar_wait<CLUSTER>(&ctl->tq_full[slot], (uint32_t)(i / kTQ) & 1u, timeout_ns, s_abort)) return false;
+  *v = *reinterpret_cast<volatile int32_t*>(&ctl->tq[slot]);
+  return true;
+}
 
 template <int MODE, int BN, bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -380,6 +556,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&ctl->tfull[b], 1);
       mbar_init(&ctl->tempty[b], 4);
+    }
+    for (int i = 0; i < kTQ; ++i) {
+      mbar_init(&ctl->tq_full[i], 1);
+      mbar_init(&ctl->tq_empty[i], 5); /* the MMA issuer and the 4 epilogue warps */
     }
     mbar_init(&ctl->drain, 1);
     ctl->abort_flag = 0;
@@ -417,91 +597,93 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int KB = p.K / BK;
 
   if (warp == 0) {
-    if constexpr (!GATHER) {
+    /* ---------------- producer: claims tiles, loads their operands ----------------
+     * Lane 0 claims each tile and passes its index on through the tile queue. The
+     * TMA form issues from lane 0 alone; the gathering form has the whole warp copy
+     * the A rows (see below). */
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t armed_phase[STAGES];
+    bool armed[STAGES];
+#pragma unroll
+    for (int s = 0; s < STAGES; ++s) {
+      armed[s] = false;
+      armed_phase[s] = 0;
+    }
+    bool abort = false;
+    bool first = true;
+    /* the claim for the next tile goes out one tile ahead, so that its round trip to
+     * L2 overlaps the loads of the current tile */
+    int next = lane == 0 ? claim_tile(p, total) : -1;
+    /* gathering: lane l moves 16-byte chunk l % 8 of rows l / 8 + 4 i (i < 32) */
+    const int chunk = lane & 7, row0 = lane >> 3;
+    /* swizzle of rows row0 + 4 i: (row0 + 4 i) % 8 == row0 ^ (4 (i % 2)) since row0 < 4 */
+    const uint32_t sw_even = (uint32_t)(chunk ^ row0) << 4, sw_odd = (uint32_t)(chunk ^ row0 ^ 4) << 4;
+    const uint32_t row_bytes = (uint32_t)p.d * 2u; /* T * d * 2 < 2^32 is checked on the host */
+    const char* xk0 = GATHER ? reinterpret_cast<const char*>(p.gather_x) + chunk * 16 : nullptr;
+    for (int i = 0; !abort; ++i) {
+      if (!GATHER && lane != 0) break;
+      int v = -1;
       if (lane == 0) {
-        /* ---------------- TMA producer ---------------- */
-        int stage = 0;
-        uint32_t phase = 0;
-        uint32_t armed_phase[STAGES];
-        bool armed[STAGES];
-  #pragma unroll
-        for (int s = 0; s < STAGES; ++s) {
-          armed[s] = false;
-          armed_phase[s] = 0;
+        const int slot = i % kTQ;
+        if (!mbar_wait(&ctl->tq_empty[slot], ((uint32_t)(i / kTQ) & 1u) ^ 1u, p.timeout_ns, s_abort)) {
+          abort = true;
+        } else {
+          v = next;
+          ctl->tq[slot] = v;
+          mbar_arrive(&ctl->tq_full[slot]);
+          if (v >= 0) next = claim_tile(p, total);
         }
-        bool abort = false;
-        for (int64_t L = blockIdx.x; L < total && !abort; L += gridDim.x) {
-          const Tile t = decode_tile<MODE, 128, BN>(L, p, ctl->off, ctl->mpref, ctl->hpref);
-          const bool shared = t.g >= p.E;
-          const CUtensorMap* mA = shared ? &tmA1 : &tmA0;
-          const CUtensorMap* mB = shared ? &tmB1 : &tmB0;
-          for (int kb = 0; kb < KB; ++kb) {
-            if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, p.timeout_ns, s_abort)) {
-              abort = true;
-              break;
-            }
-            mbar_arrive_expect_tx(&ctl->full[stage], C::STAGE_BYTES);
-            if (p.stall_first_stage && L == blockIdx.x && kb == 0) {
-              /* test hook: this stage's bytes never arrive, so the MMA's bounded wait runs out */
-              if (++stage == STAGES) {
-                stage = 0;
-                phase ^= 1u;
-              }
-              continue;
-            }
-            armed[stage] = true;
-            armed_phase[stage] = phase;
-            uint8_t* a_dst = sA + stage * HALF_TILE;
-            uint8_t* b_dst = sB + stage * C::B_BYTES;
-            tma_load_2d(a_dst, mA, &ctl->full[stage], kb * BK, t.a_row);
-            if (MODE == 0) {
-              tma_load_2d(b_dst, mB, &ctl->full[stage], kb * BK, t.b_row);
-              tma_load_2d(b_dst + HALF_TILE, mB, &ctl->full[stage], kb * BK, t.b_row + p.f);
-            } else {
-              tma_load_2d(b_dst, mB, &ctl->full[stage], kb * BK, t.b_row);
-            }
+      }
+      if (GATHER) {
+        v = __shfl_sync(0xFFFFFFFFu, v, 0);
+        abort = __shfl_sync(0xFFFFFFFFu, abort ? 1 : 0, 0) != 0;
+      }
+      if (abort || v < 0) break;
+      const Tile t = decode_tile<MODE, 128, BN>(v, p, ctl->off, ctl->mpref, ctl->hpref);
+      const bool shared = t.g >= p.E;
+      if constexpr (!GATHER) {
+        /* TMA tiles, lane 0 only */
+        const CUtensorMap* mA = shared ? &tmA1 : &tmA0;
+        const CUtensorMap* mB = shared ? &tmB1 : &tmB0;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, p.timeout_ns, s_abort)) {
+            abort = true;
+            break;
+          }
+          mbar_arrive_expect_tx(&ctl->full[stage], C::STAGE_BYTES);
+          if (p.stall_first_stage && first && kb == 0) {
+            /* test hook: this stage's bytes never arrive, so the MMA's bounded wait runs out */
             if (++stage == STAGES) {
               stage = 0;
               phase ^= 1u;
             }
+            continue;
+          }
+          armed[stage] = true;
+          armed_phase[stage] = phase;
+          uint8_t* a_dst = sA + stage * HALF_TILE;
+          uint8_t* b_dst = sB + stage * C::B_BYTES;
+          tma_load_2d(a_dst, mA, &ctl->full[stage], kb * BK, t.a_row);
+          if (MODE == 0) {
+            tma_load_2d(b_dst, mB, &ctl->full[stage], kb * BK, t.b_row);
+            tma_load_2d(b_dst + HALF_TILE, mB, &ctl->full[stage], kb * BK, t.b_row + p.f);
+          } else {
+            tma_load_2d(b_dst, mB, &ctl->full[stage], kb * BK, t.b_row);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
           }
         }
-        if (abort) {
-          raise_status(p.status, MOE_DEV_TIMEOUT);
-          *s_abort = 1;
-        }
-        /* every armed stage's copies must land before the CTA may exit */
-        for (int s = 0; s < STAGES; ++s)
-          if (armed[s]) mbar_wait(&ctl->full[s], armed_phase[s], kDrainNs, nullptr);
-      }
-    } else {
-      /* ---------------- producer warp, A gathered from x ----------------
-       * Lane 0 waits for free stages, arms them and TMA-loads B (and A for the
-       * shared expert, whose rows are x itself). The routed rows of GEMM1 come
-       * straight from x: row p of expert e is token row_src[p] / k. The whole warp
-       * copies them with 16-byte cp.async into the 128-byte swizzled layout of the
-       * stage: lane l moves 16-byte chunk l % 8 of rows l / 8 + 4 i (i < 32), so one
-       * instruction covers four 128-byte row segments, and each lane's byte offsets
-       * into x stay in registers for the whole tile. Every lane arrives on every
-       * stage barrier once its copies have landed (the barrier counts 32 + 1). */
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t armed_phase[STAGES];
-      bool armed[STAGES];
-#pragma unroll
-      for (int s = 0; s < STAGES; ++s) {
-        armed[s] = false;
-        armed_phase[s] = 0;
-      }
-      bool abort = false;
-      const int chunk = lane & 7, row0 = lane >> 3;
-      /* swizzle of rows row0 + 4 i: (row0 + 4 i) % 8 == row0 ^ (4 (i % 2)) since row0 < 4 */
-      const uint32_t sw_even = (uint32_t)(chunk ^ row0) << 4, sw_odd = (uint32_t)(chunk ^ row0 ^ 4) << 4;
-      const uint32_t row_bytes = (uint32_t)p.d * 2u; /* T * d * 2 < 2^32 is checked on the host */
-      const char* xk0 = reinterpret_cast<const char*>(p.gather_x) + chunk * 16;
-      for (int64_t L = blockIdx.x; L < total && !abort; L += gridDim.x) {
-        const Tile t = decode_tile<MODE, 128, BN>(L, p, ctl->off, ctl->mpref, ctl->hpref);
-        const bool shared = t.g >= p.E;
+      } else {
+        /* A gathered from x: lane 0 waits for free stages, arms them and TMA-loads B
+         * (and A for the shared expert, whose rows are x itself). The routed rows of
+         * GEMM1 come straight from x: row p of expert e is token row_src[p] / k. The
+         * whole warp copies them with 16-byte cp.async into the 128-byte swizzled
+         * layout of the stage; each lane's byte offsets into x stay in registers for
+         * the whole tile. Every lane arrives on every stage barrier once its copies
+         * have landed (the barrier counts 32 + 1). */
         uint32_t goff[32];
         if (!shared) {
           /* rows past the expert's end read token 0 (computed, never stored); a row index
@@ -510,14 +692,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int r0 = ctl->off[t.g] + t.m * 128 + row0;
           bool bad = false;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int r = r0 + 4 * i;
+          for (int i2 = 0; i2 < 32; ++i2) {
+            const int r = r0 + 4 * i2;
             uint32_t tok = r < r_end ? (uint32_t)__ldg(p.row_src + r) / (uint32_t)p.k : 0u;
             if (tok >= (uint32_t)p.T) {
               bad = true;
               tok = 0u;
             }
-            goff[i] = tok * row_bytes;
+            goff[i2] = tok * row_bytes;
           }
           if (bad) raise_status(p.status, MOE_DEV_BOUNDS);
         }
@@ -530,7 +712,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = mbar_wait(&ctl->empty[stage], phase ^ 1u, p.timeout_ns, s_abort) ? 1 : 0;
             if (ok) {
               mbar_arrive_expect_tx(&ctl->full[stage], tx_bytes);
-              if (p.stall_first_stage && L == blockIdx.x && kb == 0) {
+              if (p.stall_first_stage && first && kb == 0) {
                 skip = 1; /* test hook: this stage's bytes never arrive, so the MMA's bounded wait runs out */
               } else {
                 armed[stage] = true;
@@ -553,8 +735,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t a_base = smem_u32(a_dst) + (uint32_t)row0 * 128u;
             const char* xk = xk0 + (int64_t)kb * (BK * 2);
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              cp_async_16(a_base + (uint32_t)i * 512u + ((i & 1) ? sw_odd : sw_even), xk + goff[i]);
+            for (int i2 = 0; i2 < 32; ++i2)
+              cp_async_16(a_base + (uint32_t)i2 * 512u + ((i2 & 1) ? sw_odd : sw_even), xk + goff[i2]);
           }
           cp_async_mbar_arrive(&ctl->full[stage]);
           if (++stage == STAGES) {
@@ -563,15 +745,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (lane == 0) {
-        if (abort) {
-          raise_status(p.status, MOE_DEV_TIMEOUT);
-          *s_abort = 1;
-        }
-        /* every armed stage's copies must land before the CTA may exit */
-        for (int s = 0; s < STAGES; ++s)
-          if (armed[s]) mbar_wait(&ctl->full[s], armed_phase[s], kDrainNs, nullptr);
+      first = false;
+    }
+    if (lane == 0) {
+      if (abort) {
+        raise_status(p.status, MOE_DEV_TIMEOUT);
+        *s_abort = 1;
       }
+      /* every armed stage's copies must land before the CTA may exit */
+      for (int s = 0; s < STAGES; ++s)
+        if (armed[s]) mbar_wait(&ctl->full[s], armed_phase[s], kDrainNs, nullptr);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -580,7 +763,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       uint32_t acc = 0;
       bool abort = false;
-      for (int64_t L = blockIdx.x; L < total && !abort; L += gridDim.x, ++acc) {
+      for (int i = 0;; ++i, ++acc) {
+        int v;
+        if (!read_tile_index(ctl, i, p.timeout_ns, s_abort, &v)) {
+          abort = true;
+          break;
+        }
+        mbar_arrive(&ctl->tq_empty[i % kTQ]);
+        if (v < 0) break;
         const uint32_t b = acc & 1u, use = (acc >> 1) & 1u;
         if (!mbar_wait(&ctl->tempty[b], use ^ 1u, p.timeout_ns, s_abort)) {
           abort = true;
@@ -625,8 +815,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     /* ---------------- epilogue (warps 2..5, 128 threads) ---------------- */
     const int q = warp & 3; /* TMEM lane quarter this warp may access */
     uint32_t acc = 0;
-    for (int64_t L = blockIdx.x; L < total; L += gridDim.x, ++acc) {
-      const Tile t = decode_tile<MODE, 128, BN>(L, p, ctl->off, ctl->mpref, ctl->hpref);
+    for (int i = 0;; ++i, ++acc) {
+      int v = -1;
+      const bool got = read_tile_index(ctl, i, p.timeout_ns, s_abort, &v);
+      __syncwarp();
+      if (!got) {
+        if (lane == 0) {
+          raise_status(p.status, MOE_DEV_TIMEOUT);
+          *s_abort = 1;
+        }
+        break;
+      }
+      if (lane == 0) mbar_arrive(&ctl->tq_empty[i % kTQ]);
+      if (v < 0) break;
+      const Tile t = decode_tile<MODE, 128, BN>(v, p, ctl->off, ctl->mpref, ctl->hpref);
       const uint32_t b = acc & 1u, use = (acc >> 1) & 1u;
       if (!mbar_wait(&ctl->tfull[b], use, p.timeout_ns, s_abort)) {
         if (lane == 0) {
@@ -651,6 +853,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
+  if (threadIdx.x == 0) release_tile_counter(p);
 }
 
 /* ================= CTA-pair tiles (256 x 256, cta_group::2) ================= */
@@ -659,23 +862,30 @@ struct PairCfg {
   static constexpr int STAGES = 6;
   static constexpr uint32_t STAGE_BYTES = 2 * HALF_TILE;       /* per CTA: 128 rows of A + 128 rows of B */
   static constexpr uint32_t STAGE_TX = 2 * STAGE_BYTES;        /* bytes landing per stage in both CTAs */
+  static constexpr uint32_t STAGE_TX_HALF = 2 * (HALF_TILE / 2 + HALF_TILE); /* 64 rows of A per CTA */
   static constexpr uint32_t ACC_COLS = 256;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t IDESC = umma_idesc_bf16(256, 256);
+  static constexpr uint32_t IDESC_HALF = umma_idesc_bf16(128, 256);
   static constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + kEpiStagingBytes + sizeof(Ctrl);
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-/* A cluster of two CTAs (ranks 0 and 1) works on one 256-row x 256-column tile:
- * rank r stages A rows [r*128, r*128+128) of the tile and B rows
- * [r*128, r*128+128) of the 256 (GEMM1: r = 0 the gate rows, r = 1 the up rows),
- * and holds accumulator rows [r*128, r*128+128) in its own TMEM. Rank 0 arms the
- * stage barrier for the bytes of both CTAs and issues the MMAs; its commits
- * arrive on the barriers of both CTAs; rank 1's epilogue releases accumulators
- * on rank 0's barrier. */
+/* A cluster of two CTAs (ranks 0 and 1) works on one tile of up to 256 rows x 256
+ * columns. Full tile: rank r stages A rows [r*128, r*128+128) of the tile, holds
+ * accumulator rows [r*128, +128) in its own TMEM, and the MMAs are M = 256. Half
+ * tile (a group's last block of at most 128 rows): rank r stages A rows
+ * [r*64, r*64+64) and the MMAs are M = 128, at half the cost. Either way rank r
+ * stages 128 of the 256 B rows: GEMM2 rows [r*128, +128); GEMM1 the 64 gate rows
+ * [n*128 + r*64, +64) of the tile's 128 h columns and the matching 64 up rows.
+ * Rank 0 claims the tiles and writes each index into both CTAs' queues, arms the
+ * stage barrier for the bytes of both CTAs and issues the MMAs; its commits arrive
+ * on the barriers of both CTAs; rank 1's consumers release queue slots and
+ * accumulators on rank 0's barriers. */
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     ffn_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                         const __grid_constant__ CUtensorMap tmA0h, const __grid_constant__ CUtensorMap tmA1h,
                          const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
                          const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
                          const FfnParams p) {
@@ -692,7 +902,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
-  const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -703,6 +912,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ctl->tfull[b], 1);
       mbar_init(&ctl->tempty[b], 8); /* 4 epilogue warps in each CTA */
     }
+    for (int i = 0; i < kTQ; ++i) {
+      mbar_init(&ctl->tq_full[i], 1);
+      /* rank 0's barrier counts every consumer of a queue slot: its MMA issuer and 4
+       * epilogue warps, rank 1's producer and 4 epilogue warps */
+      mbar_init(&ctl->tq_empty[i], 10);
+    }
     mbar_init(&ctl->drain, 1);
     ctl->abort_flag = 0;
     fence_barrier_init();
@@ -710,6 +925,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA0);
     tma_prefetch_desc(&tmA1);
+    tma_prefetch_desc(&tmA0h);
+    tma_prefetch_desc(&tmA1h);
     tma_prefetch_desc(&tmB0);
     tma_prefetch_desc(&tmB1);
     tma_prefetch_desc(&tmO0);
@@ -738,10 +955,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(p.status, MOE_DEV_COUNT_MISMATCH);
   }
   const int KB = p.K / BK;
+  /* a consumer releases a queue slot on rank 0's barrier */
+  auto release_slot = [&](int i) {
+    if (leader)
+      mbar_arrive(&ctl->tq_empty[i % kTQ]);
+    else
+      mbar_arrive_cluster(mapa_shared(smem_u32(&ctl->tq_empty[i % kTQ]), 0));
+  };
 
   if (warp == 0) {
     if (lane == 0) {
-      /* ---------------- TMA producer (both CTAs) ---------------- */
+      /* ---------------- tile claimer (rank 0) and TMA producers (both CTAs) ---------------- */
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed_phase[STAGES];
@@ -752,21 +976,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         armed_phase[s] = 0;
       }
       bool abort = false;
-      for (int64_t L = pair; L < total && !abort; L += npairs) {
-        const Tile t = decode_tile<MODE, 256, 256>(L, p, ctl->off, ctl->mpref, ctl->hpref);
+      bool first = true;
+      int next = leader ? claim_tile(p, total) : -1; /* claimed one tile ahead (see the single kernel) */
+      for (int i = 0;; ++i) {
+        const int slot = i % kTQ;
+        int v = -1;
+        if (leader) {
+          if (!mbar_wait<true>(&ctl->tq_empty[slot], ((uint32_t)(i / kTQ) & 1u) ^ 1u, p.timeout_ns, s_abort)) {
+            abort = true;
+            break;
+          }
+          v = next;
+          ctl->tq[slot] = v;
+          st_shared_cluster_u32(mapa_shared(smem_u32(&ctl->tq[slot]), 1), (uint32_t)v);
+          mbar_arrive(&ctl->tq_full[slot]);
+          mbar_arrive_cluster(mapa_shared(smem_u32(&ctl->tq_full[slot]), 1)); /* release: orders the store */
+          if (v >= 0) next = claim_tile(p, total);
+        } else {
+          if (!read_tile_index<true>(ctl, i, p.timeout_ns, s_abort, &v)) {
+            abort = true;
+            break;
+          }
+          release_slot(i);
+        }
+        if (v < 0) break;
+        const Tile t = decode_tile<MODE, 256, 256>(v, p, ctl->off, ctl->mpref, ctl->hpref);
         const bool shared = t.g >= p.E;
-        const CUtensorMap* mA = shared ? &tmA1 : &tmA0;
+        const CUtensorMap* mA = t.half ? (shared ? &tmA1h : &tmA0h) : (shared ? &tmA1 : &tmA0);
         const CUtensorMap* mB = shared ? &tmB1 : &tmB0;
-        const int a_row = t.a_row + (int)rank * 128;
-        const int b_row = (MODE == 0) ? t.b_row + (int)rank * p.f : t.b_row + (int)rank * 128;
+        const int a_row = t.a_row + (int)rank * (t.half ? 64 : 128);
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, p.timeout_ns, s_abort)) {
             abort = true;
             break;
           }
-          const bool stall = p.stall_first_stage && L == pair && kb == 0;
+          const bool stall = p.stall_first_stage && first && kb == 0;
           if (leader) {
-            mbar_arrive_expect_tx(&ctl->full[stage], C::STAGE_TX);
+            mbar_arrive_expect_tx(&ctl->full[stage], t.half ? C::STAGE_TX_HALF : C::STAGE_TX);
             armed[stage] = !stall;
             armed_phase[stage] = phase;
           }
@@ -780,12 +1026,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t full_leader = mapa_shared(smem_u32(&ctl->full[stage]), 0);
           tma_load_2d_pair(sA + stage * HALF_TILE, mA, full_leader, kb * BK, a_row);
-          tma_load_2d_pair(sB + stage * HALF_TILE, mB, full_leader, kb * BK, b_row);
+          if (MODE == 0) {
+            /* 64 gate rows, then the matching 64 up rows */
+            const int g_row = t.b_row + (int)rank * 64;
+            tma_load_2d_pair(sB + stage * HALF_TILE, mB, full_leader, kb * BK, g_row);
+            tma_load_2d_pair(sB + stage * HALF_TILE + HALF_TILE / 2, mB, full_leader, kb * BK, g_row + p.f);
+          } else {
+            tma_load_2d_pair(sB + stage * HALF_TILE, mB, full_leader, kb * BK, t.b_row + (int)rank * 128);
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
+        if (abort) break;
+        first = false;
       }
       if (!abort) {
         /* wait until the MMAs have released every stage this CTA filled, so no
@@ -816,7 +1071,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       uint32_t acc = 0;
       bool abort = false;
-      for (int64_t L = pair; L < total && !abort; L += npairs, ++acc) {
+      for (int i = 0;; ++i, ++acc) {
+        int v;
+        if (!read_tile_index<true>(ctl, i, p.timeout_ns, s_abort, &v)) {
+          abort = true;
+          break;
+        }
+        release_slot(i);
+        if (v < 0) break;
+        const Tile t = decode_tile<MODE, 256, 256>(v, p, ctl->off, ctl->mpref, ctl->hpref);
+        const uint32_t idesc = t.half ? C::IDESC_HALF : C::IDESC;
         const uint32_t b = acc & 1u, use = (acc >> 1) & 1u;
         if (!mbar_wait(&ctl->tempty[b], use ^ 1u, p.timeout_ns, s_abort)) {
           abort = true;
@@ -834,7 +1098,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b_addr = smem_u32(sB + stage * HALF_TILE);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            umma_bf16_pair(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32), C::IDESC,
+            umma_bf16_pair(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32), idesc,
                            (kb | kk) != 0 ? 1u : 0u);
           }
           umma_commit_pair_mc(&ctl->empty[stage], 0x3);
@@ -867,8 +1131,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     /* ---------------- epilogue (warps 2..5 of both CTAs) ---------------- */
     const int q = warp & 3;
     uint32_t acc = 0;
-    for (int64_t L = pair; L < total; L += npairs, ++acc) {
-      const Tile t = decode_tile<MODE, 256, 256>(L, p, ctl->off, ctl->mpref, ctl->hpref);
+    for (int i = 0;; ++i, ++acc) {
+      int v = -1;
+      const bool got = read_tile_index<true>(ctl, i, p.timeout_ns, s_abort, &v);
+      __syncwarp();
+      if (!got) {
+        if (lane == 0) {
+          raise_status(p.status, MOE_DEV_TIMEOUT);
+          *s_abort = 1;
+        }
+        break;
+      }
+      if (lane == 0) release_slot(i);
+      if (v < 0) break;
+      const Tile t = decode_tile<MODE, 256, 256>(v, p, ctl->off, ctl->mpref, ctl->hpref);
       const uint32_t b = acc & 1u, use = (acc >> 1) & 1u;
       if (!mbar_wait(&ctl->tfull[b], use, p.timeout_ns, s_abort)) {
         if (lane == 0) {
@@ -878,8 +1154,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      epilogue_warp<MODE, 256>(p, t, tmem_base + ((uint32_t)(q * 32) << 16) + b * C::ACC_COLS,
-                               (int)rank * 128 + q * 32, lane, sEpi + q * kStageBytesPerWarp, &tmO0, &tmO1);
+      epilogue_pair_warp<MODE>(p, t, tmem_base + ((uint32_t)(q * 32) << 16) + b * C::ACC_COLS, q, rank, lane,
+                               sEpi + q * kStageBytesPerWarp, &tmO0, &tmO1);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&ctl->tempty[b]), 0));
@@ -894,6 +1170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
   }
+  if (threadIdx.x == 0) release_tile_counter(p);
 }
 
 /* ---- host side ------------------------------------------------------------ */
@@ -979,9 +1256,9 @@ int pair_clusters() {
 }
 
 template <int MODE>
-cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0, const CUtensorMap& b1,
-                        const CUtensorMap& o0, const CUtensorMap& o1, const FfnParams& p, cudaStream_t stream,
-                        bool* launched) {
+cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a0h, const CUtensorMap& a1h,
+                        const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& o0, const CUtensorMap& o1,
+                        const FfnParams& p, cudaStream_t stream, bool* launched) {
   *launched = false;
   static std::atomic<int> attr_done[kMaxDevices];
   const cudaError_t attr_err = smem_opt_in(attr_done, ffn_gemm_pair_kernel<MODE>, PairCfg::SMEM_BYTES);
@@ -990,18 +1267,13 @@ cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   if (debug_log()) std::fprintf(stderr, "[moe] pair GEMM%d: %d resident clusters of 2 CTAs\n", MODE + 1, clusters);
   if (clusters <= 0) return cudaSuccess; /* caller falls back to single-CTA tiles */
   const cudaError_t e = launch_kernel(ffn_gemm_pair_kernel<MODE>, dim3(2 * (unsigned)clusters), dim3(kThreads),
-                                     PairCfg::SMEM_BYTES, stream, 2, a0, a1, b0, b1, o0, o1, p);
+                                     PairCfg::SMEM_BYTES, stream, 2, a0, a1, a0h, a1h, b0, b1, o0, o1, p);
   if (e == cudaSuccess) *launched = true;
   return e;
 }
 
-/* Split schedule (CTA-pair tiles for whole 256-row blocks, single-CTA tiles for
- * last blocks of <= 128 rows) on request only: its tail launch streams the weights
- * of every expert with a short last block from DRAM a second time, which cost more
- * than the padding it saves on every workload measured. */
-bool split_tiles(int pol) { return pol == kGemmSplit; }
-
-FfnParams base_params(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const int32_t* expert_offsets) {
+FfnParams base_params(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const int32_t* expert_offsets,
+                      size_t ctr_offset) {
   FfnParams p;
   p.expert_offsets = expert_offsets;
   p.E = s.E;
@@ -1013,10 +1285,15 @@ FfnParams base_params(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, cons
   p.status = reinterpret_cast<uint32_t*>(ws + L.status);
   p.timeout_ns = wait_timeout_ns();
   p.stall_first_stage = test_stall() ? 1 : 0;
-  p.part = kPartAll;
+  p.tile_ctr = reinterpret_cast<uint32_t*>(ws + L.status + ctr_offset);
   p.row_src = nullptr;
   p.gather_x = nullptr;
   p.k = s.k;
+  p.fc_row_src = nullptr;
+  p.fc_assign_row = nullptr;
+  p.fc_gate = nullptr;
+  p.fc_out = nullptr;
+  p.fc_cnt = nullptr;
   return p;
 }
 
@@ -1028,26 +1305,22 @@ cudaError_t launch_gate_up(const moe_shape_t& s, const WsLayout& L, uint8_t* ws,
   if (s.T == 0) return cudaSuccess;
   const bool sh = s.n_shared != 0;
   const bool gather = x_perm == nullptr; /* A rows gathered from x through row_src */
-  /* 128-row single-CTA tiles pad small experts less and measured faster for this GEMM's
-   * short K; CTA-pair tiles only on request (and never when gathering) */
+  /* 128-row single-CTA tiles by default (measured faster for this GEMM's short K);
+   * CTA-pair tiles on request (never when gathering) */
   const int pol = gather ? kGemmSingle : gemm_policy();
-  const bool split = split_tiles(pol);
-  const bool pair = split || pol == kGemmPair;
-  CUtensorMap a0, a1, b0, b1;
+  const bool pair = pol == kGemmPair;
   /* A = x_perm [A, d] (routed; rows of x gathered by the producer warp instead when x_perm is
-   * null) / x [T, d] (shared);
-   * B = w13 [E*2f, d] / w13s [2f, d] */
+   * null) / x [T, d] (shared); B = w13 [E*2f, d] / w13s [2f, d] */
   if (gather && (uint64_t)s.T * (uint64_t)s.d * 2u > 0xFFFFFFFFull) return cudaErrorInvalidValue;
-  if (!make_map(&a0, gather ? x : x_perm, gather ? (uint64_t)s.T : (uint64_t)L.A, s.d, 128))
-    return cudaErrorInvalidValue;
-  if (!make_map(&a1, sh || gather ? x : x_perm, sh || gather ? (uint64_t)s.T : (uint64_t)L.A, s.d, 128))
-    return cudaErrorInvalidValue;
-  if (!make_map(&b0, w13, (uint64_t)s.E * 2 * s.f, s.d, 128)) return cudaErrorInvalidValue;
-  if (!make_map(&b1, sh ? w13s : w13, sh ? (uint64_t)2 * s.f : (uint64_t)s.E * 2 * s.f, s.d, 128))
-    return cudaErrorInvalidValue;
+  const uint16_t* a_routed = gather ? x : x_perm;
+  const uint64_t a_rows = gather ? (uint64_t)s.T : (uint64_t)L.A;
+  const uint16_t* a_sh = sh || gather ? x : x_perm;
+  const uint64_t a_sh_rows = sh || gather ? (uint64_t)s.T : (uint64_t)L.A;
+  const uint16_t* b_sh = sh ? w13s : w13;
+  const uint64_t b_rows = (uint64_t)s.E * 2 * s.f, b_sh_rows = sh ? (uint64_t)2 * s.f : b_rows;
   CUtensorMap o0; /* h [h_rows, f], stored as 32 x 64 blocks */
   if (!make_map(&o0, ws + L.h, (uint64_t)L.h_rows, s.f, 32)) return cudaErrorInvalidValue;
-  FfnParams p = base_params(s, L, ws, expert_offsets);
+  FfnParams p = base_params(s, L, ws, expert_offsets, kGemm1CtrOffset);
   p.K = s.d;
   p.n_tiles_n = s.f / 128;
   p.out0 = reinterpret_cast<uint16_t*>(ws + L.h);
@@ -1055,55 +1328,68 @@ cudaError_t launch_gate_up(const moe_shape_t& s, const WsLayout& L, uint8_t* ws,
   p.ld_out = s.f;
   p.row_src = gather ? row_src : nullptr;
   p.gather_x = gather ? x : nullptr;
+  CUtensorMap a0, a1, b0, b1;
+  if (!make_map(&a0, a_routed, a_rows, s.d, 128) || !make_map(&a1, a_sh, a_sh_rows, s.d, 128))
+    return cudaErrorInvalidValue;
   if (pair) {
+    /* each CTA of a pair stages 64 gate and 64 up rows (64-row B boxes) and, in a
+     * half-height tile, 64 rows of A (64-row A boxes) */
+    CUtensorMap a0h, a1h;
+    if (!make_map(&a0h, a_routed, a_rows, s.d, 64) || !make_map(&a1h, a_sh, a_sh_rows, s.d, 64) ||
+        !make_map(&b0, w13, b_rows, s.d, 64) || !make_map(&b1, b_sh, b_sh_rows, s.d, 64))
+      return cudaErrorInvalidValue;
     bool launched = false;
-    p.part = split ? kPartPair : kPartAll;
-    const cudaError_t e = launch_pair<0>(a0, a1, b0, b1, o0, o0, p, stream, &launched);
-    if (e != cudaSuccess || (launched && !split)) return e;
-    p.part = launched ? kPartTail : kPartAll;
+    const cudaError_t e = launch_pair<0>(a0, a1, a0h, a1h, b0, b1, o0, o0, p, stream, &launched);
+    if (e != cudaSuccess || launched) return e;
   }
+  if (!make_map(&b0, w13, b_rows, s.d, 128) || !make_map(&b1, b_sh, b_sh_rows, s.d, 128))
+    return cudaErrorInvalidValue;
   return gather ? launch_single<0, 256, true>(a0, a1, b0, b1, o0, o0, p, stream)
                 : launch_single<0, 256>(a0, a1, b0, b1, o0, o0, p, stream);
 }
 
 cudaError_t launch_down(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const int32_t* expert_offsets,
                         const uint16_t* w2, const uint16_t* w2s, uint16_t* y_perm, uint16_t* y_shared,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, const FusedCombine* fc) {
   if (s.T == 0) return cudaSuccess;
   const bool sh = s.n_shared != 0;
   const bool bn256 = (s.d % 256) == 0;
   /* CTA-pair tiles (256 output columns per tile) when every expert averages >= 1024
-   * rows, so that 256-row padding stays small */
+   * rows, or on request */
   const int pol = bn256 ? gemm_policy() : kGemmSingle;
-  const bool split = split_tiles(pol);
-  const bool pair = split || pol == kGemmPair || (pol == kGemmAuto && L.A >= (int64_t)1024 * s.E);
+  const bool pair = pol == kGemmPair || (pol == kGemmAuto && L.A >= (int64_t)1024 * s.E);
   const uint32_t bn = bn256 ? 256 : 128;
-  const uint32_t b_box = pair ? 128 : bn;
-  CUtensorMap a0, b0, b1;
+  const uint16_t* b_sh = sh ? w2s : w2;
+  const uint64_t b_rows = (uint64_t)s.E * s.d, b_sh_rows = sh ? (uint64_t)s.d : b_rows;
   /* A = h [h_rows, f] (workspace); B = w2 [E*d, f] / w2s [d, f] */
+  CUtensorMap a0, b0, b1;
   if (!make_map(&a0, ws + L.h, (uint64_t)L.h_rows, s.f, 128)) return cudaErrorInvalidValue;
-  if (!make_map(&b0, w2, (uint64_t)s.E * s.d, s.f, b_box)) return cudaErrorInvalidValue;
-  if (!make_map(&b1, sh ? w2s : w2, sh ? (uint64_t)s.d : (uint64_t)s.E * s.d, s.f, b_box))
-    return cudaErrorInvalidValue;
   CUtensorMap o0, o1; /* y_perm [A, d] and y_shared [T, d], stored as 32 x 64 blocks */
   if (!make_map(&o0, y_perm, (uint64_t)L.A, s.d, 32)) return cudaErrorInvalidValue;
   if (!make_map(&o1, sh ? y_shared : y_perm, sh ? (uint64_t)s.T : (uint64_t)L.A, s.d, 32)) return cudaErrorInvalidValue;
-  FfnParams p = base_params(s, L, ws, expert_offsets);
+  FfnParams p = base_params(s, L, ws, expert_offsets, kGemm2CtrOffset);
   p.K = s.f;
   p.n_tiles_n = s.d / (int)bn;
   p.out0 = y_perm;
   p.out1 = sh ? y_shared : nullptr;
   p.ld_out = s.d;
-  if (pair) {
-    bool launched = false;
-    p.part = split ? kPartPair : kPartAll;
-    const cudaError_t e = launch_pair<1>(a0, a0, b0, b1, o0, o1, p, stream, &launched);
-    if (e != cudaSuccess || (launched && !split)) return e;
-    p.part = launched ? kPartTail : kPartAll;
-    if (!make_map(&b0, w2, (uint64_t)s.E * s.d, s.f, bn)) return cudaErrorInvalidValue;
-    if (!make_map(&b1, sh ? w2s : w2, sh ? (uint64_t)s.d : (uint64_t)s.E * s.d, s.f, bn))
-      return cudaErrorInvalidValue;
+  if (fc) {
+    p.fc_row_src = fc->row_src;
+    p.fc_assign_row = fc->assign_row;
+    p.fc_gate = fc->topk_gate;
+    p.fc_out = fc->out;
+    p.fc_cnt = reinterpret_cast<uint32_t*>(ws + L.fc_cnt);
   }
+  if (pair) {
+    CUtensorMap a0h;
+    if (!make_map(&a0h, ws + L.h, (uint64_t)L.h_rows, s.f, 64) || !make_map(&b0, w2, b_rows, s.f, 128) ||
+        !make_map(&b1, b_sh, b_sh_rows, s.f, 128))
+      return cudaErrorInvalidValue;
+    bool launched = false;
+    const cudaError_t e = launch_pair<1>(a0, a0, a0h, a0h, b0, b1, o0, o1, p, stream, &launched);
+    if (e != cudaSuccess || launched) return e;
+  }
+  if (!make_map(&b0, w2, b_rows, s.f, bn) || !make_map(&b1, b_sh, b_sh_rows, s.f, bn)) return cudaErrorInvalidValue;
   return bn256 ? launch_single<1, 256>(a0, a0, b0, b1, o0, o1, p, stream)
                : launch_single<1, 128>(a0, a0, b0, b1, o0, o1, p, stream);
 }

@@ -32,6 +32,7 @@ std::atomic<uint64_t> g_wait_timeout_ns{kDefaultWaitNs};
 std::atomic<int> g_gemm_policy{kGemmAuto};
 std::atomic<int> g_test_stall{0};
 std::atomic<int> g_pdl{1};
+std::atomic<int> g_fused_combine{0};
 
 }  // namespace
 
@@ -86,6 +87,11 @@ WsLayout ws_layout(const moe_shape_t& s) {
   off = round_up(off + (size_t)L.n_chunks * s.E * sizeof(int32_t), 256);
   L.local_rank = off;
   off = round_up(off + (size_t)L.A * sizeof(int32_t), 256);
+  L.dispatch_end = off;
+  L.ep = off; /* row_base[256], keep[256], offsets[257], rank counts[256], rank offsets[257], imbalance[2] */
+  off = round_up(off + (size_t)(6 * kMaxE + 4) * sizeof(int32_t), 256);
+  L.fc_cnt = off;
+  off = round_up(off + (size_t)s.T * (size_t)(s.d / 64) * sizeof(uint32_t), 256);
   L.h = off;
   off = round_up(off + (size_t)L.h_rows * s.f * sizeof(uint16_t), 256);
   L.total = off;
@@ -112,6 +118,8 @@ int gemm_policy() { return g_gemm_policy.load(std::memory_order_relaxed); }
 bool test_stall() { return g_test_stall.load(std::memory_order_relaxed) != 0; }
 
 bool pdl_enabled() { return g_pdl.load(std::memory_order_relaxed) != 0; }
+
+bool fused_combine_enabled() { return g_fused_combine.load(std::memory_order_relaxed) != 0; }
 
 bool debug_log() {
   static const bool on = [] {
@@ -291,16 +299,20 @@ moe_status_t moe_layer(const moe_shape_t* shape, const moe_layer_buffers_t* b, v
   uint32_t* status = reinterpret_cast<uint32_t*>(w + L.status);
   cudaError_t e = launch_route(b->logits, b->topk_idx, b->topk_gate, shape->T, shape->E, shape->k, status, s);
   if (e != cudaSuccess) return cuda_fail(e);
+  const bool fused = fused_combine_enabled();
   e = launch_dispatch(*shape, L, w, b->x, b->topk_idx, b->expert_counts, b->expert_offsets, b->rank_counts,
-                      b->rank_offsets, b->row_src, b->assign_row, b->x_perm, b->imbalance, s);
+                      b->rank_offsets, b->row_src, b->assign_row, b->x_perm, b->imbalance, s,
+                      fused ? b->out : nullptr);
   if (e != cudaSuccess) return cuda_fail(e);
   const uint16_t* ysh_in = shape->n_shared ? b->y_shared : nullptr;
   /* x_perm null: dispatch writes indices only and GEMM1 gathers the rows of x itself */
   e = launch_gate_up(*shape, L, w, b->x_perm, b->row_src, b->expert_offsets, b->w13, b->x, b->w13s, s);
   if (e != cudaSuccess) return cuda_fail(e);
+  const FusedCombine fc{b->row_src, b->assign_row, b->topk_gate, b->out};
   e = launch_down(*shape, L, w, b->expert_offsets, b->w2, b->w2s, b->y_perm, shape->n_shared ? b->y_shared : nullptr,
-                  s);
+                  s, fused ? &fc : nullptr);
   if (e != cudaSuccess) return cuda_fail(e);
+  if (fused) return MOE_OK; /* out was written by the down GEMM's epilogue */
   /* combine's predecessor is the down GEMM: assign_row and topk_gate come from earlier kernels */
   e = launch_combine(*shape, b->y_perm, b->assign_row, b->topk_gate, ysh_in, b->out, status, s, true);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e);
@@ -329,8 +341,40 @@ int32_t moe_capacity_for(int64_t c_num, int64_t c_den, int32_t T, int32_t k, int
 }
 
 int moe_set_gemm_policy(int policy) {
-  if (policy != kGemmAuto && policy != kGemmSingle && policy != kGemmPair && policy != kGemmSplit) return -1;
+  if (policy != kGemmAuto && policy != kGemmSingle && policy != kGemmPair) return -1;
   return g_gemm_policy.exchange(policy, std::memory_order_relaxed);
+}
+
+int moe_set_fused_combine(int enable) {
+  return g_fused_combine.exchange(enable ? 1 : 0, std::memory_order_relaxed);
+}
+
+moe_status_t moe_expert_down_combine(const moe_shape_t* shape, const int32_t* expert_offsets, const moe_bf16_t* w2,
+                                     const moe_bf16_t* w2s, const int32_t* row_src, const int32_t* assign_row,
+                                     const float* topk_gate, moe_bf16_t* y_perm, moe_bf16_t* y_shared,
+                                     moe_bf16_t* out, void* ws, size_t ws_bytes, void* stream) {
+  const NvtxRange nvtx_range("moe_expert_down_combine");
+  moe_status_t st = validate_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!expert_offsets || !w2 || !aligned(w2, 16)) return MOE_ERR_INVALID_ARG;
+  if (shape->T > 0 && (!y_perm || !aligned(y_perm, 16) || !row_src || !assign_row || !topk_gate || !out ||
+                       !aligned(out, 16)))
+    return MOE_ERR_INVALID_ARG;
+  if (shape->n_shared && shape->T > 0 && (!w2s || !y_shared || !aligned(w2s, 16) || !aligned(y_shared, 16)))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(*shape, ws, ws_bytes)) != MOE_OK) return st;
+  if (shape->T == 0) return MOE_OK;
+  const WsLayout L = ws_layout(*shape);
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* w = (uint8_t*)ws;
+  cudaError_t e = cudaMemsetAsync(w + L.fc_cnt, 0, (size_t)shape->T * (shape->d / 64) * sizeof(uint32_t), s);
+  /* with a capacity and no shared expert a token may get no row at all: its output is zero */
+  if (e == cudaSuccess && shape->capacity > 0 && !shape->n_shared)
+    e = cudaMemsetAsync(out, 0, (size_t)shape->T * shape->d * sizeof(uint16_t), s);
+  const FusedCombine fc{row_src, assign_row, topk_gate, out};
+  if (e == cudaSuccess)
+    e = launch_down(*shape, L, w, expert_offsets, w2, w2s, y_perm, shape->n_shared ? y_shared : nullptr, s, &fc);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }
 
 int moe_set_pdl(int enable) { return g_pdl.exchange(enable ? 1 : 0, std::memory_order_relaxed); }

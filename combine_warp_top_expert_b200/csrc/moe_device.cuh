@@ -111,15 +111,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+/* try_wait with acquire at cluster scope: for a phase completed by arrivals from
+ * the peer CTA of a pair whose earlier writes (to either CTA's shared memory) this
+ * thread then reads, or whose earlier reads must precede this thread's writes. */
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 /* Bounded wait for the phase with the given parity to complete. Returns false
  * once `timeout_ns` has passed since the wait began, or as soon as another role
- * of the CTA has raised `abort_flag` (may be null). */
+ * of the CTA has raised `abort_flag` (may be null). CLUSTER: acquire at cluster
+ * scope (see mbar_try_wait_cluster). */
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns,
                                           volatile int* abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto try_wait = [&]() { return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  if (try_wait()) return true;
   uint64_t t0 = 0;
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (try_wait()) return true;
     if ((it & 63u) == 0u) {
       if (abort_flag && *abort_flag) return false;
       const uint64_t now = global_ns();
@@ -174,6 +192,12 @@ __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bu
 
 /* Wait until the issuing thread's bulk stores are complete. */
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+/* Order this thread's async-proxy accesses of global memory (completed TMA stores)
+ * with its later generic-proxy accesses. */
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 
 /* Make this thread's generic-proxy shared-memory writes visible to the async proxy (TMA). */
 __device__ __forceinline__ void fence_proxy_async_shared() {
@@ -254,6 +278,11 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t local_addr, uint32_t ra
 /* Arrive on an mbarrier given by its shared::cluster address (own or peer CTA). */
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+/* 32-bit store to a shared::cluster address (own or peer CTA). */
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 
 /* All threads of both CTAs of the cluster. */

@@ -25,8 +25,10 @@
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Every call
  *    is asynchronous on that stream, except moe_get_status which synchronises it.
  *  - `ws` is a caller-owned device workspace of at least moe_workspace_bytes()
- *    bytes, 256-byte aligned. Its first 256 bytes hold the device status word;
- *    clear it once with moe_clear_status before first use. The library
+ *    bytes, 256-byte aligned. Its first 256 bytes hold the device status word
+ *    and the counters the kernels use across CTAs (each kernel leaves its
+ *    counters at zero when it finishes); clear them once with moe_clear_status
+ *    (or allocate the workspace zeroed) before first use. The library
  *    allocates nothing and keeps no per-call state outside `ws`.
  *  - Shapes are validated on the host before anything is launched; an invalid
  *    argument returns MOE_ERR_INVALID_ARG (or MOE_ERR_UNSUPPORTED for a shape
@@ -223,6 +225,23 @@ moe_status_t moe_expert_gate_up_gather(const moe_shape_t* shape, const moe_bf16_
                                        const int32_t* expert_offsets, const moe_bf16_t* w13, const moe_bf16_t* w13s,
                                        void* ws, size_t ws_bytes, void* stream);
 
+/* moe_expert_down with the combine folded into its epilogue: the per-expert overlap
+ * of the page "Balancing and Beyond: Communication-Centric Optimizations in Expert
+ * Parallelism" (key idea: compute and combine pipelined along the experts), on one
+ * GPU. Each output tile, once stored, counts its rows in on their tokens' counters
+ * (one per token and 64 columns); the row that completes a token's count (its kept
+ * assignments, plus its shared row) sums that token's rows of those 64 columns in j
+ * order, as moe_combine does: out is bit for bit moe_combine's, whatever order the
+ * tiles finish in. y_perm (and y_shared) are written as by moe_expert_down.
+ *   row_src, assign_row [T*k] int32 in, topk_gate [T, k] fp32 in (from dispatch and
+ *   route); out [T, d] bf16 out. The counters live in the workspace; this call zeroes
+ *   them first (and out, when a capacity can leave a token with no row and there is
+ *   no shared expert). Other arguments as moe_expert_down. */
+moe_status_t moe_expert_down_combine(const moe_shape_t* shape, const int32_t* expert_offsets, const moe_bf16_t* w2,
+                                     const moe_bf16_t* w2s, const int32_t* row_src, const int32_t* assign_row,
+                                     const float* topk_gate, moe_bf16_t* y_perm, moe_bf16_t* y_shared,
+                                     moe_bf16_t* out, void* ws, size_t ws_bytes, void* stream);
+
 /* Combine: un-permute and gate-weighted sum, back in original token order.
  * Page "Expert Parallelism" §4 COMBINE.
  *   out[t] = sum_{j<k} topk_gate[t,j] * y_perm[assign_row[t*k+j]] (+ y_shared[t])
@@ -263,6 +282,98 @@ typedef struct moe_layer_buffers {
 moe_status_t moe_layer(const moe_shape_t* shape, const moe_layer_buffers_t* buf, void* ws, size_t ws_bytes,
                        void* stream);
 
+/* ---- Expert parallelism across GPUs ------------------------------------------
+ * Page "Expert Parallelism" §1 (experts on GPUs in contiguous blocks: rank r of R
+ * owns experts [r*E/R, (r+1)*E/R)) and §4 "The All-to-All": DISPATCH counts the
+ * tokens per GPU, exchanges the counts, then the token rows, so that every GPU
+ * holds one contiguous run of rows per expert it owns; COMPUTE runs each GPU's
+ * experts as one grouped GEMM; COMBINE returns every result to the GPU its token
+ * came from, in the original order, and sums it with its gate; §4 "The
+ * communication volume": k * d * 2 bytes per token and direction.
+ * One process (or host thread) per GPU, R ranks, each with its own batch of T
+ * tokens (shape->T), all E experts' router logits, and the weights of its own
+ * E/R experts. shape->R is the number of ranks; shape->capacity, if non-zero,
+ * applies to every expert's rows from all ranks together.
+ * The exchanges are done by the kernels themselves over peer memory (NVLink): the
+ * dispatch permute stores each row into the owning rank's receive buffer, the
+ * combine loads each result row from the owning rank's output buffer, and the
+ * per-expert counts are stored into every rank's count table. Each rank's receive
+ * buffer then holds exactly the rows that a single-GPU moe_dispatch of the R
+ * batches taken as one batch (rank after rank) places in logical rank r's slice,
+ * in the same order.
+ * Ranks signal each step through flags in peer memory (release and acquire at
+ * system scope); a wait that runs out (moe_set_wait_timeout_ns) raises
+ * MOE_DEV_TIMEOUT and returns. `epoch` numbers the layer calls, 1, 2, 3, ...,
+ * the same on every rank. One layer call on rank r, all on one stream:
+ *   moe_route                  (local)
+ *   moe_ep_exchange_counts     histogram, counts to every rank
+ *   moe_ep_dispatch            wait for all counts, plan, rows to their owners
+ *   moe_ep_wait(slot 1)        every rank's rows have arrived
+ *   moe_expert_ffn             on the receive buffer: shape (T = rows_cap, k = 1,
+ *                              E = E/R, R = 1, d, f), expert_offsets =
+ *                              recv_offsets, this rank's weights, y = its output
+ *                              buffer (+ a shared expert on the local x, if any)
+ *   moe_ep_signal(slot 2)      this rank's expert outputs are ready
+ *   moe_ep_combine             wait for every rank's outputs, gather and sum
+ *   moe_ep_wait(slot 3)        every rank has read the outputs: the buffers may
+ *                              be written by the next call */
+typedef struct moe_ep_peers {
+  int32_t* const* counts;       /* [R] device array of device pointers: rank r's count table, int32 [R][E] */
+  moe_bf16_t* const* recv_rows; /* [R] ...: rank r's receive buffer, bf16 [rows_cap][d] */
+  moe_bf16_t* const* y_rows;    /* [R] ...: rank r's expert-output buffer, bf16 [rows_cap][d] */
+  uint64_t* const* flags;       /* [R] ...: rank r's flags, uint64 [4][R], zero before the first call */
+  int64_t rows_cap;             /* rows of every receive and output buffer; R * T * k holds any routing */
+} moe_ep_peers_t;
+
+#define MOE_EP_SLOT_COUNTS 0  /* a rank's counts are in every table */
+#define MOE_EP_SLOT_ROWS 1    /* a rank's rows are in their owners' receive buffers */
+#define MOE_EP_SLOT_OUTPUTS 2 /* a rank's expert outputs are ready to be read */
+#define MOE_EP_SLOT_DONE 3    /* a rank has read every output it needs */
+
+/* Per-expert histogram of this rank's topk_idx (T*k assignments, no capacity):
+ * expert_counts [E] out (device); stores the row into every rank's count table and
+ * signals MOE_EP_SLOT_COUNTS. ws: a workspace for `shape` (moe_workspace_bytes). */
+moe_status_t moe_ep_exchange_counts(const moe_shape_t* shape, int32_t rank, uint64_t epoch, const int32_t* topk_idx,
+                                    int32_t* expert_counts, const moe_ep_peers_t* peers, void* ws, size_t ws_bytes,
+                                    void* stream);
+
+/* Waits for every rank's counts, computes the plan (moe_ep_plan_host is the same
+ * arithmetic on the host) and stores each row of x into its owner's receive buffer;
+ * signals MOE_EP_SLOT_ROWS.
+ *   send_row     [T*k] int32 out: row of assignment a in its owner's buffers (-1: dropped)
+ *   recv_offsets [E/R + 1] int32 out: this rank's experts' rows in its own receive
+ *                buffer, [E/R] = rows received (the expert_offsets of its expert FFN)
+ * ws must be the workspace of the preceding moe_ep_exchange_counts. */
+moe_status_t moe_ep_dispatch(const moe_shape_t* shape, int32_t rank, uint64_t epoch, const moe_bf16_t* x,
+                             const int32_t* topk_idx, int32_t* send_row, int32_t* recv_offsets,
+                             const moe_ep_peers_t* peers, void* ws, size_t ws_bytes, void* stream);
+
+/* Store epoch into flag `slot` of this rank in every rank's flags (after this
+ * stream's earlier work). */
+moe_status_t moe_ep_signal(int32_t R, int32_t rank, int32_t slot, uint64_t epoch, const moe_ep_peers_t* peers,
+                           void* stream);
+
+/* Wait (bounded) on the stream until every rank's flag `slot` has reached epoch;
+ * on timeout raises MOE_DEV_TIMEOUT in ws's status word. */
+moe_status_t moe_ep_wait(int32_t R, int32_t rank, int32_t slot, uint64_t epoch, const moe_ep_peers_t* peers, void* ws,
+                         size_t ws_bytes, void* stream);
+
+/* Waits for every rank's expert outputs, then
+ *   out[t] = sum_j topk_gate[t, j] * y_rows[owner(topk_idx[t, j])][send_row[t*k + j]] (+ y_shared[t])
+ * (fp32 in j order, one bf16 rounding; a dropped assignment adds nothing), and
+ * signals MOE_EP_SLOT_DONE. y_shared [T, d] may be NULL. */
+moe_status_t moe_ep_combine(const moe_shape_t* shape, int32_t rank, uint64_t epoch, const int32_t* send_row,
+                            const int32_t* topk_idx, const float* topk_gate, const moe_bf16_t* y_shared,
+                            moe_bf16_t* out, const moe_ep_peers_t* peers, void* ws, size_t ws_bytes, void* stream);
+
+/* The exchange plan on the host, from all ranks' counts (host int32 [R][E]):
+ *   row_base[e]  first row, in the owner of e's receive buffer, of `rank`'s rows of e
+ *   keep[e]      how many of `rank`'s assignments to e are kept (capacity)
+ *   recv_offsets [E/R + 1] this rank's experts' rows in its receive buffer
+ * Returns 0, or -1 for invalid arguments. */
+int32_t moe_ep_plan_host(int32_t R, int32_t E, int32_t rank, int32_t capacity, const int32_t* counts_all,
+                         int32_t* row_base, int32_t* keep, int32_t* recv_offsets);
+
 /* Human-readable name of a status code (static string). */
 const char* moe_status_string(moe_status_t status);
 
@@ -280,19 +391,23 @@ uint64_t moe_set_wait_timeout_ns(uint64_t ns);
 /* Diagnostic knob: tile shape of the grouped GEMM for launches made after the
  * call, process-wide. Two tile shapes exist: 128 x 256 tiles of one CTA, and
  * 256 x 256 tiles computed by a cluster of two CTAs on neighbouring SMs
- * (cta_group::2; the down GEMM needs d % 256 == 0 for them).
+ * (cta_group::2; the down GEMM needs d % 256 == 0 for them), where a group's last
+ * block of at most 128 rows runs as a half-height tile (128 x 256, 64 rows per
+ * CTA), so both shapes pad a group to a multiple of 128 rows.
  *   0 (default) = single-CTA tiles, except CTA-pair tiles for the down GEMM
  *       when the routed experts average at least 1024 rows (T*k >= 1024*E);
  *   1 = single-CTA tiles only;
- *   2 = CTA-pair tiles wherever they apply (every group padded to 256 rows);
- *   3 = split: each group's whole 256-row blocks, and a last block of more than
- *       128 rows, as CTA-pair tiles; a last block of 1..128 rows as one
- *       single-CTA tile in a second launch (padding as with single tiles, but
- *       the second launch reads those experts' weights again: slower on the
- *       workloads measured).
- * Results are the same up to fp32 summation order. Returns the previous value,
- * or -1 for an unknown policy (unchanged). */
+ *   2 = CTA-pair tiles wherever they apply.
+ * Either way the CTAs claim tiles at run time from a counter in the workspace
+ * header (zero between calls). Results are the same up to fp32 summation order.
+ * Returns the previous value, or -1 for an unknown policy (unchanged). */
 int moe_set_gemm_policy(int policy);
+
+/* Whole-layer knob: while enabled (non-zero), moe_layer folds the combine into the
+ * down GEMM's epilogue (as moe_expert_down_combine; its dispatch zeroes the counters)
+ * instead of launching moe_combine's kernel. Results are bit for bit the same.
+ * Process-wide, for calls made after this one; default 0. Returns the previous value. */
+int moe_set_fused_combine(int enable);
 
 /* Launch-overlap knob: while enabled (the default, non-zero), every kernel the
  * library launches carries programmatic stream serialization (programmatic

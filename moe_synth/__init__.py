@@ -258,6 +258,32 @@ def device_inputs(wl: Workload, device="cuda", weights: bool = True) -> dict:
     return out
 
 
+def device_expert_weights(wl: Workload, e0: int, e1: int, device="cuda") -> dict:
+    """w13 [e1-e0, 2f, d] and w2 [e1-e0, d, f] of experts e0..e1-1 (and the shared expert's, if any),
+    filled on the device with the same values as the full tensors' rows (expert parallelism:
+    every rank holds its own experts only)."""
+    import torch
+    L = lib()
+    stream = torch.cuda.current_stream(device).cuda_stream
+    out = {}
+
+    def bf16(shape, tid, offset):
+        t = torch.empty(shape, dtype=torch.bfloat16, device=device)
+        if t.numel():
+            assert L.synth_fill_normal_bf16_device(t.data_ptr(), t.numel(), wl.seed, tid, offset, float(_c_w()),
+                                                   stream) == 0
+        return t
+
+    n = e1 - e0
+    out["w13"] = bf16((n, 2 * wl.f, wl.d), W13, e0 * 2 * wl.f * wl.d)
+    out["w2"] = bf16((n, wl.d, wl.f), W2, e0 * wl.d * wl.f)
+    if wl.n_shared:
+        out["w13s"] = bf16((2 * wl.f, wl.d), W13S, 0)
+        out["w2s"] = bf16((wl.d, wl.f), W2S, 0)
+    torch.cuda.synchronize(device)
+    return out
+
+
 def bf16_to_f32(a: np.ndarray) -> np.ndarray:
     """Exact upcast of bf16 bit patterns."""
     return (a.astype(np.uint32) << 16).view(np.float32)

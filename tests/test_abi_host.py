@@ -38,7 +38,10 @@ def test_workspace_bytes_layout():
     A = TINY.T * TINY.k
     chunks = -(-TINY.T // (2048 // TINY.k))
     h_rows = 256 * (A // 256 + min(TINY.E, A))
-    expect = 256 + (-(-chunks * TINY.E * 4 // 256) * 256) + (-(-A * 4 // 256) * 256) + (-(-h_rows * TINY.f * 2 // 256) * 256)
+    ep_scratch = -(-(6 * 256 + 4) * 4 // 256) * 256                 # expert-parallel plan and local scan
+    combine_counters = -(-TINY.T * (TINY.d // 64) * 4 // 256) * 256  # the combine folded into GEMM2
+    expect = (256 + (-(-chunks * TINY.E * 4 // 256) * 256) + (-(-A * 4 // 256) * 256) + ep_scratch
+              + combine_counters + (-(-h_rows * TINY.f * 2 // 256) * 256))
     assert n == expect
     # shared expert adds its padded hidden rows
     sh = moe.Shape(T=256, d=512, E=8, k=2, f=1024, R=2, n_shared=1)
@@ -169,10 +172,12 @@ def test_status_strings_and_timeout_knob():
     assert lib.moe_set_gemm_policy(1) == 0
     assert lib.moe_set_gemm_policy(7) == -1
     assert lib.moe_set_gemm_policy(2) == 1
-    assert lib.moe_set_gemm_policy(3) == 2
-    assert lib.moe_set_gemm_policy(0) == 3
+    assert lib.moe_set_gemm_policy(3) == -1                       # the split schedule is gone
+    assert lib.moe_set_gemm_policy(0) == 2
     assert lib.moe_set_test_stall(1) == 0
     assert lib.moe_set_test_stall(0) == 1
+    assert lib.moe_set_pdl(0) == 1                                # on by default
+    assert lib.moe_set_pdl(1) == 0
 
 
 def test_gathering_gemm_rejects_inputs_past_32_bit_row_offsets():
@@ -272,3 +277,17 @@ def test_layer_binding_checks_every_output_buffer():
     o["y_shared"] = None
     with pytest.raises(ValueError, match=r"outs\['y_shared'\] is required"):
         moe.moe_layer(sh, None, None, None, None, None, None, o, ws)
+
+
+def test_static_dispatch_limit_counts_only_the_dispatch_scratch():
+    """The 1 MiB array holds what the dispatch kernels use (header, chunk counts, in-chunk ranks):
+    the skewed-prefill shape (590,080 bytes) passes the size check, whatever else the full
+    workspace holds; T 131072 x top-8 (4 MiB of ranks) does not. Without a GPU the accepted
+    shape then fails at its first CUDA call, never as MOE_ERR_UNSUPPORTED."""
+    lib = moe.load()
+    ok = moe.Shape(T=16384, d=7168, E=256, k=8, f=2048, R=8, n_shared=1)
+    assert moe.workspace_bytes(ok) > (1 << 20)
+    rc = lib.moe_dispatch_static(ctypes.byref(ok.c()), *([FAKE] * 10), None, None)
+    assert rc != moe.MOE_ERR_UNSUPPORTED
+    big = moe.Shape(T=131072, d=128, E=256, k=8, f=128, R=8)
+    assert lib.moe_dispatch_static(ctypes.byref(big.c()), *([FAKE] * 10), None, None) == moe.MOE_ERR_UNSUPPORTED

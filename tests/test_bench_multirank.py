@@ -32,7 +32,9 @@ def _worker(rank, world, port, q):
 def test_two_gloo_ranks_report_max_time_and_total_tokens():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = 29500 + (os.getpid() % 1000)
+    sys.path.insert(0, ROOT)
+    import bench
+    port = bench.free_port()
     procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
     for p in procs:
         p.start()
@@ -78,7 +80,9 @@ def test_gpus_flag_launches_that_many_ranks():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--rank-check"],
                        capture_output=True, text=True, timeout=240, env=env)
     assert r.returncode == 0, r.stderr[-2000:]
-    lines = [json.loads(ln)["rank_check"] for ln in r.stdout.splitlines() if ln.startswith('{"rank_check"')]
+    found = [json.loads(ln)["rank_check"] for ln in r.stdout.splitlines() if ln.startswith('{"rank_check"')]
+    assert len(found) == 1                         # rank 0 prints every rank's report on one line
+    lines = found[0]
     assert sorted(x["rank"] for x in lines) == [0, 1]
     for x in lines:
         assert x["world"] == 2 and x["gpus"] == 2

@@ -77,8 +77,8 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("policy", [moe.GEMM_AUTO, moe.GEMM_SINGLE, moe.GEMM_PAIR, moe.GEMM_SPLIT],
-                         ids=["auto", "single", "pair", "split"])
+@pytest.mark.parametrize("policy", [moe.GEMM_AUTO, moe.GEMM_SINGLE, moe.GEMM_PAIR],
+                         ids=["auto", "single", "pair"])
 @pytest.mark.parametrize("wl,cf,gather", CASES, ids=[c[0].name for c in CASES])
 def test_layer_writes_stay_inside_their_buffers(wl, cf, gather, policy):
     cap = moe.capacity_for(cf, wl.T, wl.k, wl.E) if cf else 0
@@ -120,3 +120,30 @@ def test_separate_entry_points_write_inside_their_buffers():
     for n, b in g.items():
         assert b.intact(), f"{n}: a guard byte was overwritten"
     assert ws.intact(), "workspace guard overwritten"
+
+
+@pytest.mark.parametrize("policy", [moe.GEMM_SINGLE, moe.GEMM_PAIR], ids=["single", "pair"])
+@pytest.mark.parametrize("wl,cf,gather", CASES, ids=[c[0].name for c in CASES])
+def test_layer_with_the_fused_combine_writes_inside_its_buffers(wl, cf, gather, policy):
+    """The combine folded into the down GEMM's epilogue (and the dispatch that zeroes its
+    counters) writes out and the workspace's counters only inside their buffers."""
+    cap = moe.capacity_for(cf, wl.T, wl.k, wl.E) if cf else 0
+    shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, n_shared=wl.n_shared, capacity=cap)
+    dv = moe_synth.device_inputs(wl)
+    g, outs = _guarded_outputs(shape, x_perm=not gather)
+    ws = _ws(shape)
+    old, old_f = moe.set_gemm_policy(policy), moe.set_fused_combine(True)
+    try:
+        moe.moe_layer(shape, dv["logits"], dv["x"], dv["w13"], dv["w2"], dv.get("w13s"), dv.get("w2s"), outs, ws.t)
+        status = moe.get_status(ws.t)
+    finally:
+        moe.set_gemm_policy(old)
+        moe.set_fused_combine(old_f)
+    assert status == 0
+    for n, b in g.items():
+        assert b.intact(), f"{n}: a guard byte was overwritten"
+    assert ws.intact(), "workspace guard overwritten"
+    res = oracle.layer(moe_synth.host_x(wl), moe_synth.host_logits(wl), moe_synth.host_w13(wl),
+                       moe_synth.host_w2(wl), wl.k, wl.R, moe_synth.host_w13s(wl) if wl.n_shared else None,
+                       moe_synth.host_w2s(wl) if wl.n_shared else None, capacity=cap)
+    close(f64(bits(outs["out"])), res["out"], "out (fused combine, guarded buffers)")

@@ -1,19 +1,21 @@
 """Element-wise parity of the persistent grouped GEMM when every CTA runs several tiles.
 
-The grouped GEMM is persistent: a CTA (or CTA pair) walks tiles L = b, b + grid,
-b + 2 grid, ... and carries two pieces of state from one tile to the next: the
-operand ring's stage and phase, and which of its two TMEM accumulators the tile
-uses (and that buffer's phase). Both only show up from a CTA's second and third
-tile on. Every case here is sized so that each CTA, or each CTA pair, runs at
-least three tiles in both GEMMs (checked from the routed counts before the
-comparison), and y_perm, y_shared and out are compared element by element with
-the oracle (the page "Expert Parallelism", §4 COMPUTE and COMBINE), under each
-tile policy: single-CTA tiles, CTA-pair tiles, and the split schedule.
+The grouped GEMM is persistent: a CTA (or CTA pair) claims tile after tile from a
+counter and carries state from one tile to the next: the operand ring's stage and
+phase, the tile queue's slot and phase, and which of its two TMEM accumulators the
+tile uses (and that buffer's phase). All of it only shows up from a CTA's second
+and third tile on. Every case here is sized so that the CTAs (the CTA pairs) run
+at least 4 tiles each on average in both GEMMs (checked from the routed counts
+before the comparison; tiles are claimed at run time, so a CTA's own count varies
+around that mean), and y_perm, y_shared and out are compared element by element
+with the oracle (the page "Expert Parallelism", §4 COMPUTE and COMBINE), under
+both tile shapes: single-CTA tiles, and CTA-pair tiles with half-height last
+blocks.
 
 The full Mixtral-like workload (T 4096, d 4096, f 14336: about 50 single tiles per
-CTA in gate/up, 7 to 8 pair tiles per cluster in down) is also compared in full: every
-element of y_perm and out against the oracle's whole-layer run (about a minute of
-host CPU).
+CTA in gate/up, 7 to 8 pair tiles per cluster in down) is also compared in full:
+every element of y_perm and out against the oracle's whole-layer run (about a
+minute of host CPU).
 """
 import functools
 
@@ -25,11 +27,11 @@ import moe_synth
 import oracle
 from parity_util import bits, close, f64, np_i32
 
-POLICIES = {"single": moe.GEMM_SINGLE, "pair": moe.GEMM_PAIR, "split": moe.GEMM_SPLIT}
+POLICIES = {"single": moe.GEMM_SINGLE, "pair": moe.GEMM_PAIR}
 
 CASES = {
     # 8 experts, ~1024 rows each (Zipf-skewed): ragged expert ends, ~68 m-tiles of 128 rows
-    "e8_k2": (moe_synth.Workload("mt_e8", T=4096, d=2048, E=8, k=2, f=1024, R=4, bias_kind="zipf",
+    "e8_k2": (moe_synth.Workload("mt_e8", T=4096, d=3072, E=8, k=2, f=1536, R=4, bias_kind="zipf",
                                  zipf_s=0.5, seed=5), 0.0),
     # 64 experts, top-8, 6 hot ones, a shared expert and a capacity factor of 1.25 (drops)
     "e64_k8_shared_cap": (moe_synth.Workload("mt_e64", T=1536, d=2048, E=64, k=8, f=1024, R=8, n_shared=1,
@@ -47,23 +49,13 @@ def _tiles(rows, tm):
 
 
 def tiles_per_unit(counts, T, n_shared, d, f, policy, sms):
-    """Fewest tiles any CTA (single) or CTA pair (pair, split) runs in either GEMM, from
-    the kernels' schedule: groups = experts (+ shared), m-tiles of 128 or 256 rows inner,
-    n-tiles of 128 h columns (gate/up) or 256 output columns (down), grid-stride over the
-    tile list. For the split schedule this is its CTA-pair launch (whole 256-row blocks,
-    and a last block of more than 128 rows); its second launch, last blocks of at most 128
-    rows, runs the single-CTA kernel, whose multi-tile walk the single policy covers."""
+    """Mean tiles per CTA (single) or per CTA pair (pair) in the GEMM with fewer tiles,
+    from the kernels' schedule: groups = experts (+ shared), m-tiles of 128 rows
+    (single) or 256 rows with a half-height last block of <= 128 rows (pair), n-tiles
+    of 128 h columns (gate/up) or 256 output columns (down)."""
     groups = list(counts) + ([T] * n_shared)
-    out = []
-    for n_tiles_n in (f // 128, d // 256):
-        if policy == "single":
-            tiles, units = sum(_tiles(r, 128) for r in groups) * n_tiles_n, sms
-        elif policy == "pair":
-            tiles, units = sum(_tiles(r, 256) for r in groups) * n_tiles_n, sms // 2
-        else:
-            tiles, units = sum(r // 256 + (1 if r % 256 > 128 else 0) for r in groups) * n_tiles_n, sms // 2
-        out.append(tiles // units)
-    return min(out)
+    tm, units = (128, sms) if policy == "single" else (256, sms // 2)
+    return min(sum(_tiles(r, tm) for r in groups) * n_tiles_n / units for n_tiles_n in (f // 128, d // 256))
 
 
 @functools.lru_cache(maxsize=None)
@@ -85,7 +77,7 @@ def test_multi_tile_layer_matches_oracle_element_by_element(case, policy):
     cap, res = _oracle_case(case)
     counts = res["expert_counts"].tolist()
     per_unit = tiles_per_unit(counts, wl.T, wl.n_shared, wl.d, wl.f, policy, _sm_count())
-    assert per_unit >= 3, f"only {per_unit} tiles per CTA/cluster: the case does not reach the persistent loop"
+    assert per_unit >= 4, f"only {per_unit:.1f} tiles per CTA/cluster: the case does not reach the persistent loop"
     if cf:
         assert res["dropped"] > 0
     shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, n_shared=wl.n_shared, capacity=cap)
@@ -117,15 +109,12 @@ def test_multi_tile_layer_matches_oracle_element_by_element(case, policy):
 def test_tile_count_model_matches_a_hand_count():
     """The tiles-per-unit count used above, on a hand-worked case: two experts of 300 and
     100 rows, d = 512, f = 256 (2 n-tiles in either GEMM), 4 SMs. Single: (3 + 1) m-tiles
-    x 2 = 8 tiles over 4 CTAs -> 2. Pair: (2 + 1) x 2 = 6 over 2 clusters -> 3. Split: one
-    whole 256-row block (300 = 256 + 44) as a pair tile, the 44- and 100-row last blocks
-    in the single-CTA launch: 1 x 2 = 2 pair tiles over 2 clusters -> 1; with 200 rows in
-    place of 100 (a last block of more than 128 rows), 2 x 2 = 4 -> 2."""
+    x 2 = 8 tiles over 4 CTAs -> 2. Pair: (2 + 1) x 2 = 6 (the 44- and 100-row last
+    blocks are half-height tiles) over 2 clusters -> 3. A shared expert is one more
+    group of T rows."""
     assert tiles_per_unit([300, 100], 0, 0, 512, 256, "single", 4) == 2
     assert tiles_per_unit([300, 100], 0, 0, 512, 256, "pair", 4) == 3
-    assert tiles_per_unit([300, 100], 0, 0, 512, 256, "split", 4) == 1
-    assert tiles_per_unit([300, 200], 0, 0, 512, 256, "split", 4) == 2
-    assert tiles_per_unit([300], 300, 1, 512, 256, "single", 4) == 3   # the shared expert is a group of T rows
+    assert tiles_per_unit([300], 300, 1, 512, 256, "single", 4) == 3
 
 
 @pytest.mark.gpu
@@ -143,7 +132,7 @@ def test_mixtral_prefill_full_output_matches_oracle():
     counts = np_i32(outs["expert_counts"]).tolist()
     del layer, outs, dv
     torch.cuda.empty_cache()
-    assert tiles_per_unit(counts, wl.T, 0, wl.d, wl.f, "single", _sm_count()) >= 3
+    assert tiles_per_unit(counts, wl.T, 0, wl.d, wl.f, "single", _sm_count()) >= 4
     res = oracle.layer(moe_synth.host_x(wl), moe_synth.host_logits(wl), moe_synth.host_w13(wl),
                        moe_synth.host_w2(wl), wl.k, wl.R)
     close(y_gpu, res["y_perm"], "y_perm mixtral_prefill (full)")

@@ -300,8 +300,8 @@ def _ffn_case(wl, idx=None):
         close(f64(bits(ys)), ys_ref, "y_shared")
 
 
-@pytest.fixture(params=[moe.GEMM_AUTO, moe.GEMM_SINGLE, moe.GEMM_PAIR, moe.GEMM_SPLIT],
-                ids=["auto_tiles", "single_tiles", "pair_tiles", "split_tiles"])
+@pytest.fixture(params=[moe.GEMM_AUTO, moe.GEMM_SINGLE, moe.GEMM_PAIR],
+                ids=["auto_tiles", "single_tiles", "pair_tiles"])
 def gemm_policy(request):
     old = moe.set_gemm_policy(request.param)
     yield request.param

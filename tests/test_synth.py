@@ -1,5 +1,7 @@
-"""The seeded input generator: reproducibility, distribution and workload structure (no GPU)."""
+"""The seeded input generator: reproducibility, distribution and workload structure (the per-rank
+weight fill, marked gpu, needs a device)."""
 import numpy as np
+import pytest
 
 import moe_synth
 import oracle
@@ -56,3 +58,15 @@ def test_skewed_prefill_hot_share_is_half():
     c = np.bincount(idx.reshape(-1), minlength=wl.E)
     hot = moe_synth.popularity_perm(wl) < wl.n_hot
     assert wl.n_hot == 26 and 0.48 <= c[hot].sum() / c.sum() <= 0.52
+
+
+@pytest.mark.gpu
+def test_device_expert_weights_are_the_rows_of_the_full_tensors():
+    """A rank's own experts' weights (expert parallelism) equal the matching rows of the full
+    tensors, bit for bit (host fill, the same generator)."""
+    import torch
+    wl = moe_synth.Workload("w", T=4, d=128, E=8, k=2, f=128, R=4, n_shared=1)
+    part = moe_synth.device_expert_weights(wl, 2, 6)
+    assert np.array_equal(part["w13"].view(torch.int16).cpu().numpy().view(np.uint16), moe_synth.host_w13(wl)[2:6])
+    assert np.array_equal(part["w2"].view(torch.int16).cpu().numpy().view(np.uint16), moe_synth.host_w2(wl)[2:6])
+    assert np.array_equal(part["w13s"].view(torch.int16).cpu().numpy().view(np.uint16), moe_synth.host_w13s(wl))
