@@ -453,6 +453,63 @@ def run_gpu(args, wl, rank, world, local_rank):
 
 
 # ---------------------------------------------------------------------------
+# the grouped GEMM against cuBLAS on the dense-equivalent problem (--dense-compare)
+# ---------------------------------------------------------------------------
+
+def run_dense_compare(args):
+    """One expert holding every row (no padding: rows % 256 == 0), our two GEMMs against
+    torch.matmul (cuBLAS) on the same bf16 operands, L2 flushed before every call, median of
+    the timed calls; both tile shapes of ours."""
+    import torch
+
+    import combine_warp_top_expert_b200 as moe
+    import moe_synth
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def timed(fn, reps=10, warm=3):
+        ts = []
+        for i in range(warm + reps):
+            flush.zero_()
+            a, b = ev(), ev()
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            if i >= warm:
+                ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    for rows, d, f in ((8192, 4096, 14336), (16384, 7168, 2048)):
+        wl = moe_synth.Workload("dense", T=rows, d=d, E=1, k=1, f=f, R=1)
+        dv = moe_synth.device_inputs(wl)
+        shape = moe.Shape(T=rows, d=d, E=1, k=1, f=f, R=1)
+        ws = moe.new_workspace(shape)
+        offs = torch.tensor([0, rows], dtype=torch.int32, device="cuda")
+        y = torch.empty((rows, d), dtype=torch.bfloat16, device="cuda")
+        h = torch.empty((rows, f), dtype=torch.bfloat16, device="cuda")
+        line = {"dense_compare": {"rows": rows, "d": d, "f": f}}
+        for name, pol in (("single", moe.GEMM_SINGLE), ("pair", moe.GEMM_PAIR)):
+            old = moe.set_gemm_policy(pol)
+            try:
+                gu = timed(lambda: moe.moe_expert_gate_up(shape, dv["x"], offs, dv["w13"], None, None, ws))
+                dn = timed(lambda: moe.moe_expert_down(shape, offs, dv["w2"], None, y, None, ws))
+            finally:
+                moe.set_gemm_policy(old)
+            line["dense_compare"][f"ours_{name}_gate_up_tflops"] = round(4.0 * rows * d * f / gu / 1e9, 1)
+            line["dense_compare"][f"ours_{name}_down_tflops"] = round(2.0 * rows * d * f / dn / 1e9, 1)
+        w13t, w2t = dv["w13"][0].t(), dv["w2"][0].t()
+        gu = timed(lambda: torch.matmul(dv["x"], w13t))
+        dn = timed(lambda: torch.matmul(h, w2t))
+        line["dense_compare"]["cublas_gate_up_tflops"] = round(4.0 * rows * d * f / gu / 1e9, 1)
+        line["dense_compare"]["cublas_down_tflops"] = round(2.0 * rows * d * f / dn / 1e9, 1)
+        line["dense_compare"]["device_status"] = moe.get_status(ws)
+        print(json.dumps(line), flush=True)
+        del dv, ws, y, h
+        torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------
 # expert parallelism across GPUs (--ep)
 # ---------------------------------------------------------------------------
 
@@ -667,6 +724,9 @@ def main():
                     help="override the workload's batch size T (smaller cases for profiling)")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch every kernel in plain stream order (no programmatic dependent launch)")
+    ap.add_argument("--dense-compare", action="store_true",
+                    help="our grouped GEMM on one expert holding every row against cuBLAS (torch.matmul) on the "
+                         "same operands")
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism across the --gpus ranks (E/R experts per GPU, rows exchanged over "
                          "NVLink inside dispatch and combine) instead of independent replicas")
@@ -687,6 +747,9 @@ def main():
 
     if args.regime_sweep:
         run_regime_sweep(args)
+        return
+    if args.dense_compare:
+        run_dense_compare(args)
         return
     import moe_synth
     wl = moe_synth.workload(args.config)
