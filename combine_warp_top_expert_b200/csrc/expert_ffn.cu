@@ -39,9 +39,9 @@
  *          of at most 128 rows runs as a half-height pair tile (M = 128, 64 rows
  *          per CTA, half the MMA time), so pairs pad a group to a multiple of 128
  *          rows, like single tiles.
- * moe_set_gemm_policy chooses the shape: by default single tiles for GEMM1 and
- * pair tiles for GEMM2 when d % 256 == 0 and the experts average at least 1024
- * rows.
+ * moe_set_gemm_policy chooses the shape: by default pair tiles when the experts
+ * average at least 1024 rows (GEMM2 also needs d % 256 == 0), single tiles
+ * otherwise.
  * GEMM1 can also gather its A rows straight from x through row_src instead of
  * reading x_perm (the GATHER instantiation: a warp of cp.async copies instead of
  * one TMA tile per stage).
@@ -1305,10 +1305,12 @@ cudaError_t launch_gate_up(const moe_shape_t& s, const WsLayout& L, uint8_t* ws,
   if (s.T == 0) return cudaSuccess;
   const bool sh = s.n_shared != 0;
   const bool gather = x_perm == nullptr; /* A rows gathered from x through row_src */
-  /* 128-row single-CTA tiles by default (measured faster for this GEMM's short K);
-   * CTA-pair tiles on request (never when gathering) */
+  /* CTA-pair tiles when the experts average at least 1024 rows (each SM then stages a
+   * third fewer operand bytes per K step, which is what holds this GEMM back at full
+   * clock); single-CTA tiles otherwise, where short groups end in half-height pair
+   * tiles that cost nearly as much as full ones. Never pairs when gathering rows. */
   const int pol = gather ? kGemmSingle : gemm_policy();
-  const bool pair = pol == kGemmPair;
+  const bool pair = pol == kGemmPair || (pol == kGemmAuto && L.A >= (int64_t)1024 * s.E);
   /* A = x_perm [A, d] (routed; rows of x gathered by the producer warp instead when x_perm is
    * null) / x [T, d] (shared); B = w13 [E*2f, d] / w13s [2f, d] */
   if (gather && (uint64_t)s.T * (uint64_t)s.d * 2u > 0xFFFFFFFFull) return cudaErrorInvalidValue;

@@ -197,7 +197,7 @@ moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_bf16_t* x_perm, 
 /* The two halves of moe_expert_ffn, for callers that schedule or time them
  * separately; moe_expert_ffn is exactly gate_up followed by down.
  * moe_expert_gate_up: GEMM1 + SwiGLU, h = silu(x W_gate^T) * (x W_up^T), written
- *   to the workspace (each expert's rows padded to a multiple of 128).
+ *   to the workspace (each expert's rows padded to a multiple of 256).
  * moe_expert_down: GEMM2, y_perm (and y_shared) = h W2^T, reading the h rows that
  *   the preceding moe_expert_gate_up on the same workspace, shape and
  *   expert_offsets left there. Arguments as for moe_expert_ffn. */
@@ -394,8 +394,8 @@ uint64_t moe_set_wait_timeout_ns(uint64_t ns);
  * (cta_group::2; the down GEMM needs d % 256 == 0 for them), where a group's last
  * block of at most 128 rows runs as a half-height tile (128 x 256, 64 rows per
  * CTA), so both shapes pad a group to a multiple of 128 rows.
- *   0 (default) = single-CTA tiles, except CTA-pair tiles for the down GEMM
- *       when the routed experts average at least 1024 rows (T*k >= 1024*E);
+ *   0 (default) = CTA-pair tiles when the routed experts average at least 1024
+ *       rows (T*k >= 1024*E), single-CTA tiles otherwise;
  *   1 = single-CTA tiles only;
  *   2 = CTA-pair tiles wherever they apply.
  * Either way the CTAs claim tiles at run time from a counter in the workspace
