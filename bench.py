@@ -289,6 +289,7 @@ def run_gpu(args, wl, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     moe.set_gemm_policy({"auto": moe.GEMM_AUTO, "single": moe.GEMM_SINGLE, "pair": moe.GEMM_PAIR}[args.gemm_policy])
     moe.set_pdl(not args.no_pdl)
+    moe.set_dispatch_path(DISPATCH_PATHS[args.dispatch_path])
     wl_r = wl.with_(seed=replica_seed(wl.seed, rank))
     cap = moe.capacity_for(args.capacity_factor, wl.T, wl.k, wl.E) if args.capacity_factor else 0
     shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, n_shared=wl.n_shared, capacity=cap)
@@ -344,6 +345,7 @@ def run_gpu(args, wl, rank, world, local_rank):
     events = [(ev(), ev()) for _ in range(args.steps)]
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
     smi_index = vis.split(",")[local_rank].strip() if vis else str(local_rank)
+    launches0 = moe.kernel_launches()
     with ClockSampler(smi_index) as clocks:
         for i in range(args.steps):
             flush.zero_()
@@ -351,6 +353,7 @@ def run_gpu(args, wl, rank, world, local_rank):
             layer_step()
             events[i][1].record(stream)
         torch.cuda.synchronize(dev)
+    gpu_launches = moe.kernel_launches() - launches0  # the library's own count of its kernel launches
     if world > 1:
         dist.barrier()
     per_step = [a.elapsed_time(b) for a, b in events]
@@ -421,6 +424,7 @@ def run_gpu(args, wl, rank, world, local_rank):
                    "l2": "flushed between steps (512 MiB write, outside the step's events)",
                    "gemm_tiles": args.gemm_policy,
                    "launch_overlap": "off" if args.no_pdl else "programmatic dependent launch",
+                   "dispatch_path": args.dispatch_path,
                    "x_perm": "not materialised (rows gathered in the gate/up GEMM)" if args.gather else "materialised",
                    "capacity_factor": args.capacity_factor, "capacity": cap,
                    "dropped_fraction": 1.0 - sum(counts) / float(wl.T * wl.k) if wl.T else 0.0,
@@ -445,7 +449,7 @@ def run_gpu(args, wl, rank, world, local_rank):
                 "timing": "wall clock over the K steps issued back to back (copies of each step overlap the "
                           "neighbouring steps' compute), one synchronize at the end",
                 "isolated_call_ms": e2e_single_ms},
-        "gpu_launches": args.steps * launches_per_layer(shape, args.gemm_policy),
+        "gpu_launches": gpu_launches,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
@@ -550,12 +554,14 @@ def run_gpu_ep(args, wl, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    launches0 = moe.kernel_launches()
     for i in range(args.steps):
         flush.zero_()
         evs[i][0].record()
         layer(dv["logits"], dv["x"])
         evs[i][1].record()
     torch.cuda.synchronize(dev)
+    gpu_launches = moe.kernel_launches() - launches0
     status = layer.status()
     local_ms = sum(a.elapsed_time(b) for a, b in evs)
     max_ms = max_over_ranks(local_ms, world, dev)
@@ -572,7 +578,7 @@ def run_gpu_ep(args, wl, rank, world, local_rank):
                        "l2": "flushed between steps (512 MiB write, outside the step's events)"},
             # route 1; counts 2 (histogram, exchange); dispatch 4 (wait, plan, rows, signal); expert FFN 2
             # (+2 shared) between a wait and a signal; combine 3 (wait, gather-sum, signal); final wait 1
-            "gpu_launches": args.steps * (15 + 2 * wl.n_shared),
+            "gpu_launches": gpu_launches,
         }), flush=True)
     del layer, peers
     torch.cuda.synchronize(dev)
@@ -659,12 +665,7 @@ def run_regime_sweep(args):
         print(json.dumps(dict(regime_fit=fit)), flush=True)
 
 
-def launches_per_layer(shape, gemm_policy: str) -> int:
-    """Kernels one moe_layer call launches: route 1, dispatch 2 (histogram + scan, permute),
-    gate/up 1, down 1, combine 1."""
-    if shape.T == 0:
-        return 1  # dispatch's empty-batch kernel
-    return 6
+DISPATCH_PATHS = {"auto": 0, "two_pass": 1, "one_pass": 2}
 
 
 def free_port() -> int:
@@ -709,6 +710,9 @@ def main():
     ap.add_argument("--gemm-policy", default="auto", choices=["auto", "single", "pair"],
                     help="grouped-GEMM tiles: chosen from the shape (auto), single-CTA 128-row, or CTA-pair 256x256 "
                          "(a group's last block of <= 128 rows as a half-height pair tile)")
+    ap.add_argument("--dispatch-path", default="auto", choices=list(DISPATCH_PATHS),
+                    help="dispatch: one kernel for small batches and two otherwise (auto), always the histogram "
+                         "kernel + permute kernel (two_pass), or the one-pass kernel wherever it applies")
     ap.add_argument("--capacity-factor", type=float, default=None,
                     help="per-expert capacity ceil(C*T*k/E); excess assignments are dropped (default: none)")
     ap.add_argument("--regime-sweep", action="store_true",

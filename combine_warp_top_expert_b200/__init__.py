@@ -26,10 +26,12 @@ ABI_FUNCTIONS = (
     "moe_expert_gate_up", "moe_expert_down", "moe_dispatch_static", "moe_set_gemm_policy",
     "moe_set_test_stall", "moe_expert_gate_up_gather", "moe_capacity_for", "moe_dispatch_static_scratch",
     "moe_set_pdl", "moe_ep_exchange_counts", "moe_ep_dispatch", "moe_ep_signal", "moe_ep_wait", "moe_ep_combine",
-    "moe_ep_plan_host", "moe_expert_down_combine", "moe_set_fused_combine",
+    "moe_ep_plan_host", "moe_expert_down_combine", "moe_set_fused_combine", "moe_set_dispatch_path",
+    "moe_kernel_launches",
 )
 EP_SLOT_COUNTS, EP_SLOT_ROWS, EP_SLOT_OUTPUTS, EP_SLOT_DONE = 0, 1, 2, 3
 GEMM_AUTO, GEMM_SINGLE, GEMM_PAIR = 0, 1, 2
+DISPATCH_AUTO, DISPATCH_TWO_PASS, DISPATCH_ONE_PASS = 0, 1, 2
 
 
 class MoEError(RuntimeError):
@@ -122,6 +124,10 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     L.moe_set_fused_combine.argtypes = [ctypes.c_int]
     L.moe_set_pdl.restype = ctypes.c_int
     L.moe_set_pdl.argtypes = [ctypes.c_int]
+    L.moe_set_dispatch_path.restype = ctypes.c_int
+    L.moe_set_dispatch_path.argtypes = [ctypes.c_int]
+    L.moe_kernel_launches.restype = ctypes.c_uint64
+    L.moe_kernel_launches.argtypes = []
     L.moe_set_test_stall.restype = ctypes.c_int
     L.moe_set_test_stall.argtypes = [ctypes.c_int]
     L.moe_set_wait_timeout_ns.restype = ctypes.c_uint64
@@ -240,6 +246,17 @@ def set_test_stall(enable: bool) -> int:
 def set_pdl(enable: bool) -> int:
     """Programmatic dependent launch of the library's kernels on (default) or off (see moe_set_pdl)."""
     return load().moe_set_pdl(1 if enable else 0)
+
+
+def kernel_launches() -> int:
+    """Kernels the library has launched in this process so far (see moe_kernel_launches)."""
+    return int(load().moe_kernel_launches())
+
+
+def set_dispatch_path(path: int) -> int:
+    """DISPATCH_AUTO, DISPATCH_TWO_PASS or DISPATCH_ONE_PASS (see moe_set_dispatch_path); returns
+    the previous path, -1 if `path` is unknown."""
+    return load().moe_set_dispatch_path(int(path))
 
 
 def set_fused_combine(enable: bool) -> int:

@@ -28,70 +28,44 @@ namespace {
 constexpr int kHistThreads = 512;
 constexpr int kHistWarps = kHistThreads / 32;
 constexpr int kScanThreads = 512;
+constexpr int kOnePassThreads = 512;
+constexpr int kOnePassWarps = kOnePassThreads / 32;
+constexpr int kOnePassMaxLocal = 1024; /* assignments of one CTA's tokens (rows kept in shared memory) */
 
-/* Scan over the per-chunk counts (run by one whole CTA of kScanThreads threads):
- * each expert keeps min(demand, cap) rows; offsets over the kept counts; chunk
- * counts -> rank bases (the expert-local rank of each chunk's first assignment,
- * in place); rank counts/offsets, imbalance; row_src beyond the kept total = -1. */
-__device__ void scan_chunks(int32_t* chunk, int64_t C, int E, int R, int64_t A, int32_t cap, int32_t* expert_counts,
-                            int32_t* expert_offsets, int32_t* rank_counts, int32_t* rank_offsets, float* imbalance,
-                            int32_t* row_src) {
-  __shared__ int32_t part[kScanThreads]; /* [G][E] partial sums over chunk ranges */
-  __shared__ int32_t cnt[kMaxE];
-  __shared__ int32_t off[kMaxE + 1];
+/* Exclusive scan of cnt[0..E) into off[0..E] (off[E] = total), run by warp 0 alone:
+ * each lane owns a contiguous slice of the experts. */
+__device__ void expert_offsets_warp0(const int32_t* cnt, int32_t* off, int E) {
+  const int lane = threadIdx.x & 31;
+  const int per = (E + 31) / 32;
+  const int b = min(E, lane * per), en = min(E, b + per);
+  int local = 0;
+  for (int i = b; i < en; ++i) local += cnt[i];
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int run = incl - local;
+  for (int i = b; i < en; ++i) {
+    off[i] = run;
+    run += cnt[i];
+  }
+  if (lane == 31) off[E] = incl;
+}
+
+/* The per-expert and per-rank outputs of dispatch from the kept counts cnt[E] and
+ * their offsets off[E+1] (shared memory, complete): expert counts/offsets, logical-rank
+ * counts/offsets and the imbalance ratios. Called by every thread of the CTA. */
+__device__ void write_dispatch_totals(const int32_t* cnt, const int32_t* off, int E, int R, int32_t* expert_counts,
+                                      int32_t* expert_offsets, int32_t* rank_counts, int32_t* rank_offsets,
+                                      float* imbalance) {
   __shared__ int32_t s_max[2];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int G = max(1, kScanThreads / E);
-  const int e = tid % E, g = tid / E;
-  const bool active = g < G;
-  const int64_t c_begin = active ? (C * g) / G : 0, c_end = active ? (C * (g + 1)) / G : 0;
-  int32_t s = 0;
-  for (int64_t c = c_begin; c < c_end; ++c) s += __ldcg(chunk + c * E + e);
-  if (active) part[g * E + e] = s;
-  __syncthreads();
-  if (tid < E) {
-    int run = 0;
-    for (int q = 0; q < G; ++q) {
-      const int v = part[q * E + tid];
-      part[q * E + tid] = run;
-      run += v;
-    }
-    cnt[tid] = min(run, cap); /* kept rows */
-  }
-  __syncthreads();
-  /* exclusive scan of cnt[0..E) by warp 0: each lane owns a contiguous slice */
-  if (warp == 0) {
-    const int per = (E + 31) / 32;
-    const int b = min(E, lane * per), en = min(E, b + per);
-    int local = 0;
-    for (int i = b; i < en; ++i) local += cnt[i];
-    int incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int run = incl - local;
-    for (int i = b; i < en; ++i) {
-      off[i] = run;
-      run += cnt[i];
-    }
-    if (lane == 31) off[E] = incl;
-  }
-  __syncthreads();
   const int total = off[E];
-  /* chunk rank bases, in place */
-  if (active) {
-    int32_t base = part[g * E + e];
-    for (int64_t c = c_begin; c < c_end; ++c) {
-      const int32_t v = __ldcg(chunk + c * E + e);
-      chunk[c * E + e] = base;
-      base += v;
-    }
-  }
-  if (tid < E) {
-    expert_counts[tid] = cnt[tid];
-    expert_offsets[tid] = off[tid];
+  for (int e = tid; e < E; e += blockDim.x) {
+    expert_counts[e] = cnt[e];
+    expert_offsets[e] = off[e];
   }
   if (tid == 0) expert_offsets[E] = total;
   const int per_rank = E / R;
@@ -127,6 +101,50 @@ __device__ void scan_chunks(int32_t* chunk, int64_t C, int E, int R, int64_t A, 
       imbalance[1] = (float)((double)((int64_t)s_max[1] * E) / (double)total);
     }
   }
+}
+
+/* Scan over the per-chunk counts (run by one whole CTA of kScanThreads threads):
+ * each expert keeps min(demand, cap) rows; offsets over the kept counts; chunk
+ * counts -> rank bases (the expert-local rank of each chunk's first assignment,
+ * in place); rank counts/offsets, imbalance; row_src beyond the kept total = -1. */
+__device__ void scan_chunks(int32_t* chunk, int64_t C, int E, int R, int64_t A, int32_t cap, int32_t* expert_counts,
+                            int32_t* expert_offsets, int32_t* rank_counts, int32_t* rank_offsets, float* imbalance,
+                            int32_t* row_src) {
+  __shared__ int32_t part[kScanThreads]; /* [G][E] partial sums over chunk ranges */
+  __shared__ int32_t cnt[kMaxE];
+  __shared__ int32_t off[kMaxE + 1];
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int G = max(1, kScanThreads / E);
+  const int e = tid % E, g = tid / E;
+  const bool active = g < G;
+  const int64_t c_begin = active ? (C * g) / G : 0, c_end = active ? (C * (g + 1)) / G : 0;
+  int32_t s = 0;
+  for (int64_t c = c_begin; c < c_end; ++c) s += __ldcg(chunk + c * E + e);
+  if (active) part[g * E + e] = s;
+  __syncthreads();
+  if (tid < E) {
+    int run = 0;
+    for (int q = 0; q < G; ++q) {
+      const int v = part[q * E + tid];
+      part[q * E + tid] = run;
+      run += v;
+    }
+    cnt[tid] = min(run, cap); /* kept rows */
+  }
+  __syncthreads();
+  if (warp == 0) expert_offsets_warp0(cnt, off, E);
+  __syncthreads();
+  const int total = off[E];
+  /* chunk rank bases, in place */
+  if (active) {
+    int32_t base = part[g * E + e];
+    for (int64_t c = c_begin; c < c_end; ++c) {
+      const int32_t v = __ldcg(chunk + c * E + e);
+      chunk[c * E + e] = base;
+      base += v;
+    }
+  }
+  write_dispatch_totals(cnt, off, E, R, expert_counts, expert_offsets, rank_counts, rank_offsets, imbalance);
   if (row_src)
     for (int64_t p = total + tid; p < A; p += blockDim.x) row_src[p] = -1;
 }
@@ -230,6 +248,178 @@ __global__ void __launch_bounds__(kScanThreads) dispatch_empty_kernel(int E, int
   pdl_trigger();
   scan_chunks(nullptr, 0, E, R, 0, 0x7FFFFFFF, expert_counts, expert_offsets, rank_counts, rank_offsets, imbalance,
               nullptr);
+}
+
+/* One-pass dispatch (small batches): histogram, scan and permute in one launch, with
+ * no CTA waiting on another. Each CTA owns a contiguous range of (token, slice) items
+ * and counts all A expert ids itself (A is small: they are L2-resident after the
+ * router), split at its first token: the totals give every expert's kept count and
+ * offset, the counts before its range the rank of its first assignment to each
+ * expert; warp 0 then ranks the CTA's own assignments in order (the same stable
+ * order as the two-kernel path, so the same rows). Every CTA derives the same totals
+ * from the same ids; CTA 0 writes them out. The first item's row vectors are loaded
+ * before the counting (before pdl_wait when early_x: x then comes from before the
+ * kernel this one follows). */
+template <int U>
+__global__ void __launch_bounds__(kOnePassThreads, 2) dispatch_onepass_kernel(
+    const uint16_t* __restrict__ x, const int32_t* __restrict__ topk_idx, int64_t T, int d, int E, int R, int k,
+    int32_t cap, int64_t ipc, int slices, int vps, int32_t* expert_counts, int32_t* expert_offsets,
+    int32_t* rank_counts, int32_t* rank_offsets, float* imbalance, int32_t* __restrict__ row_src,
+    int32_t* __restrict__ assign_row, uint16_t* __restrict__ x_perm, uint32_t* status, int early_x) {
+  extern __shared__ int32_t sh[];
+  int32_t* hpre = sh;                           /* [warps][E]: ids before the CTA's first assignment */
+  int32_t* htot = sh + kOnePassWarps * E;       /* [warps][E]: all ids */
+  int32_t* s_pos = htot + kOnePassWarps * E;    /* [kOnePassMaxLocal]: rows of the CTA's assignments */
+  __shared__ int32_t s_run[kMaxE];
+  __shared__ int32_t s_cnt[kMaxE];
+  __shared__ int32_t s_off[kMaxE + 1];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t A = T * k;
+  const int64_t items = T * slices;
+  const int64_t i_lo = (int64_t)blockIdx.x * ipc;
+  const int64_t i_hi = min(items, i_lo + ipc);
+  const int64_t t_lo = i_lo / slices, t_hi = (i_hi - 1) / slices + 1;
+  const int64_t a_lo = t_lo * k, a_hi = t_hi * k;
+  const bool move = x_perm != nullptr;
+  const int nv = d >> 3;
+  for (int i = tid; i < 2 * kOnePassWarps * E; i += blockDim.x) sh[i] = 0;
+
+  uint4 buf[U];
+  auto load_item = [&](int64_t w) {
+    const int64_t t = w / slices;
+    const int sl = (int)(w - t * slices);
+    const uint16_t* src = x + t * d;
+    const int v_begin = sl * vps + lane, v_end = min(nv, (sl + 1) * vps);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int v = v_begin + 32 * u;
+      if (v < v_end) buf[u] = ld_nc_v4(src + (int64_t)v * 8);
+    }
+  };
+  const int64_t w0 = i_lo + warp;
+  if (early_x && move && w0 < i_hi) load_item(w0);
+  pdl_wait(); /* topk_idx comes from the kernel before */
+  pdl_trigger();
+  if (!early_x && move && w0 < i_hi) load_item(w0);
+  __syncthreads();
+
+  /* 1. per-warp histograms of all ids and of the ids before a_lo (4 loads in flight) */
+  bool bad = false;
+  int32_t* my_pre = hpre + warp * E;
+  int32_t* my_tot = htot + warp * E;
+  constexpr int kStep = kOnePassThreads; /* ids per CTA-wide step */
+  for (int64_t base = (int64_t)warp * 32; base < A; base += 4 * kStep) {
+    int ev[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t a = base + (int64_t)u * kStep + lane;
+      ev[u] = a < A ? __ldg(topk_idx + a) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t a = base + (int64_t)u * kStep + lane;
+      int e = ev[u];
+      if (a < A && (e < 0 || e >= E)) {
+        bad = true;
+        e = -1;
+      }
+      const unsigned before = __ballot_sync(0xFFFFFFFFu, a < a_lo);
+      const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+      if (e >= 0 && lane == __ffs(peers) - 1) {
+        my_tot[e] += __popc(peers);
+        my_pre[e] += __popc(peers & before);
+      }
+    }
+  }
+  __syncthreads();
+  /* 2. totals, kept counts, offsets; the rank bases of this CTA */
+  for (int e = tid; e < E; e += blockDim.x) {
+    int p = 0, t = 0;
+#pragma unroll
+    for (int w = 0; w < kOnePassWarps; ++w) {
+      p += hpre[w * E + e];
+      t += htot[w * E + e];
+    }
+    s_run[e] = p;
+    s_cnt[e] = min(t, cap);
+  }
+  __syncthreads();
+  if (warp == 0) expert_offsets_warp0(s_cnt, s_off, E);
+  __syncthreads();
+  const int total = s_off[E];
+  /* 3. warp 0 ranks the CTA's own assignments in order; the CTA holding a token's
+   * slice 0 writes its row_src / assign_row entries */
+  if (warp == 0) {
+    for (int64_t b = a_lo; b < a_hi; b += 32) {
+      const int64_t a = b + lane;
+      int e = a < a_hi ? __ldg(topk_idx + a) : -1;
+      if (e >= E) e = -1;
+      if (e < 0) e = -1;
+      const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+      int pos = -1;
+      if (e >= 0) {
+        const int rank = s_run[e] + __popc(peers & ((1u << lane) - 1u));
+        if (rank < cap) {
+          const int64_t q = (int64_t)s_off[e] + rank;
+          if (q >= 0 && q < A)
+            pos = (int)q;
+          else
+            bad = true;
+        }
+      }
+      __syncwarp();
+      if (e >= 0 && lane == __ffs(peers) - 1) s_run[e] += __popc(peers);
+      __syncwarp();
+      if (a < a_hi) {
+        s_pos[a - a_lo] = pos;
+        if ((a / k) * slices >= i_lo) {
+          assign_row[a] = pos;
+          if (pos >= 0) row_src[pos] = (int32_t)a;
+        }
+      }
+    }
+  }
+  for (int64_t p = total + (int64_t)blockIdx.x * blockDim.x + tid; p < A; p += (int64_t)gridDim.x * blockDim.x)
+    row_src[p] = -1;
+  if (blockIdx.x == 0)
+    write_dispatch_totals(s_cnt, s_off, E, R, expert_counts, expert_offsets, rank_counts, rank_offsets, imbalance);
+  __syncthreads();
+  /* 4. the permute of this CTA's items */
+  if (move) {
+    for (int64_t w = w0; w < i_hi; w += kOnePassWarps) {
+      const int64_t t = w / slices;
+      const int sl = (int)(w - t * slices);
+      const uint16_t* src = x + t * d;
+      const int v_begin = sl * vps + lane, v_end = min(nv, (sl + 1) * vps);
+      if (w != w0) load_item(w);
+      const int pos = lane < k ? s_pos[t * k + lane - a_lo] : -1;
+      uint16_t* dst[kMaxK];
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j) {
+        const int p = __shfl_sync(0xFFFFFFFFu, pos, j);
+        dst[j] = (j < k && p >= 0) ? x_perm + (int64_t)p * d : nullptr;
+      }
+      for (int v0 = v_begin; v0 < v_end; v0 += 32 * U) {
+        if (v0 != v_begin) {
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const int v = v0 + 32 * u;
+            if (v < v_end) buf[u] = ld_nc_v4(src + (int64_t)v * 8);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j) {
+          if (dst[j] == nullptr) continue;
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const int v = v0 + 32 * u;
+            if (v < v_end) st_v4(dst[j] + (int64_t)v * 8, buf[u]);
+          }
+        }
+      }
+    }
+  }
+  if (bad) raise_status(status, MOE_DEV_BOUNDS);
 }
 
 /* EP form: rows go to the receive buffer of the rank that owns their expert, at the
@@ -368,10 +558,39 @@ RowSlices row_slices(int64_t T, int d) {
   return r;
 }
 
+OnePass onepass_plan(const moe_shape_t& s, bool index_only) {
+  OnePass op;
+  const int path = dispatch_path();
+  const int64_t A = (int64_t)s.T * s.k;
+  if (s.T <= 0 || path == kDispatchTwoPass || (path == kDispatchAuto && A > kOnePassAutoMaxA)) return op;
+  RowSlices rs = row_slices(s.T, s.d);
+  if (index_only) {
+    rs.slices = 1;
+    rs.vps = s.d / 8;
+  }
+  const int64_t items = (int64_t)s.T * rs.slices;
+  const int64_t max_blocks = (int64_t)num_sms() * 2;
+  int64_t blocks = (items + kOnePassWarps - 1) / kOnePassWarps;
+  if (blocks > max_blocks) blocks = max_blocks;
+  if (blocks < 1) blocks = 1;
+  const int64_t ipc = (items + blocks - 1) / blocks;
+  blocks = (items + ipc - 1) / ipc;
+  /* tokens one CTA touches: at most ceil(ipc / slices) + 1 */
+  const int64_t local = ((ipc + rs.slices - 1) / rs.slices + 1) * s.k;
+  if (local > kOnePassMaxLocal) return op;
+  op.use = true;
+  op.blocks = (int)blocks;
+  op.ipc = ipc;
+  op.slices = rs.slices;
+  op.vps = rs.vps;
+  return op;
+}
+
 cudaError_t launch_dispatch(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const uint16_t* x,
                             const int32_t* topk_idx, int32_t* expert_counts, int32_t* expert_offsets,
                             int32_t* rank_counts, int32_t* rank_offsets, int32_t* row_src, int32_t* assign_row,
-                            uint16_t* x_perm, float* imbalance, cudaStream_t stream, uint16_t* fc_out) {
+                            uint16_t* x_perm, float* imbalance, cudaStream_t stream, uint16_t* fc_out,
+                            bool early_x) {
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
   uint32_t* ticket = reinterpret_cast<uint32_t*>(ws + L.status + kTicketOffset);
   int32_t* chunk = reinterpret_cast<int32_t*>(ws + L.chunk);
@@ -381,8 +600,18 @@ cudaError_t launch_dispatch(const moe_shape_t& s, const WsLayout& L, uint8_t* ws
     return launch_kernel(dispatch_empty_kernel, dim3(1), dim3(kScanThreads), 0, stream, 1, s.E, s.R, expert_counts,
                          expert_offsets, rank_counts, rank_offsets, imbalance);
   }
-  const size_t smem = (size_t)kHistWarps * s.E * sizeof(int32_t);
   const int32_t cap = s.capacity > 0 ? s.capacity : 0x7FFFFFFF;
+  if (fc_out == nullptr) {
+    const OnePass op = onepass_plan(s, x_perm == nullptr);
+    if (op.use) {
+      const size_t osmem = (size_t)(2 * kOnePassWarps * s.E + kOnePassMaxLocal) * sizeof(int32_t);
+      return launch_kernel(dispatch_onepass_kernel<4>, dim3((unsigned)op.blocks), dim3(kOnePassThreads), osmem,
+                           stream, 1, x, topk_idx, (int64_t)s.T, s.d, s.E, s.R, s.k, cap, op.ipc, op.slices, op.vps,
+                           expert_counts, expert_offsets, rank_counts, rank_offsets, imbalance, row_src, assign_row,
+                           x_perm, status, early_x ? 1 : 0);
+    }
+  }
+  const size_t smem = (size_t)kHistWarps * s.E * sizeof(int32_t);
   cudaError_t e = launch_kernel(dispatch_count_kernel, dim3((unsigned)L.n_chunks), dim3(kHistThreads), smem, stream,
                                 1, topk_idx, L.A, s.E, s.R, cap, chunk_assign, L.n_chunks, chunk, lrank, status,
                                 ticket, expert_counts, expert_offsets, rank_counts, rank_offsets, imbalance, row_src);

@@ -167,7 +167,14 @@ __device__ __forceinline__ bool build_schedule(const FfnParams& p, int32_t* s_of
   return __all_sync(0xFFFFFFFFu, ok);
 }
 
-/* Linear tile index -> tile. Inside a group the m-tiles are the inner index. */
+/* Tile order inside a group: bands of consecutive m-tiles whose A rows take at most
+ * kBandBytes; inside a band the m-tiles are the inner index. So the tiles running at
+ * once share their weight tile, and a band's A rows stay in L2 while every weight
+ * column tile passes over them; a group with more rows than one band (a shared expert
+ * over a long batch) then reads its A rows from DRAM once, not once per column tile. */
+constexpr int64_t kBandBytes = int64_t(24) << 20;
+
+/* Linear tile index -> tile (groups in order; bands of m-tiles inside a group). */
 template <int MODE, int TM, int BN>
 __device__ __forceinline__ Tile decode_tile(int64_t L, const FfnParams& p, const int32_t* s_off,
                                             const int32_t* s_mpref, const int32_t* s_hpref) {
@@ -187,8 +194,13 @@ __device__ __forceinline__ Tile decode_tile(int64_t L, const FfnParams& p, const
   const int local = (int)(L - (int64_t)s_mpref[lo] * p.n_tiles_n);
   const bool shared = lo >= p.E;
   const int rows = shared ? (int)p.T : s_off[lo + 1] - s_off[lo];
-  t.n = local / mt;
-  t.m = local - t.n * mt;
+  const int64_t band_bytes = (int64_t)TM * p.K * 2;
+  const int band = (int)max((int64_t)1, kBandBytes / band_bytes);
+  const int b = local / (band * p.n_tiles_n);         /* band of this tile */
+  const int r = local - b * band * p.n_tiles_n;       /* index inside the band */
+  const int gm = min(band, mt - b * band);             /* m-tiles in this band */
+  t.n = r / gm;
+  t.m = b * band + (r - t.n * gm);
   t.valid = min(TM, rows - t.m * TM);
   t.half = (TM == 256 && t.valid <= 128) ? 1 : 0;
   const int hrow = s_hpref[lo] * kHPad + t.m * TM;

@@ -33,6 +33,8 @@ std::atomic<int> g_gemm_policy{kGemmAuto};
 std::atomic<int> g_test_stall{0};
 std::atomic<int> g_pdl{1};
 std::atomic<int> g_fused_combine{0};
+std::atomic<int> g_dispatch_path{kDispatchAuto};
+std::atomic<uint64_t> g_launches{0};
 
 }  // namespace
 
@@ -120,6 +122,10 @@ bool test_stall() { return g_test_stall.load(std::memory_order_relaxed) != 0; }
 bool pdl_enabled() { return g_pdl.load(std::memory_order_relaxed) != 0; }
 
 bool fused_combine_enabled() { return g_fused_combine.load(std::memory_order_relaxed) != 0; }
+
+int dispatch_path() { return g_dispatch_path.load(std::memory_order_relaxed); }
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 bool debug_log() {
   static const bool on = [] {
@@ -302,7 +308,7 @@ moe_status_t moe_layer(const moe_shape_t* shape, const moe_layer_buffers_t* b, v
   const bool fused = fused_combine_enabled();
   e = launch_dispatch(*shape, L, w, b->x, b->topk_idx, b->expert_counts, b->expert_offsets, b->rank_counts,
                       b->rank_offsets, b->row_src, b->assign_row, b->x_perm, b->imbalance, s,
-                      fused ? b->out : nullptr);
+                      fused ? b->out : nullptr, /*early_x=*/true);
   if (e != cudaSuccess) return cuda_fail(e);
   const uint16_t* ysh_in = shape->n_shared ? b->y_shared : nullptr;
   /* x_perm null: dispatch writes indices only and GEMM1 gathers the rows of x itself */
@@ -378,6 +384,13 @@ moe_status_t moe_expert_down_combine(const moe_shape_t* shape, const int32_t* ex
 }
 
 int moe_set_pdl(int enable) { return g_pdl.exchange(enable ? 1 : 0, std::memory_order_relaxed); }
+
+uint64_t moe_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int moe_set_dispatch_path(int path) {
+  if (path != kDispatchAuto && path != kDispatchTwoPass && path != kDispatchOnePass) return -1;
+  return g_dispatch_path.exchange(path, std::memory_order_relaxed);
+}
 
 int moe_set_test_stall(int enable) { return g_test_stall.exchange(enable ? 1 : 0, std::memory_order_relaxed); }
 

@@ -37,6 +37,23 @@ struct RowSlices {
 };
 RowSlices row_slices(int64_t T, int d);
 
+/* Dispatch path (see moe_set_dispatch_path). */
+constexpr int kDispatchAuto = 0;     /* one pass when A <= kOnePassAutoMaxA, else two kernels */
+constexpr int kDispatchTwoPass = 1;  /* histogram/scan kernel, then the permute kernel */
+constexpr int kDispatchOnePass = 2;  /* one kernel wherever a CTA's assignments fit its shared memory */
+constexpr int64_t kOnePassAutoMaxA = 16384;
+int dispatch_path();
+
+/* Launch shape of the one-pass dispatch (use = false: the two-kernel path runs). */
+struct OnePass {
+  bool use = false;
+  int blocks = 0;
+  int64_t ipc = 0; /* (token, slice) items per CTA, contiguous */
+  int slices = 1;
+  int vps = 32;
+};
+OnePass onepass_plan(const moe_shape_t& s, bool index_only);
+
 /* Byte offsets into the caller's workspace (all 256-byte aligned). */
 struct WsLayout {
   size_t status = 0;      /* uint32 device status word (first 256 bytes) */
@@ -88,6 +105,9 @@ bool debug_log();
 /* Launches carry programmatic stream serialization (see moe_set_pdl). */
 bool pdl_enabled();
 
+/* Count one successful kernel launch (see moe_kernel_launches). */
+void count_launch();
+
 /* Launch `kernel` on `stream`, with programmatic stream serialization when
  * pdl_enabled() (the kernel keeps the pdl_wait / pdl_trigger protocol of
  * moe_device.cuh), and an optional cluster of `cluster_x` CTAs. */
@@ -115,18 +135,23 @@ cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e == cudaSuccess) count_launch();
+  return e;
 }
 
 cudaError_t launch_route(const float* logits, int32_t* topk_idx, float* topk_gate, int64_t T, int E, int k,
                          uint32_t* status, cudaStream_t stream);
 
 /* fc_out non-null: a GEMM2 with the combine folded in follows (zero its counters, and
- * the output rows of tokens none of whose rows will arrive) */
+ * the output rows of tokens none of whose rows will arrive). early_x: x is written by
+ * nothing after the kernel before this call's first one (inside moe_layer: the router
+ * follows x's producer), so the one-pass kernel may load rows of x before its pdl_wait. */
 cudaError_t launch_dispatch(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const uint16_t* x,
                             const int32_t* topk_idx, int32_t* expert_counts, int32_t* expert_offsets,
                             int32_t* rank_counts, int32_t* rank_offsets, int32_t* row_src, int32_t* assign_row,
-                            uint16_t* x_perm, float* imbalance, cudaStream_t stream, uint16_t* fc_out = nullptr);
+                            uint16_t* x_perm, float* imbalance, cudaStream_t stream, uint16_t* fc_out = nullptr,
+                            bool early_x = false);
 
 /* The combine folded into GEMM2's epilogue for moe_layer (see moe_set_fused_combine). */
 bool fused_combine_enabled();

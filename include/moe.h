@@ -409,6 +409,25 @@ int moe_set_gemm_policy(int policy);
  * Process-wide, for calls made after this one; default 0. Returns the previous value. */
 int moe_set_fused_combine(int enable);
 
+/* Kernels this library has launched in this process so far, over every entry point
+ * and thread (successful launches only); the difference across a region of calls is
+ * the number of the library's kernels that region put on the GPU. */
+uint64_t moe_kernel_launches(void);
+
+/* Dispatch-path knob (moe_dispatch, moe_dispatch_static and the dispatch step of
+ * moe_layer; results are bit for bit the same on every path):
+ *   0 (default) = one pass when T*k <= 16384, the two-kernel path otherwise;
+ *   1 = two kernels: a histogram kernel whose last CTA scans the per-chunk counts,
+ *       then the permute kernel;
+ *   2 = one pass wherever it applies: a single kernel in which every CTA counts all
+ *       T*k expert ids itself (its reads grow with T*k), ranks its own contiguous
+ *       range of assignments and copies their rows.
+ * The one-pass kernel needs none of the workspace's scratch besides the status
+ * word; moe_layer with the combine folded into the down GEMM always takes the
+ * two-kernel path. Process-wide, for calls made after this one. Returns the
+ * previous value, or -1 for an unknown path (unchanged). */
+int moe_set_dispatch_path(int path);
+
 /* Launch-overlap knob: while enabled (the default, non-zero), every kernel the
  * library launches carries programmatic stream serialization (programmatic
  * dependent launch): it may be scheduled while the kernel before it in the

@@ -178,6 +178,21 @@ def test_status_strings_and_timeout_knob():
     assert lib.moe_set_test_stall(0) == 1
     assert lib.moe_set_pdl(0) == 1                                # on by default
     assert lib.moe_set_pdl(1) == 0
+    assert lib.moe_set_dispatch_path(moe.DISPATCH_ONE_PASS) == moe.DISPATCH_AUTO   # auto by default
+    assert lib.moe_set_dispatch_path(3) == -1
+    assert lib.moe_set_dispatch_path(moe.DISPATCH_TWO_PASS) == moe.DISPATCH_ONE_PASS
+    assert lib.moe_set_dispatch_path(moe.DISPATCH_AUTO) == moe.DISPATCH_TWO_PASS
+
+
+def test_rejected_calls_launch_nothing():
+    """moe_kernel_launches counts the library's launches; calls refused on the host add none."""
+    lib = moe.load()
+    before = lib.moe_kernel_launches()
+    bad = moe.Shape(T=16, d=100, E=8, k=2, f=128, R=2).c()          # d not a multiple of 128
+    assert lib.moe_route(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == moe.MOE_ERR_UNSUPPORTED
+    b = moe.moe_layer_buffers_t(*([FAKE] * len(moe.moe_layer_buffers_t._fields_)))
+    assert lib.moe_layer(ctypes.byref(bad), ctypes.byref(b), FAKE, 1 << 30, None) == moe.MOE_ERR_UNSUPPORTED
+    assert lib.moe_kernel_launches() == before
 
 
 def test_gathering_gemm_rejects_inputs_past_32_bit_row_offsets():

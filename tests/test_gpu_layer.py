@@ -341,3 +341,39 @@ def test_layer_is_bit_identical_with_and_without_launch_overlap(name):
         if a.dtype == torch.bfloat16:
             a, b = a.view(torch.int16), b.view(torch.int16)
         assert torch.equal(a, b), n
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen3_mixed", "dsv3_decode", "mixtral_prefill"])
+def test_layer_is_bit_identical_on_both_dispatch_paths(name):
+    """The one-pass dispatch kernel (which, inside moe_layer, loads rows of x before its
+    wait on the router) and the two-kernel path place the same rows: every output of
+    moe_layer is bit for bit the same, over two calls in a row, with the launch overlap
+    on and off."""
+    import torch
+    wl = moe_synth.workload(name)
+    dv = moe_synth.device_inputs(wl)
+    shape = _shape(wl)
+    names = ("topk_idx", "topk_gate", "expert_counts", "expert_offsets", "rank_counts", "rank_offsets", "row_src",
+             "assign_row", "x_perm", "y_perm", "out", "imbalance")
+    results = {}
+    old_path, old_pdl = moe.set_dispatch_path(moe.DISPATCH_AUTO), moe.set_pdl(True)
+    try:
+        for path in (moe.DISPATCH_TWO_PASS, moe.DISPATCH_ONE_PASS):
+            for pdl in (True, False):
+                moe.set_dispatch_path(path)
+                moe.set_pdl(pdl)
+                layer = moe.MoELayer(shape, dv["w13"], dv["w2"], dv.get("w13s"), dv.get("w2s"))
+                for _ in range(2):
+                    outs = layer(dv["logits"], dv["x"])
+                assert moe.get_status(layer.ws) == 0
+                results[(path, pdl)] = {n: outs[n].clone() for n in names}
+    finally:
+        moe.set_dispatch_path(old_path)
+        moe.set_pdl(old_pdl)
+    base = results[(moe.DISPATCH_TWO_PASS, True)]
+    for key, res in results.items():
+        for n in names:
+            a, b = base[n], res[n]
+            if a.dtype == torch.bfloat16:
+                a, b = a.view(torch.int16), b.view(torch.int16)
+            assert torch.equal(a, b), (key, n)

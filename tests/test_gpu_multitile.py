@@ -137,3 +137,80 @@ def test_mixtral_prefill_full_output_matches_oracle():
                        moe_synth.host_w2(wl), wl.k, wl.R)
     close(y_gpu, res["y_perm"], "y_perm mixtral_prefill (full)")
     close(out_gpu, res["out"], "out mixtral_prefill (full)")
+
+
+# ---------------------------------------------------------------------------
+# groups longer than one L2 band of m-tiles
+# ---------------------------------------------------------------------------
+
+BAND_BYTES = 24 << 20   # A rows per band of m-tiles (the kernels' tile order)
+
+
+def band_m_tiles(tm, K):
+    """m-tiles per band: the most whose A rows (tm rows x K bf16 each) fit BAND_BYTES."""
+    return max(1, BAND_BYTES // (tm * K * 2))
+
+
+BAND_CASES = {
+    # gate/up reduces over d = 7168: 13 single (6 pair) m-tiles per band; the shared
+    # expert's 4096 rows are 32 single (16 pair) m-tiles, 3 bands with a short last one
+    "gate_up_bands": moe_synth.Workload("band_g", T=4096, d=7168, E=8, k=2, f=256, R=4, n_shared=1,
+                                        bias_kind="zipf", zipf_s=1.0, seed=21),
+    # down reduces over f = 7168: the same band sizes in the down GEMM
+    "down_bands": moe_synth.Workload("band_d", T=4096, d=256, E=8, k=2, f=7168, R=4, n_shared=1,
+                                     bias_kind="zipf", zipf_s=1.0, seed=22),
+}
+
+
+def test_band_model_on_a_hand_count():
+    """24 MiB / (128 rows x 7168 x 2 bytes) = 13.7 -> 13 m-tiles per band; 256-row tiles: 6;
+    a K of 2048 gives 48; a group of 32 m-tiles in 13-tile bands runs as 13 + 13 + 6."""
+    assert band_m_tiles(128, 7168) == 13 and band_m_tiles(256, 7168) == 6
+    assert band_m_tiles(128, 2048) == 48
+    assert -(-32 // band_m_tiles(128, 7168)) == 3
+
+
+@functools.lru_cache(maxsize=None)
+def _oracle_band_case(name):
+    wl = BAND_CASES[name]
+    return oracle.layer(moe_synth.host_x(wl), moe_synth.host_logits(wl), moe_synth.host_w13(wl),
+                        moe_synth.host_w2(wl), wl.k, wl.R, moe_synth.host_w13s(wl), moe_synth.host_w2s(wl))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("policy", list(POLICIES))
+@pytest.mark.parametrize("case", list(BAND_CASES))
+def test_groups_spanning_several_bands_match_oracle(case, policy):
+    """The shared expert (and the largest routed experts) run their m-tiles in several
+    bands, the last one short, in one of the GEMMs: every element of y_perm, y_shared
+    and out against the oracle."""
+    import torch
+    wl = BAND_CASES[case]
+    res = _oracle_band_case(case)
+    tm = 128 if policy == "single" else 256
+    K = wl.d if case == "gate_up_bands" else wl.f
+    band = band_m_tiles(tm, K)
+    m_shared = _tiles(wl.T, tm)
+    assert m_shared >= 2 * band + 1 and m_shared % band != 0    # several bands, a short last one
+    shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, n_shared=1)
+    dv = moe_synth.device_inputs(wl)
+    old = moe.set_gemm_policy(POLICIES[policy])
+    try:
+        layer = moe.MoELayer(shape, dv["w13"], dv["w2"], dv["w13s"], dv["w2s"])
+        outs = layer(dv["logits"], dv["x"])
+        assert moe.get_status(layer.ws) == 0
+    finally:
+        moe.set_gemm_policy(old)
+    close(f64(bits(outs["y_shared"])), res["y_shared"], f"y_shared {case} {policy}")
+    off = res["expert_offsets"]
+    y = f64(bits(outs["y_perm"]))
+    for e in range(wl.E):
+        if off[e + 1] > off[e]:
+            close(y[off[e]:off[e + 1]], res["y_perm"][off[e]:off[e + 1]], f"y_perm expert {e} {case} {policy}")
+    close(f64(bits(outs["out"])), res["out"], f"out {case} {policy}")
+    # the shared expert's rows band by band, so that one misplaced band cannot hide
+    ys = f64(bits(outs["y_shared"]))
+    for b0 in range(0, wl.T, band * tm):
+        close(ys[b0:b0 + band * tm], res["y_shared"][b0:b0 + band * tm], f"y_shared band at row {b0} {case}")
+    del layer, outs, dv
+    torch.cuda.empty_cache()

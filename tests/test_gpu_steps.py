@@ -63,6 +63,16 @@ def _gpu_dispatch(shape, x_dev, idx_np):
     return o
 
 
+@pytest.fixture(params=[moe.DISPATCH_AUTO, moe.DISPATCH_TWO_PASS, moe.DISPATCH_ONE_PASS],
+                ids=["auto", "two_pass", "one_pass"])
+def dispatch_path(request):
+    """Every dispatch path must give the same bits: the two-kernel path (histogram, last
+    CTA's scan, permute) and the one-pass kernel (every CTA counts all ids itself)."""
+    old = moe.set_dispatch_path(request.param)
+    yield request.param
+    moe.set_dispatch_path(old)
+
+
 # ---------------------------------------------------------------------------
 # generator: device fill == host fill
 # ---------------------------------------------------------------------------
@@ -159,7 +169,7 @@ def _check_dispatch(o, ref, x_np=None, k=None):
 
 
 @pytest.mark.parametrize("name", WORKLOADS)
-def test_dispatch_matches_oracle(name):
+def test_dispatch_matches_oracle(name, dispatch_path):
     torch = _torch()
     wl = moe_synth.workload(name)
     shape = _shape(wl)
@@ -186,7 +196,7 @@ def test_dispatch_matches_oracle(name):
         assert np.array_equal(got, moe_synth.host_x(wl, toks))
 
 
-def test_dispatch_worked_imbalance_example():
+def test_dispatch_worked_imbalance_example(dispatch_path):
     counts = np.array([140, 95, 78, 62, 48, 40, 31, 18])
     experts = np.repeat(np.arange(8), counts)
     np.random.default_rng(7).shuffle(experts)
@@ -203,7 +213,7 @@ def test_dispatch_worked_imbalance_example():
 
 @pytest.mark.parametrize("T,E,k,R", [(0, 8, 2, 2), (1, 1, 1, 1), (1, 256, 8, 8), (1000, 37, 5, 1), (4099, 64, 3, 16),
                                      (2049, 8, 1, 4), (3000, 256, 8, 8)])
-def test_dispatch_edge_shapes(T, E, k, R):
+def test_dispatch_edge_shapes(T, E, k, R, dispatch_path):
     rng = np.random.default_rng(T + E)
     idx = rng.integers(0, E, size=(T, k)).astype(np.int32)   # repeats within a token allowed
     shape = moe.Shape(T=T, d=128, E=E, k=k, f=128, R=R)
@@ -215,7 +225,7 @@ def test_dispatch_edge_shapes(T, E, k, R):
         assert o["imbalance"].cpu().numpy().tolist() == [1.0, 1.0]
 
 
-def test_dispatch_out_of_range_entries_are_skipped_and_flagged():
+def test_dispatch_out_of_range_entries_are_skipped_and_flagged(dispatch_path):
     T, E, k = 300, 16, 2
     idx = np.random.default_rng(3).integers(0, E, size=(T, k)).astype(np.int32)
     idx[5, 1] = E
@@ -346,7 +356,7 @@ def test_expert_ffn_tail_sizes(rows, gemm_policy):
 
 @pytest.mark.parametrize("name,C", [("mixtral_prefill", 1.0), ("mixtral_prefill", 1.25), ("qwen3_mixed", 1.5),
                                     ("dsv3_skewed_prefill", 1.0), ("tiny", 2.0)])
-def test_dispatch_with_capacity_matches_oracle(name, C):
+def test_dispatch_with_capacity_matches_oracle(name, C, dispatch_path):
     wl = moe_synth.workload(name)
     cap = moe.capacity_for(C, wl.T, wl.k, wl.E)
     shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, capacity=cap)
@@ -400,7 +410,7 @@ def test_expert_ffn_gathering_rows_from_x(wl, gemm_policy):
     _ffn_gather_case(wl)
 
 
-def test_index_only_dispatch_equals_full_dispatch():
+def test_index_only_dispatch_equals_full_dispatch(dispatch_path):
     torch = _torch()
     wl = moe_synth.workload("qwen3_mixed")
     shape = _shape(wl)
@@ -448,7 +458,7 @@ def _random_dispatch_cases(n=24, seed=2024):
 
 
 @pytest.mark.parametrize("T,E,k,R,cap,seed", _random_dispatch_cases())
-def test_dispatch_random_shapes_bit_exact(T, E, k, R, cap, seed):
+def test_dispatch_random_shapes_bit_exact(T, E, k, R, cap, seed, dispatch_path):
     """Seeded random shapes (chunk boundaries, many or few experts, capacity drops) against the oracle."""
     torch = _torch()
     rng = np.random.default_rng(seed)

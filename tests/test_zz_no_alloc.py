@@ -12,9 +12,10 @@ one left behind) give exactly what moe_dispatch gives on the same inputs (bit
 for bit, the bar for integer and byte outputs), that the status output is
 per call, that a call is not thrown off by what an earlier call left in the
 array's header (a non-zero last-chunk ticket), that the largest workload (64
-histogram chunks) and the index-only form (x_perm NULL) match too, and that a
-shape needing more scratch than the array holds is refused before anything
-runs. The test only allocates the caller's own buffers.
+histogram chunks) and the index-only form (x_perm NULL) match too, that the
+one-pass and the two-kernel dispatch paths give the same bits through it, and
+that a shape needing more scratch than the array holds is refused before
+anything runs. The test only allocates the caller's own buffers.
 """
 import ctypes
 
@@ -54,10 +55,24 @@ def _static_call(shape, x, idx, b, status):
     assert rc == moe.MOE_OK, lib.moe_status_string(rc)
 
 
-def _reference_call(shape, x, idx, b):
-    ws = moe.new_workspace(shape)
-    moe.moe_dispatch(shape, x, idx, *(b[n] for n in OUTS), ws)
-    return moe.get_status(ws)
+def _reference_call(shape, x, idx, b, path=None):
+    """moe_dispatch with a workspace (on `path`, else the current dispatch path)."""
+    old = moe.set_dispatch_path(path) if path is not None else None
+    try:
+        ws = moe.new_workspace(shape)
+        moe.moe_dispatch(shape, x, idx, *(b[n] for n in OUTS), ws)
+        return moe.get_status(ws)
+    finally:
+        if old is not None:
+            moe.set_dispatch_path(old)
+
+
+@pytest.fixture
+def two_pass():
+    """The ticket tests run the two-kernel path (the one-pass kernel has no ticket)."""
+    old = moe.set_dispatch_path(moe.DISPATCH_TWO_PASS)
+    yield
+    moe.set_dispatch_path(old)
 
 
 def _scratch():
@@ -109,17 +124,24 @@ def _same(a, b):
         assert torch.equal(u, v), n
 
 
-def test_static_dispatch_matches_workspace_dispatch_on_two_calls_in_a_row():
+@pytest.mark.parametrize("path", ["auto", "two_pass", "one_pass"])
+def test_static_dispatch_matches_workspace_dispatch_on_two_calls_in_a_row(path):
+    """Static calls on each dispatch path against the workspace call on the two-kernel path."""
     import torch
     status = torch.full((1,), 0xFFFF, dtype=torch.int32, device="cuda")
     cases = [_case(moe_synth.workload("qwen3_mixed")), _case(moe_synth.workload("tiny"))]
-    for shape, x, idx in cases:
-        got, want = _buffers(shape), _buffers(shape)
-        _static_call(shape, x, idx, got, status)
-        ref_status = _reference_call(shape, x, idx, want)
-        torch.cuda.synchronize()
-        _same(got, want)
-        assert int(status.item()) == ref_status == 0
+    p = {"auto": moe.DISPATCH_AUTO, "two_pass": moe.DISPATCH_TWO_PASS, "one_pass": moe.DISPATCH_ONE_PASS}[path]
+    old = moe.set_dispatch_path(p)
+    try:
+        for shape, x, idx in cases:
+            got, want = _buffers(shape), _buffers(shape)
+            _static_call(shape, x, idx, got, status)
+            ref_status = _reference_call(shape, x, idx, want, moe.DISPATCH_TWO_PASS)
+            torch.cuda.synchronize()
+            _same(got, want)
+            assert int(status.item()) == ref_status == 0
+    finally:
+        moe.set_dispatch_path(old)
 
 
 def test_static_dispatch_reports_per_call_status_and_refuses_oversized_shapes():
@@ -153,7 +175,7 @@ def _chunks(shape):
     return -(-shape.T // per)
 
 
-def test_static_dispatch_ignores_a_stale_ticket_and_status_left_in_the_header():
+def test_static_dispatch_ignores_a_stale_ticket_and_status_left_in_the_header(two_pass):
     """A call that was interrupted or raced could leave the last-chunk ticket and the
     status word non-zero; the next call zeroes the header first and is still exact."""
     import torch
@@ -172,7 +194,7 @@ def test_static_dispatch_ignores_a_stale_ticket_and_status_left_in_the_header():
     assert hdr[16] == 0 and hdr[0] == 0                        # ticket back at zero, no status bits
 
 
-def test_static_dispatch_three_then_two_chunks_leaves_the_ticket_at_zero():
+def test_static_dispatch_three_then_two_chunks_leaves_the_ticket_at_zero(two_pass):
     import torch
     status = torch.zeros((1,), dtype=torch.int32, device="cuda")
     for T in (768, 512):                                      # k = 8: 3 chunks, then 2
