@@ -13,6 +13,8 @@
  *
  * Bytes per token: k*d*2 + (shared) d*2 read, d*2 written, k*8 of indices.
  */
+#include <algorithm>
+
 #include "moe_device.cuh"
 
 namespace moe {
@@ -30,8 +32,9 @@ struct EpSource {
 
 /* U vectors per lane per step, rows of up to KMAX experts in flight together.
  * Local form: rows come from y_perm (A rows). EP form: from the owners' buffers
- * (ep; A is then the rows each of them holds). */
-template <int U, int KMAX, bool EP>
+ * (ep; A is then the rows each of them holds). SH: a shared-expert row is added
+ * (y_shared non-null); without it the kernel holds fewer registers. */
+template <int U, int KMAX, bool EP, bool SH>
 __global__ void __launch_bounds__(256, 2) combine_kernel(const uint16_t* __restrict__ y_perm,
                                                       const int32_t* __restrict__ assign_row,
                                                       const float* __restrict__ topk_gate,
@@ -81,11 +84,11 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(const uint16_t* __restr
       const uint16_t* base = EP ? ep.y_rows[o] : y_perm;
       src[j] = (j < k && r >= 0) ? base + (int64_t)r * d : nullptr;
     }
-    const uint16_t* ysh = y_shared ? y_shared + t * d : nullptr;
+    const uint16_t* ysh = SH ? y_shared + t * d : nullptr;
     uint16_t* o = out + t * d;
     for (int v0 = sl * vps + lane; v0 < v_end; v0 += 32 * U) {
       uint4 wv[KMAX][U];
-      uint4 sv[U];
+      uint4 sv[SH ? U : 1];
 #pragma unroll
       for (int j = 0; j < KMAX; ++j)
 #pragma unroll
@@ -93,10 +96,12 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(const uint16_t* __restr
           const int v = v0 + 32 * u;
           wv[j][u] = (src[j] != nullptr && v < v_end) ? ld_nc_v4(src[j] + (int64_t)v * 8) : make_uint4(0, 0, 0, 0);
         }
+      if (SH) {
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int v = v0 + 32 * u;
-        sv[u] = (ysh && v < v_end) ? ld_nc_v4(ysh + (int64_t)v * 8) : make_uint4(0, 0, 0, 0);
+        for (int u = 0; u < U; ++u) {
+          const int v = v0 + 32 * u;
+          sv[SH ? u : 0] = v < v_end ? ld_nc_v4(ysh + (int64_t)v * 8) : make_uint4(0, 0, 0, 0);
+        }
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -113,8 +118,9 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(const uint16_t* __restr
             acc[2 * q + 1] = fmaf(gs[j], bf16hi(ww[q]), acc[2 * q + 1]);
           }
         }
-        if (ysh) {
-          const uint32_t ss[4] = {sv[u].x, sv[u].y, sv[u].z, sv[u].w};
+        if (SH) {
+          const uint4 q4 = sv[SH ? u : 0];
+          const uint32_t ss[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             acc[2 * q] += bf16lo(ss[q]);
@@ -139,9 +145,13 @@ cudaError_t launch_combine(const moe_shape_t& s, const uint16_t* y_perm, const i
   if (s.T == 0) return cudaSuccess;
   const RowSlices rs = row_slices(s.T, s.d);
   const int64_t A = (int64_t)s.T * s.k;
-  auto kernel = s.k <= 2 ? combine_kernel<4, 2, false>
-                         : (s.k <= 4 ? combine_kernel<2, 4, false> : combine_kernel<1, 8, false>);
-  return launch_kernel(kernel, dim3((unsigned)rs.blocks), dim3(256), 0, stream, 1, y_perm, assign_row, topk_gate,
+  auto kernel = y_shared ? (s.k <= 2 ? combine_kernel<4, 2, false, true>
+                                     : (s.k <= 4 ? combine_kernel<2, 4, false, true> : combine_kernel<1, 8, false, true>))
+                         : (s.k <= 2 ? combine_kernel<4, 2, false, false>
+                                     : (s.k <= 4 ? combine_kernel<2, 4, false, false> : combine_kernel<1, 8, false, false>));
+  /* one wave of CTAs (the warps loop over their items) */
+  const int blocks = std::min(rs.blocks, resident_blocks(reinterpret_cast<const void*>(kernel), 256));
+  return launch_kernel(kernel, dim3((unsigned)blocks), dim3(256), 0, stream, 1, y_perm, assign_row, topk_gate,
                        y_shared, out, (int64_t)s.T, s.d, s.k, A, rs.slices, rs.vps, status,
                        early_index_reads ? 1 : 0, EpSource{});
 }
@@ -155,8 +165,10 @@ cudaError_t launch_ep_combine(const moe_shape_t& s, uint16_t* const* y_rows, int
   ep.y_rows = y_rows;
   ep.topk_idx = topk_idx;
   ep.experts_per_rank = experts_per_rank;
-  auto kernel = s.k <= 2 ? combine_kernel<4, 2, true>
-                         : (s.k <= 4 ? combine_kernel<2, 4, true> : combine_kernel<1, 8, true>);
+  auto kernel = y_shared ? (s.k <= 2 ? combine_kernel<4, 2, true, true>
+                                     : (s.k <= 4 ? combine_kernel<2, 4, true, true> : combine_kernel<1, 8, true, true>))
+                         : (s.k <= 2 ? combine_kernel<4, 2, true, false>
+                                     : (s.k <= 4 ? combine_kernel<2, 4, true, false> : combine_kernel<1, 8, true, false>));
   return launch_kernel(kernel, dim3((unsigned)rs.blocks), dim3(256), 0, stream, 1, (const uint16_t*)nullptr, send_row,
                        topk_gate, y_shared, out, (int64_t)s.T, s.d, s.k, rows_cap, rs.slices, rs.vps, status, 0, ep);
 }

@@ -167,11 +167,13 @@ __device__ __forceinline__ bool build_schedule(const FfnParams& p, int32_t* s_of
   return __all_sync(0xFFFFFFFFu, ok);
 }
 
-/* Tile order inside a group: bands of consecutive m-tiles whose A rows take at most
- * kBandBytes; inside a band the m-tiles are the inner index. So the tiles running at
- * once share their weight tile, and a band's A rows stay in L2 while every weight
- * column tile passes over them; a group with more rows than one band (a shared expert
- * over a long batch) then reads its A rows from DRAM once, not once per column tile. */
+/* Tile order inside a group: the m-tiles are the inner index, so the tiles running
+ * at once share their weight tile and the group's A rows are re-read from L2 by every
+ * weight column tile. A group whose A rows outnumber its weight rows (a shared expert
+ * over a long batch) runs its m-tiles in bands of at most kBandBytes of A rows instead,
+ * m-tiles inner inside a band: a band's rows stay in L2 while every column tile passes
+ * over them, so the group's A rows come from DRAM once, and its (smaller) weights once
+ * per band. */
 constexpr int64_t kBandBytes = int64_t(24) << 20;
 
 /* Linear tile index -> tile (groups in order; bands of m-tiles inside a group). */
@@ -194,8 +196,8 @@ __device__ __forceinline__ Tile decode_tile(int64_t L, const FfnParams& p, const
   const int local = (int)(L - (int64_t)s_mpref[lo] * p.n_tiles_n);
   const bool shared = lo >= p.E;
   const int rows = shared ? (int)p.T : s_off[lo + 1] - s_off[lo];
-  const int64_t band_bytes = (int64_t)TM * p.K * 2;
-  const int band = (int)max((int64_t)1, kBandBytes / band_bytes);
+  const int w_rows = p.n_tiles_n * (MODE == 0 ? 256 : BN); /* weight rows of a group */
+  const int band = rows > w_rows ? (int)max((int64_t)1, kBandBytes / ((int64_t)TM * p.K * 2)) : mt;
   const int b = local / (band * p.n_tiles_n);         /* band of this tile */
   const int r = local - b * band * p.n_tiles_n;       /* index inside the band */
   const int gm = min(band, mt - b * band);             /* m-tiles in this band */

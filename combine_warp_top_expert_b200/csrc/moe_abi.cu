@@ -5,6 +5,8 @@
  * allocates no memory and holds no per-call state.
  */
 #include <atomic>
+#include <mutex>
+#include <vector>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -111,6 +113,28 @@ int num_sms() {
     cache[slot].store(n, std::memory_order_relaxed);
   }
   return n;
+}
+
+int resident_blocks(const void* kernel, int threads) {
+  struct Entry {
+    int dev;
+    const void* kernel;
+    int threads;
+    int blocks;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry& e : cache)
+    if (e.dev == dev && e.kernel == kernel && e.threads == threads) return e.blocks;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  const int blocks = per_sm * num_sms();
+  cache.push_back(Entry{dev, kernel, threads, blocks});
+  return blocks;
 }
 
 uint64_t wait_timeout_ns() { return g_wait_timeout_ns.load(std::memory_order_relaxed); }

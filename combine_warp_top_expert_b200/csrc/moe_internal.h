@@ -37,6 +37,10 @@ struct RowSlices {
 };
 RowSlices row_slices(int64_t T, int d);
 
+/* CTAs of `kernel` (block of `threads`, no dynamic shared memory) that fit on the
+ * current device at once: SMs x resident blocks per SM (cached per device and kernel). */
+int resident_blocks(const void* kernel, int threads);
+
 /* Dispatch path (see moe_set_dispatch_path). */
 constexpr int kDispatchAuto = 0;     /* one pass when A <= kOnePassAutoMaxA, else two kernels */
 constexpr int kDispatchTwoPass = 1;  /* histogram/scan kernel, then the permute kernel */
