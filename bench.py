@@ -60,6 +60,10 @@ def algorithmic(wl, counts):
     return w
 
 
+NOMINAL_BF16_TFLOPS = 2250.0  # dense bf16 tensor peak of a B200 (data sheet, without sparsity)
+NOMINAL_HBM_GBS = 8000.0      # HBM3e bandwidth of a B200 (data sheet)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -190,7 +194,7 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
+        sm, mx, pw, reasons = [], [], [], set()
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
@@ -201,13 +205,17 @@ class ClockSampler:
                 mx.append(float(parts[1]))
             except ValueError:
                 continue
+            try:
+                pw.append(float(parts[2]))
+            except ValueError:
+                pass
             for n, v in zip(names, parts[4:8]):
                 if v.lower() == "active":
                     reasons.add(n)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "power_w_median": statistics.median(pw) if pw else None, "samples": len(sm)}
 
 
 # ---------------------------------------------------------------------------
@@ -405,10 +413,12 @@ def run_gpu(args, wl, rank, world, local_rank):
     # roofline of each step and of the layer
     roof = {}
     t_roof = 0.0
+    t_roof_nominal = 0.0
     for n in names:
         b = work[n]["bytes"] / (peaks["hbm"] * 1e9)
         fl = work[n]["flops"] / (peaks["bf16"] * 1e12)
         t_roof += max(b, fl)
+        t_roof_nominal += max(work[n]["bytes"] / (NOMINAL_HBM_GBS * 1e9), work[n]["flops"] / (NOMINAL_BF16_TFLOPS * 1e12))
         roof[n] = dict(ms=kern_ms[n], bound="tensor" if fl > b else "hbm",
                        achieved=(work[n]["flops"] / (kern_ms[n] * 1e-3) / 1e12) if fl > b
                        else (work[n]["bytes"] / (kern_ms[n] * 1e-3) / 1e9),
@@ -431,6 +441,7 @@ def run_gpu(args, wl, rank, world, local_rank):
                    "experts_active": work["_n_act"], "imbalance_rank_expert": imbalance,
                    "expert_counts": counts,
                    "layer_roofline_frac": t_roof / (max_ms / args.steps / 1e3),
+                   "layer_roofline_frac_nominal": t_roof_nominal / (max_ms / args.steps / 1e3),
                    "per_step_ms": {n: round(v, 4) for n, v in kern_ms.items()},
                    "per_step_split": "a second pass of K steps through the five entry points, CUDA events "
                                      f"between calls ({split_ms:.4f} ms per step in that pass)",
@@ -441,6 +452,10 @@ def run_gpu(args, wl, rank, world, local_rank):
                      "unit": "TFLOP/s" if d["bound"] == "tensor" else "GB/s",
                      "frac": d["achieved"] / (peaks["bf16"] if d["bound"] == "tensor" else peaks["hbm"]),
                      "peak_kind": f"{peaks['source']} burst",
+                     # context: the same against the sustained (power-capped) GEMM figure, for a kernel
+                     # timed inside long steps, and against the nominal data-sheet peaks
+                     "frac_sustained": d["achieved"] / peaks["bf16_sustained"] if d["bound"] == "tensor" else None,
+                     "frac_nominal": d["achieved"] / (NOMINAL_BF16_TFLOPS if d["bound"] == "tensor" else NOMINAL_HBM_GBS),
                      "traffic": recorded_traffic(wl.name, f"moe_expert_{dom}")
                      if args.tokens is None and args.seed is None else None},
         "clocks": clocks.summary(),
@@ -511,6 +526,61 @@ def run_dense_compare(args):
         print(json.dumps(line), flush=True)
         del dv, ws, y, h
         torch.cuda.empty_cache()
+
+
+def run_sustain(args, wl):
+    """--sustain S: the workload's moe_layer back to back for about S seconds (L2 flushed
+    before every call, as in the timed region), nvidia-smi sampling SM clock and board power
+    every 100 ms. Prints per-window throughput with the clock and power seen in that window,
+    and the steady state (second half): what the layer sustains under the board's power
+    limit, against the short bursts of the timed region."""
+    import torch
+
+    import combine_warp_top_expert_b200 as moe
+    import moe_synth
+    dv = moe_synth.device_inputs(wl)
+    shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, n_shared=wl.n_shared)
+    layer = moe.MoELayer(shape, dv["w13"], dv["w2"], dv.get("w13s"), dv.get("w2s"))
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    for _ in range(args.warmup):
+        flush.zero_()
+        layer(dv["logits"], dv["x"])
+    torch.cuda.synchronize()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    smi_index = vis.split(",")[0].strip() if vis else "0"
+    windows = []  # (host time at the window's end, calls, summed layer ms)
+    t_start = time.perf_counter()
+    with ClockSampler(smi_index) as clocks:
+        while time.perf_counter() - t_start < args.sustain:
+            evs = [(ev(), ev()) for _ in range(25)]
+            for a, b in evs:
+                flush.zero_()
+                a.record()
+                layer(dv["logits"], dv["x"])
+                b.record()
+            torch.cuda.synchronize()
+            windows.append((time.perf_counter() - t_start, len(evs), sum(a.elapsed_time(b) for a, b in evs)))
+    t_samples = [i * 0.1 for i in range(len(clocks.lines))]  # sampler period
+    samples = []
+    for t, ln in zip(t_samples, clocks.lines):
+        parts = [p.strip() for p in ln.split(",")]
+        try:
+            samples.append((t, float(parts[0]), float(parts[2])))
+        except (ValueError, IndexError):
+            continue
+    half = [w for w in windows if w[0] >= args.sustain / 2] or windows
+    ms_steady = sum(w[2] for w in half) / sum(w[1] for w in half)
+    steady_s = [x for x in samples if x[0] >= args.sustain / 2 + 0.3] or samples
+    out = {"sustain": {
+        "workload": wl.name, "seconds": round(windows[-1][0], 2) if windows else 0.0, "calls": sum(w[1] for w in windows),
+        "first_window_ms_per_call": round(windows[0][2] / windows[0][1], 4) if windows else None,
+        "steady_ms_per_call": round(ms_steady, 4), "steady_tokens_per_s": round(wl.T / (ms_steady * 1e-3)),
+        "steady_sm_mhz": statistics.median(x[1] for x in steady_s) if steady_s else None,
+        "steady_power_w": statistics.median(x[2] for x in steady_s) if steady_s else None,
+        "clocks": clocks.summary(), "device_status": moe.get_status(layer.ws),
+        "note": "L2 flushed before every call; per-call CUDA events; nvidia-smi every 100 ms"}}
+    print(json.dumps(out), flush=True)
 
 
 # ---------------------------------------------------------------------------
@@ -734,6 +804,9 @@ def main():
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism across the --gpus ranks (E/R experts per GPU, rows exchanged over "
                          "NVLink inside dispatch and combine) instead of independent replicas")
+    ap.add_argument("--sustain", type=float, default=0.0,
+                    help="run the layer back to back for this many seconds, sampling SM clock and board power, "
+                         "and report the steady-state throughput (one GPU)")
     ap.add_argument("--rank-check", action="store_true",
                     help="start the ranks, join a gloo process group, print one line per rank and exit (no GPU)")
     args = ap.parse_args()
@@ -767,6 +840,9 @@ def main():
 
     if args.rank_check:
         rank_check(args, rank, world)
+        return
+    if args.sustain:
+        run_sustain(args, wl)
         return
     if args.impl == "reference":
         run_reference(args, wl, rank, world)
