@@ -546,7 +546,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     ffn_gemm_single_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                            const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
                            const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
-                           const FfnParams p) {
+                           const __grid_constant__ CUtensorMap tmA0r16, const __grid_constant__ CUtensorMap tmA0r32,
+                           const __grid_constant__ CUtensorMap tmA0r64, const FfnParams p) {
   using C = SingleCfg<MODE, BN>;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -658,14 +659,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool shared = t.g >= p.E;
       if constexpr (!GATHER) {
         /* TMA tiles, lane 0 only */
-        const CUtensorMap* mA = shared ? &tmA1 : &tmA0;
+        /* A routed group's last tile of at most 16, 32 or 64 real rows loads a box of
+         * that many rows of A: the rows past it keep what an earlier tile left in the
+         * stage, and their accumulator rows are never stored (GEMM1: h padding rows,
+         * which GEMM2 computes on but never stores either) */
+        const int a_rows =
+            shared ? 128 : (t.valid <= 16 ? 16 : (t.valid <= 32 ? 32 : (t.valid <= 64 ? 64 : 128)));
+        const CUtensorMap* mA = shared ? &tmA1
+                                       : (a_rows == 16 ? &tmA0r16
+                                                       : (a_rows == 32 ? &tmA0r32 : (a_rows == 64 ? &tmA0r64 : &tmA0)));
         const CUtensorMap* mB = shared ? &tmB1 : &tmB0;
+        const uint32_t stage_tx = (uint32_t)a_rows * (BK * 2) + C::B_BYTES;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, p.timeout_ns, s_abort)) {
             abort = true;
             break;
           }
-          mbar_arrive_expect_tx(&ctl->full[stage], C::STAGE_BYTES);
+          mbar_arrive_expect_tx(&ctl->full[stage], stage_tx);
           if (p.stall_first_stage && first && kb == 0) {
             /* test hook: this stage's bytes never arrive, so the MMA's bounded wait runs out */
             if (++stage == STAGES) {
@@ -1235,13 +1245,15 @@ cudaError_t smem_opt_in(std::atomic<int> (&done)[kMaxDevices], Kernel kernel, si
 
 template <int MODE, int BN, bool GATHER = false>
 cudaError_t launch_single(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0, const CUtensorMap& b1,
-                          const CUtensorMap& o0, const CUtensorMap& o1, const FfnParams& p, cudaStream_t stream) {
+                          const CUtensorMap& o0, const CUtensorMap& o1, const CUtensorMap& a0r16,
+                          const CUtensorMap& a0r32, const CUtensorMap& a0r64, const FfnParams& p,
+                          cudaStream_t stream) {
   using C = SingleCfg<MODE, BN>;
   static std::atomic<int> attr_done[kMaxDevices];
   const cudaError_t attr_err = smem_opt_in(attr_done, ffn_gemm_single_kernel<MODE, BN, GATHER>, C::SMEM_BYTES);
   if (attr_err != cudaSuccess) return attr_err;
   return launch_kernel(ffn_gemm_single_kernel<MODE, BN, GATHER>, dim3((unsigned)num_sms()), dim3(kThreads),
-                       C::SMEM_BYTES, stream, 1, a0, a1, b0, b1, o0, o1, p);
+                       C::SMEM_BYTES, stream, 1, a0, a1, b0, b1, o0, o1, a0r16, a0r32, a0r64, p);
 }
 
 /* Number of CTA pairs that can be resident at once (per device, cached). */
@@ -1360,8 +1372,12 @@ cudaError_t launch_gate_up(const moe_shape_t& s, const WsLayout& L, uint8_t* ws,
   }
   if (!make_map(&b0, w13, b_rows, s.d, 128) || !make_map(&b1, b_sh, b_sh_rows, s.d, 128))
     return cudaErrorInvalidValue;
-  return gather ? launch_single<0, 256, true>(a0, a1, b0, b1, o0, o0, p, stream)
-                : launch_single<0, 256>(a0, a1, b0, b1, o0, o0, p, stream);
+  if (gather) return launch_single<0, 256, true>(a0, a1, b0, b1, o0, o0, a0, a0, a0, p, stream);
+  CUtensorMap a0r16, a0r32, a0r64; /* short A boxes for a group's last tile of <= 16 / 32 / 64 rows */
+  if (!make_map(&a0r16, a_routed, a_rows, s.d, 16) || !make_map(&a0r32, a_routed, a_rows, s.d, 32) ||
+      !make_map(&a0r64, a_routed, a_rows, s.d, 64))
+    return cudaErrorInvalidValue;
+  return launch_single<0, 256>(a0, a1, b0, b1, o0, o0, a0r16, a0r32, a0r64, p, stream);
 }
 
 cudaError_t launch_down(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, const int32_t* expert_offsets,
@@ -1406,8 +1422,13 @@ cudaError_t launch_down(const moe_shape_t& s, const WsLayout& L, uint8_t* ws, co
     if (e != cudaSuccess || launched) return e;
   }
   if (!make_map(&b0, w2, b_rows, s.f, bn) || !make_map(&b1, b_sh, b_sh_rows, s.f, bn)) return cudaErrorInvalidValue;
-  return bn256 ? launch_single<1, 256>(a0, a0, b0, b1, o0, o1, p, stream)
-               : launch_single<1, 128>(a0, a0, b0, b1, o0, o1, p, stream);
+  CUtensorMap a0r16, a0r32, a0r64; /* short A boxes (rows of h) for a group's last tile of <= 16 / 32 / 64 rows */
+  if (!make_map(&a0r16, ws + L.h, (uint64_t)L.h_rows, s.f, 16) ||
+      !make_map(&a0r32, ws + L.h, (uint64_t)L.h_rows, s.f, 32) ||
+      !make_map(&a0r64, ws + L.h, (uint64_t)L.h_rows, s.f, 64))
+    return cudaErrorInvalidValue;
+  return bn256 ? launch_single<1, 256>(a0, a0, b0, b1, o0, o1, a0r16, a0r32, a0r64, p, stream)
+               : launch_single<1, 128>(a0, a0, b0, b1, o0, o1, a0r16, a0r32, a0r64, p, stream);
 }
 
 }  // namespace moe
