@@ -412,13 +412,15 @@ __device__ __forceinline__ void fused_combine_warp(const FfnParams& p, const Til
  * addresses the warp's TMEM lane quarter at the accumulator's first column; `row0`
  * is the warp's first row inside the tile (this thread's row is row0 + lane).
  * GEMM1: the accumulator holds gate in columns [0, 128) and up in [128, 256); h =
- *        silu(gate) * up, 128 columns, always stored (h is padded), as two blocks.
+ *        silu(gate) * up, 128 columns, stored as two blocks by every warp holding a real
+ *        row (the rest of a 32-row block is h padding).
  * GEMM2: BN columns, BN / 64 blocks, masked to the group's real rows. */
 template <int MODE, int BN>
 __device__ __forceinline__ void epilogue_warp(const FfnParams& p, const Tile& t, uint32_t taddr, int row0, int lane,
                                               uint8_t* stage, const CUtensorMap* out0, const CUtensorMap* out1) {
   const int32_t grow = (int32_t)(t.out_row + row0); /* output row of lane 0 */
   if (MODE == 0) {
+    if (row0 >= t.valid) return; /* no real row in this warp's 32: its h rows are padding, never read as results */
 #pragma unroll 1
     for (int j = 0; j < 2; ++j) epi_swiglu_block(taddr, j * 64, 128 + j * 64, stage, out0, t.n * 128 + j * 64, grow, lane);
   } else {
