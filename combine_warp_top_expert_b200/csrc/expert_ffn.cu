@@ -424,6 +424,7 @@ __device__ __forceinline__ void epilogue_warp(const FfnParams& p, const Tile& t,
 #pragma unroll 1
     for (int j = 0; j < 2; ++j) epi_swiglu_block(taddr, j * 64, 128 + j * 64, stage, out0, t.n * 128 + j * 64, grow, lane);
   } else {
+    if (row0 >= t.valid) return; /* no real row in this warp's 32: nothing to store or count */
     const bool shared = t.g >= p.E;
     const CUtensorMap* map = shared ? out1 : out0;
     const bool whole = row0 + 32 <= t.valid; /* warp-uniform */
