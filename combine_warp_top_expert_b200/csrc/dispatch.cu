@@ -569,7 +569,10 @@ OnePass onepass_plan(const moe_shape_t& s, bool index_only) {
     rs.vps = s.d / 8;
   }
   const int64_t items = (int64_t)s.T * rs.slices;
-  const int64_t max_blocks = (int64_t)num_sms() * 2;
+  /* one CTA per SM: every CTA counts all A ids, so fewer CTAs do less of that; 16
+   * warps per SM keep enough row copies in flight (two CTAs per SM measured ~1 us slower
+   * per call on 100 MB) */
+  const int64_t max_blocks = (int64_t)num_sms();
   int64_t blocks = (items + kOnePassWarps - 1) / kOnePassWarps;
   if (blocks > max_blocks) blocks = max_blocks;
   if (blocks < 1) blocks = 1;
