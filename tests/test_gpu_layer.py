@@ -281,15 +281,22 @@ def _random_layer_cases(n=12, seed=77):
     return cases
 
 
+@pytest.mark.parametrize("policy", [moe.GEMM_AUTO, moe.GEMM_SINGLE, moe.GEMM_PAIR], ids=["auto", "single", "pair"])
 @pytest.mark.parametrize("wl,cf", _random_layer_cases(), ids=[c[0].name for c in _random_layer_cases()])
-def test_layer_random_shapes_match_oracle(wl, cf):
-    """Seeded random shapes through the whole layer (default tile policy) against the oracle."""
+def test_layer_random_shapes_match_oracle(wl, cf, policy):
+    """Seeded random shapes through the whole layer, under each tile policy, against the oracle
+    (ragged groups of every size exercise the short A boxes of single-CTA tiles and the
+    half-height pair tiles)."""
     cap = moe.capacity_for(cf, wl.T, wl.k, wl.E) if cf else 0
     shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, n_shared=wl.n_shared, capacity=cap)
     dv = moe_synth.device_inputs(wl)
-    layer = moe.MoELayer(shape, dv["w13"], dv["w2"], dv.get("w13s"), dv.get("w2s"))
-    outs = layer(dv["logits"], dv["x"])
-    assert moe.get_status(layer.ws) == 0
+    old = moe.set_gemm_policy(policy)
+    try:
+        layer = moe.MoELayer(shape, dv["w13"], dv["w2"], dv.get("w13s"), dv.get("w2s"))
+        outs = layer(dv["logits"], dv["x"])
+        assert moe.get_status(layer.ws) == 0
+    finally:
+        moe.set_gemm_policy(old)
     res = oracle.layer(moe_synth.host_x(wl), moe_synth.host_logits(wl), moe_synth.host_w13(wl),
                        moe_synth.host_w2(wl), wl.k, wl.R, moe_synth.host_w13s(wl) if wl.n_shared else None,
                        moe_synth.host_w2s(wl) if wl.n_shared else None, capacity=cap)
