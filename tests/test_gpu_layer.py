@@ -384,3 +384,43 @@ def test_layer_is_bit_identical_on_both_dispatch_paths(name):
             if a.dtype == torch.bfloat16:
                 a, b = a.view(torch.int16), b.view(torch.int16)
             assert torch.equal(a, b), (key, n)
+
+
+@pytest.mark.parametrize("policy", [moe.GEMM_SINGLE, moe.GEMM_PAIR], ids=["single", "pair"])
+@pytest.mark.parametrize("fused", [False, True], ids=["combine", "fused_combine"])
+def test_stale_workspace_contents_never_reach_a_result(policy, fused):
+    """Padding rows of h, the rows a short A box leaves in a pipeline stage, and every other
+    scratch row past a group's real rows are computed on but never stored as results. With
+    everything in the workspace past its 256-byte header (which holds the zeroed counters)
+    set to 0xFF bytes (NaN in every bf16 of h) the layer gives the same bits as on a zeroed
+    workspace, two calls in a row, on a batch of many one-tile groups and a few long ones."""
+    import torch
+    wl = moe_synth.Workload("stale", T=320, d=512, E=48, k=6, f=384, R=4, n_shared=1, bias_kind="zipf",
+                            zipf_s=1.3, seed=31)
+    shape = _shape(wl)
+    dv = moe_synth.device_inputs(wl)
+    names = ("topk_idx", "topk_gate", "expert_offsets", "row_src", "assign_row", "x_perm", "y_perm", "y_shared",
+             "out")
+    old_p, old_f = moe.set_gemm_policy(policy), moe.set_fused_combine(fused)
+    try:
+        results = []
+        for fill in (0x00, 0xFF):
+            layer = moe.MoELayer(shape, dv["w13"], dv["w2"], dv["w13s"], dv["w2s"])
+            layer.ws[256:].fill_(fill)
+            for _ in range(2):
+                outs = layer(dv["logits"], dv["x"])
+            torch.cuda.synchronize()
+            assert moe.get_status(layer.ws) == 0
+            results.append({n: outs[n].clone() for n in names})
+    finally:
+        moe.set_gemm_policy(old_p)
+        moe.set_fused_combine(old_f)
+    A = int(results[0]["expert_offsets"][-1])
+    for n in names:
+        a, b = results[0][n], results[1][n]
+        if n in ("x_perm", "y_perm"):
+            a, b = a[:A], b[:A]
+        if a.dtype == torch.bfloat16:
+            assert not torch.isnan(b.float()).any(), n
+            a, b = a.view(torch.int16), b.view(torch.int16)
+        assert torch.equal(a, b), n
