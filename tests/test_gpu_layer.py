@@ -424,3 +424,29 @@ def test_stale_workspace_contents_never_reach_a_result(policy, fused):
             assert not torch.isnan(b.float()).any(), n
             a, b = a.view(torch.int16), b.view(torch.int16)
         assert torch.equal(a, b), n
+
+
+def test_the_launch_counter_counts_each_kernel_of_a_layer_call():
+    """moe_kernel_launches (the bench's `gpu_launches`): one moe_layer call launches route,
+    dispatch (one kernel for T*k <= 16384, else histogram + permute), gate/up, down and
+    combine; with the combine folded into the down GEMM the combine kernel is not launched
+    (and dispatch takes its two-kernel form)."""
+    import torch
+    wl = moe_synth.workload("tiny")
+    dv = moe_synth.device_inputs(wl)
+    layer = moe.MoELayer(_shape(wl), dv["w13"], dv["w2"])
+    cases = [(moe.DISPATCH_AUTO, False, 5), (moe.DISPATCH_ONE_PASS, False, 5), (moe.DISPATCH_TWO_PASS, False, 6),
+             (moe.DISPATCH_AUTO, True, 5)]
+    old_p, old_f = moe.set_dispatch_path(moe.DISPATCH_AUTO), moe.set_fused_combine(False)
+    try:
+        for path, fused, want in cases:
+            moe.set_dispatch_path(path)
+            moe.set_fused_combine(fused)
+            before = moe.kernel_launches()
+            layer(dv["logits"], dv["x"])
+            assert moe.kernel_launches() - before == want, (path, fused)
+        torch.cuda.synchronize()
+        assert moe.get_status(layer.ws) == 0
+    finally:
+        moe.set_dispatch_path(old_p)
+        moe.set_fused_combine(old_f)
