@@ -450,3 +450,46 @@ def test_the_launch_counter_counts_each_kernel_of_a_layer_call():
     finally:
         moe.set_dispatch_path(old_p)
         moe.set_fused_combine(old_f)
+
+
+def _soak_cases(n=40, seed=2026):
+    """Seeded random layers, each with a random tile policy, dispatch path and combine form."""
+    rng = np.random.default_rng(seed)
+    cases = []
+    for i in range(n):
+        E = int(rng.integers(1, 65))
+        k = int(rng.integers(1, min(E, 8) + 1))
+        R = int(rng.choice([r for r in range(1, E + 1) if E % r == 0]))
+        wl = moe_synth.Workload(f"soak{i}", T=int(rng.integers(1, 1500)), d=int(rng.choice([128, 256, 384, 512, 768])),
+                                E=E, k=k, f=int(rng.choice([128, 256, 384, 512])), R=R,
+                                n_shared=int(rng.integers(0, 2)), bias_kind="zipf",
+                                zipf_s=float(rng.uniform(0.0, 1.6)), seed=5000 + i)
+        cases.append((wl, float(rng.choice([0.0, 0.0, 1.0, 1.25, 2.0])), int(rng.choice([0, 1, 2])),
+                      int(rng.choice([0, 1, 2])), bool(rng.integers(0, 2))))
+    return cases
+
+
+@pytest.mark.parametrize("wl,cf,policy,path,fused", _soak_cases(), ids=[c[0].name for c in _soak_cases()])
+def test_layer_random_configurations_against_oracle(wl, cf, policy, path, fused):
+    """Random shape x tile policy x dispatch path x combine form, on a workspace whose scratch
+    starts as 0xFF bytes: indices bit-exact, `out` within tolerance of the oracle."""
+    cap = moe.capacity_for(cf, wl.T, wl.k, wl.E) if cf else 0
+    shape = moe.Shape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, R=wl.R, n_shared=wl.n_shared, capacity=cap)
+    dv = moe_synth.device_inputs(wl)
+    old = (moe.set_gemm_policy(policy), moe.set_dispatch_path(path), moe.set_fused_combine(fused))
+    try:
+        layer = moe.MoELayer(shape, dv["w13"], dv["w2"], dv.get("w13s"), dv.get("w2s"))
+        layer.ws[256:].fill_(0xFF)
+        outs = layer(dv["logits"], dv["x"])
+        assert moe.get_status(layer.ws) == 0
+    finally:
+        moe.set_gemm_policy(old[0])
+        moe.set_dispatch_path(old[1])
+        moe.set_fused_combine(old[2])
+    res = oracle.layer(moe_synth.host_x(wl), moe_synth.host_logits(wl), moe_synth.host_w13(wl),
+                       moe_synth.host_w2(wl), wl.k, wl.R, moe_synth.host_w13s(wl) if wl.n_shared else None,
+                       moe_synth.host_w2s(wl) if wl.n_shared else None, capacity=cap)
+    assert np.array_equal(np_i32(outs["topk_idx"]), res["topk_idx"])
+    for n in ("expert_counts", "expert_offsets", "rank_counts", "rank_offsets", "row_src", "assign_row"):
+        assert np.array_equal(np_i32(outs[n]), res[n]), n
+    close(f64(bits(outs["out"])), res["out"], f"out {wl.name}")
