@@ -440,6 +440,7 @@ def run_gpu(args, wl, rank, world, local_rank):
                    "dropped_fraction": 1.0 - sum(counts) / float(wl.T * wl.k) if wl.T else 0.0,
                    "experts_active": work["_n_act"], "imbalance_rank_expert": imbalance,
                    "expert_counts": counts,
+                   "ms_per_step_median": statistics.median(per_step),
                    "layer_roofline_frac": t_roof / (max_ms / args.steps / 1e3),
                    "layer_roofline_frac_nominal": t_roof_nominal / (max_ms / args.steps / 1e3),
                    "per_step_ms": {n: round(v, 4) for n, v in kern_ms.items()},
