@@ -149,6 +149,17 @@ def max_over_ranks(local_value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def sum_over_ranks(local_value: int, world: int, device=None) -> int:
+    """All ranks' counts added up (the whole job's); identity at world = 1."""
+    if world <= 1:
+        return int(local_value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([int(local_value)], dtype=torch.int64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return int(t.item())
+
+
 def aggregate_throughput(tokens_per_rank: int, steps: int, world: int, max_seconds: float) -> float:
     """Whole-job tokens/s: all ranks' tokens over the slowest rank's timed region (weak scaling)."""
     return world * tokens_per_rank * steps / max_seconds
@@ -361,7 +372,8 @@ def run_gpu(args, wl, rank, world, local_rank):
             layer_step()
             events[i][1].record(stream)
         torch.cuda.synchronize(dev)
-    gpu_launches = moe.kernel_launches() - launches0  # the library's own count of its kernel launches
+    # the library's own count of its kernel launches, over all ranks
+    gpu_launches = sum_over_ranks(moe.kernel_launches() - launches0, world, dev)
     if world > 1:
         dist.barrier()
     per_step = [a.elapsed_time(b) for a, b in events]
@@ -632,7 +644,7 @@ def run_gpu_ep(args, wl, rank, world, local_rank):
         layer(dv["logits"], dv["x"])
         evs[i][1].record()
     torch.cuda.synchronize(dev)
-    gpu_launches = moe.kernel_launches() - launches0
+    gpu_launches = sum_over_ranks(moe.kernel_launches() - launches0, world, dev)
     status = layer.status()
     local_ms = sum(a.elapsed_time(b) for a, b in evs)
     max_ms = max_over_ranks(local_ms, world, dev)
@@ -761,7 +773,9 @@ def rank_check(args, rank, world):
     dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
     try:
         mx = max_over_ranks(100.0 * (rank + 1), world)
-        mine = {"rank": rank, "world": world, "gpus": args.gpus, "max_ms": mx, "seed": replica_seed(0, rank)}
+        launches = sum_over_ranks(5 * (rank + 1), world)
+        mine = {"rank": rank, "world": world, "gpus": args.gpus, "max_ms": mx, "launches_all_ranks": launches,
+                "seed": replica_seed(0, rank)}
         every = [None] * world
         dist.all_gather_object(every, mine)
         if rank == 0:  # one line for all ranks (the ranks share one output stream)

@@ -87,6 +87,7 @@ def test_gpus_flag_launches_that_many_ranks():
     for x in lines:
         assert x["world"] == 2 and x["gpus"] == 2
         assert x["max_ms"] == 200.0                # the slower rank's value, on every rank
+        assert x["launches_all_ranks"] == 5 + 10   # every rank's count added up, on every rank
         assert x["seed"] == x["rank"]
 
 
