@@ -419,9 +419,11 @@ uint64_t moe_kernel_launches(void);
  *   0 (default) = one pass when T*k <= 16384, the two-kernel path otherwise;
  *   1 = two kernels: a histogram kernel whose last CTA scans the per-chunk counts,
  *       then the permute kernel;
- *   2 = one pass wherever it applies: a single kernel in which every CTA counts all
- *       T*k expert ids itself (its reads grow with T*k), ranks its own contiguous
- *       range of assignments and copies their rows.
+ *   2 = one pass wherever it applies: a single kernel (one CTA per SM) in which
+ *       every CTA counts all T*k expert ids itself (its reads grow with T*k), ranks
+ *       its own contiguous range of assignments and copies their rows; it applies
+ *       while one CTA's range holds at most 1024 assignments (about T*k / SMs plus
+ *       two tokens' worth), else the two-kernel path runs.
  * The one-pass kernel needs none of the workspace's scratch besides the status
  * word; moe_layer with the combine folded into the down GEMM always takes the
  * two-kernel path. Process-wide, for calls made after this one. Returns the
