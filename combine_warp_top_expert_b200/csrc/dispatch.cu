@@ -257,11 +257,12 @@ __global__ void __launch_bounds__(kScanThreads) dispatch_empty_kernel(int E, int
  * offset, the counts before its range the rank of its first assignment to each
  * expert; warp 0 then ranks the CTA's own assignments in order (the same stable
  * order as the two-kernel path, so the same rows). Every CTA derives the same totals
- * from the same ids; CTA 0 writes them out. The first item's row vectors are loaded
- * before the counting (before pdl_wait when early_x: x then comes from before the
- * kernel this one follows). */
+ * from the same ids; CTA 0 writes them out. The first item's row vectors (U per lane:
+ * a whole 256-vector slice at U = 8) are loaded before the counting (before pdl_wait
+ * when early_x: x then comes from before the kernel this one follows), so that part
+ * of the read overlaps the count. */
 template <int U>
-__global__ void __launch_bounds__(kOnePassThreads, 2) dispatch_onepass_kernel(
+__global__ void __launch_bounds__(kOnePassThreads, 1) dispatch_onepass_kernel(
     const uint16_t* __restrict__ x, const int32_t* __restrict__ topk_idx, int64_t T, int d, int E, int R, int k,
     int32_t cap, int64_t ipc, int slices, int vps, int32_t* expert_counts, int32_t* expert_offsets,
     int32_t* rank_counts, int32_t* rank_offsets, float* imbalance, int32_t* __restrict__ row_src,
@@ -608,7 +609,7 @@ cudaError_t launch_dispatch(const moe_shape_t& s, const WsLayout& L, uint8_t* ws
     const OnePass op = onepass_plan(s, x_perm == nullptr);
     if (op.use) {
       const size_t osmem = (size_t)(2 * kOnePassWarps * s.E + kOnePassMaxLocal) * sizeof(int32_t);
-      return launch_kernel(dispatch_onepass_kernel<4>, dim3((unsigned)op.blocks), dim3(kOnePassThreads), osmem,
+      return launch_kernel(dispatch_onepass_kernel<8>, dim3((unsigned)op.blocks), dim3(kOnePassThreads), osmem,
                            stream, 1, x, topk_idx, (int64_t)s.T, s.d, s.E, s.R, s.k, cap, op.ipc, op.slices, op.vps,
                            expert_counts, expert_offsets, rank_counts, rank_offsets, imbalance, row_src, assign_row,
                            x_perm, status, early_x ? 1 : 0);
